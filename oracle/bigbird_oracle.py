@@ -1,0 +1,230 @@
+"""fp64 CPU oracle for BigBird ITC block-sparse attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only the tests, the smoke check and the CPU-baseline leg
+of the benchmark do.  It shares no code with the CUDA library.
+
+What it computes, and where the pages state it
+----------------------------------------------
+Sources (web pages; titles and sections):
+
+* [GC] "models 仓库中的 BigBird：线性复杂度稀疏注意力与长序列训练的完整实践"
+  (blog.gitcode.com), section "BigBird：从二次方注意力到线性稀疏注意力":
+  the three-part pattern (banded window of 3 blocks around the query block,
+  first and last blocks global, num_rand_blocks random blocks that are not
+  adjacent), the five segments first / second / middle / second_last / last,
+  and masked positions receiving a -10000 offset before the softmax.
+* [GC] section "随机块掩码是如何生成的": random blocks are drawn per head from
+  the block ids without the first and last block, excluding the row's own
+  window; the blocked key mask is the [B, L] mask reshaped to
+  [B, L/bs, bs].
+* [XZ] "Big Bird: Transformers for Longer Sequences" paper card
+  (ai-papers.xuzou.cn), section "方法适配": queries/keys are blockified and the
+  attended block budget per query block is constant, so work is linear in L.
+
+Readings taken where the pages are silent (each listed in the design doc):
+
+* The attended set A(i) of query block i is a SET of key blocks: rows 0 and
+  nb-1 (global) attend every block; every other row attends
+  {i-1, i, i+1} U {0, nb-1} U rand[h, i, :r_eff], each block once.  The
+  "second" and "second_last" segments exist because the window of rows 1
+  and nb-2 overlaps a global block; union means no double counting.
+* score s_tu = scale * <q_t, k_u> + (key_mask[b, u] ? 0 : mask_value),
+  scale = 1/sqrt(d) by default, mask_value = -10000 by default.  The scale is
+  applied before the offset; the offset is not scaled.  Blocks outside A(i)
+  are absent (as if -inf), masked keys inside A(i) get the finite offset.
+* lse_t = ln sum_u exp(s_tu) over the attended keys (natural log).
+* The key mask is key-side only: query rows of padding are computed like
+  any other row.
+* The random table follows this library's own specification (the pages'
+  NumPy stream is not given): per head h and middle row i, the candidates are
+  the ascending block ids j in [1, nb-2] with |j - i| > 1; a SplitMix64
+  stream (Steele, Lea and Flood, "Fast splittable pseudorandom number
+  generators", OOPSLA 2014) is seeded with seed XOR ((h << 32) | i); a partial
+  Fisher-Yates shuffle draws r_eff = min(r, |cand|) of them; the chosen ids
+  are written sorted ascending, unused slots and rows 0 and nb-1 hold -1.
+
+The backward pass is the gradient of the forward's definition (the pages do
+not spell it out; the pages' layer trains with autodiff and recomputation):
+D_t = <dO_t, o_t>, dS_tu = p_tu (<dO_t, v_u> - D_t), dq_t = scale sum_u
+dS_tu k_u, dk_u = scale sum_t dS_tu q_t, dv_u = sum_t p_tu dO_t.
+
+Pins: tests/test_oracle.py checks this module against brute-force dense
+masked softmax attention, torch fp64 autograd, finite differences, library
+SDPA on the shapes where the pattern is dense, a closed-form adjacency
+read-out and invariants; tests/test_rand_table.py checks the generator
+against the published SplitMix64 outputs and the table's defining
+properties.
+"""
+
+import math
+
+import numpy as np
+
+_MASK64 = (1 << 64) - 1
+# SplitMix64 constants from the published generator (Steele, Lea and Flood
+# 2014; the public-domain reference code by S. Vigna): golden-ratio
+# increment and the two multipliers of the output mix.
+_SM64_GAMMA = 0x9E3779B97F4A7C15
+_SM64_MUL1 = 0xBF58476D1CE4E5B9
+_SM64_MUL2 = 0x94D049BB133111EB
+
+DEFAULT_MASK_VALUE = -10000.0
+
+
+class SplitMix64:
+    """SplitMix64 stream: advance the state by the golden gamma, then mix."""
+
+    def __init__(self, state):
+        self.state = int(state) & _MASK64
+
+    def next(self):
+        self.state = (self.state + _SM64_GAMMA) & _MASK64
+        z = self.state
+        z = ((z ^ (z >> 30)) * _SM64_MUL1) & _MASK64
+        z = ((z ^ (z >> 27)) * _SM64_MUL2) & _MASK64
+        return z ^ (z >> 31)
+
+
+def random_candidates(i, num_blocks):
+    """Block ids a middle row i may draw at random ([GC] 随机块掩码是如何生成的):
+    the middle blocks [1, nb-2] (first and last dropped) minus the row's own
+    window {i-1, i, i+1}, ascending."""
+    return [j for j in range(1, num_blocks - 1) if abs(j - i) > 1]
+
+
+def rand_table(seed, heads, num_blocks, r):
+    """int32 [heads, num_blocks, r] random block table (spec in module doc)."""
+    if heads < 0 or num_blocks < 0 or r < 0:
+        raise ValueError("negative size")
+    table = np.full((heads, num_blocks, r), -1, dtype=np.int32)
+    for h in range(heads):
+        for i in range(1, num_blocks - 1):
+            cand = random_candidates(i, num_blocks)
+            r_eff = min(r, len(cand))
+            rng = SplitMix64((int(seed) ^ ((h << 32) | i)) & _MASK64)
+            for kk in range(r_eff):
+                u = rng.next()
+                t = kk + u % (len(cand) - kk)
+                cand[kk], cand[t] = cand[t], cand[kk]
+            table[h, i, :r_eff] = sorted(cand[:r_eff])
+    return table
+
+
+def attended_blocks(i, num_blocks, rand_row):
+    """Sorted set A(i) of key blocks query block i attends ([GC] 从二次方注意力
+    到线性稀疏注意力; union reading for rows 1 and nb-2)."""
+    if i == 0 or i == num_blocks - 1:
+        return list(range(num_blocks))
+    s = {i - 1, i, i + 1, 0, num_blocks - 1}
+    s.update(int(j) for j in rand_row if j >= 0)
+    return sorted(j for j in s if 0 <= j < num_blocks)
+
+
+def _prep(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def _key_offsets(key_mask, B, L, mask_value):
+    """Additive offset per key: 0 where attended, mask_value where masked."""
+    if key_mask is None:
+        return np.zeros((B, L), dtype=np.float64)
+    km = np.asarray(key_mask).reshape(B, L).astype(bool)
+    return np.where(km, 0.0, float(mask_value))
+
+
+def _token_cols(blocks, bs):
+    return np.concatenate([np.arange(j * bs, (j + 1) * bs) for j in blocks])
+
+
+def block_probs(q, k, key_mask, table, block_size, b, h, i, scale=None,
+                mask_value=DEFAULT_MASK_VALUE):
+    """Softmax probabilities of query block i of (b, h).
+
+    Returns (key token indices, p [bs, n_keys], lse [bs]).  Softmax is taken
+    in fp64 with the row maximum subtracted."""
+    q = _prep(q)
+    k = _prep(k)
+    B, H, L, d = q.shape
+    bs = block_size
+    nb = L // bs
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    off = _key_offsets(key_mask, B, L, mask_value)
+    cols = _token_cols(attended_blocks(i, nb, table[h, i]), bs)
+    qi = q[b, h, i * bs:(i + 1) * bs]
+    s = scale * (qi @ k[b, h, cols].T) + off[b, cols][None, :]
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = e.sum(axis=1, keepdims=True)
+    return cols, e / z, (m + np.log(z))[:, 0]
+
+
+def forward(q, k, v, key_mask, table, block_size, scale=None,
+            mask_value=DEFAULT_MASK_VALUE):
+    """Block-sparse attention forward: (o [B,H,L,d], lse [B,H,L]) in fp64.
+
+    q, k, v: [B, H, L, d] (any float dtype, read as fp64); key_mask: None or
+    [B, L] with nonzero = attend; table: int [H, nb, r]."""
+    q = _prep(q)
+    k = _prep(k)
+    v = _prep(v)
+    B, H, L, d = q.shape
+    bs = block_size
+    if L % bs:
+        raise ValueError("L must be a multiple of block_size")
+    nb = L // bs
+    o = np.zeros((B, H, L, d))
+    lse = np.zeros((B, H, L))
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                cols, p, l = block_probs(q, k, key_mask, table, bs, b, h, i,
+                                         scale, mask_value)
+                o[b, h, i * bs:(i + 1) * bs] = p @ v[b, h, cols]
+                lse[b, h, i * bs:(i + 1) * bs] = l
+    return o, lse
+
+
+def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
+             mask_value=DEFAULT_MASK_VALUE):
+    """Gradient of forward's o with respect to q, k, v for upstream dout.
+
+    Returns (dq, dk, dv), each [B, H, L, d] fp64.  Probabilities and o are
+    recomputed here from the definition, in fp64."""
+    q = _prep(q)
+    k = _prep(k)
+    v = _prep(v)
+    dout = _prep(dout)
+    B, H, L, d = q.shape
+    bs = block_size
+    nb = L // bs
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nb):
+                cols, p, _ = block_probs(q, k, key_mask, table, bs, b, h, i,
+                                         scale, mask_value)
+                rows = slice(i * bs, (i + 1) * bs)
+                vc = v[b, h, cols]
+                kc = k[b, h, cols]
+                do_i = dout[b, h, rows]
+                o_i = p @ vc
+                D = (do_i * o_i).sum(axis=1)
+                dP = do_i @ vc.T
+                dS = p * (dP - D[:, None])
+                dq[b, h, rows] = scale * (dS @ kc)
+                # cols holds each key token once, so fancy-index += is exact.
+                dk[b, h, cols] += scale * (dS.T @ q[b, h, rows])
+                dv[b, h, cols] += p.T @ do_i
+    return dq, dk, dv
+
+
+def pair_count(num_blocks, table_h):
+    """Number of attended (query block, key block) pairs for one head."""
+    return sum(len(attended_blocks(i, num_blocks, table_h[i]))
+               for i in range(num_blocks))

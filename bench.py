@@ -1,0 +1,545 @@
+"""Benchmark of the block-sparse attention hot path (forward + backward).
+
+python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                [--workload NAME]
+
+One step = one forward + backward pass of the whole hot path over one batch
+of the named synthetic workload (default: BigBird-large attention layer at
+L=4096: B=4, H=16, block 64, d=64, r=3, bf16).  For N > 1 (torchrun) every
+rank runs its own batch (weak scaling: batches are independent, there is no
+collective in the data path); the timed region is bracketed by a barrier and
+a synchronize on both sides and the slowest rank's device time is reported.
+
+Rank 0 prints one JSON line.  `value` is tokens/s over all ranks with inputs
+resident in HBM, timed with CUDA events; between timed steps the L2 is
+flushed by writing a 256 MiB buffer outside the timed events.  `e2e` is the
+same metric through the public API with pinned host buffers: host->device
+copies of the inputs (and the random table build), the two calls, and
+device->host copies of all results inside the timed region.
+"""
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_bwd_b200 import synth  # noqa: E402
+
+METRIC = ("block-sparse attn fwd+bwd tokens/s and attended TFLOP/s at "
+          "L=4096 (% bf16 TC peak)")
+DEFAULT_WORKLOAD = "large_train_l4096"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+# DRAM bytes per launch from one ncu capture, keyed by kernel name, with the
+# sha256 of the source file the kernel was built from when captured.  A
+# mismatch (the kernel changed since) reports traffic as null.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args()
+
+
+def workload(name):
+    if name in synth.WORKLOADS:
+        return dict(synth.WORKLOADS[name])
+    if name.startswith("sweep_"):  # sweep_L_bs_r
+        _, L, bs, r = name.split("_")
+        return synth.sweep_point(int(L), int(bs), int(r))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def pairs_per_head(nb, table_h):
+    """Attended (query block, key block) pairs of one head: nb for each of
+    the two global rows, and for middle rows the size of the set
+    {0, nb-1, i-1, i, i+1} U rand(i)."""
+    total = 0
+    for i in range(nb):
+        if i == 0 or i == nb - 1:
+            total += nb
+        else:
+            s = {0, nb - 1, i - 1, i, i + 1}
+            s.update(int(j) for j in table_h[i] if 0 <= j < nb)
+            total += len(s)
+    return total
+
+
+def load_peaks():
+    if os.path.exists(PEAKS_FILE):
+        with open(PEAKS_FILE) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the run."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}",
+                 f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0],
+                                                   "%Y/%m/%d %H:%M:%S"))
+                    rows.append((ts, float(parts[2]), float(parts[3]),
+                                 parts[6:10]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        inside = [r for r in rows if t0 - 1 <= r[0] <= t1 + 1] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[k] for r in inside
+                          for k, v in enumerate(r[3]) if v == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+def smi_id(local):
+    """nvidia-smi --id for this rank's device (UUID survives remapping by
+    CUDA_VISIBLE_DEVICES)."""
+    try:
+        u = str(torch.cuda.get_device_properties(local).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(local)
+
+
+def init_dist(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        if args.impl == "reference":
+            return world, rank, local  # rank 0 alone runs the CPU oracle
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl",
+                                timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def algorithmic(cfg, pairs_total):
+    """Algorithmic FLOPs and bytes per launch of each kernel kind."""
+    B, H, L, d, bs = cfg["B"], cfg["H"], cfg["L"], cfg["d"], cfg["block_size"]
+    e = 2 if cfg["dtype"] == "bf16" else 4
+    rows = B * H * L
+    elems = rows * d
+    unit = pairs_total * bs * bs * d  # one bs x bs x d contraction per pair
+    return {
+        "fwd": (4 * unit, 4 * elems * e + 4 * rows),
+        "bwd_pre": (0, 2 * elems * e + 4 * rows),
+        "csr_build": (0, 0),
+        "dq": (6 * unit, 5 * elems * e + 8 * rows),
+        "dkdv": (8 * unit, 6 * elems * e + 8 * rows),
+    }
+
+
+def kernel_kind(name):
+    """Which algorithmic figure a launch name counts against."""
+    for kind in ("dkdv", "dq", "fwd", "bwd_pre", "csr_build"):
+        if kind in name:
+            return kind
+    return None
+
+
+def kernel_bound(name):
+    if name.startswith("simt_"):
+        return "alu"      # fp32 FFMA on the CUDA cores
+    if name.startswith("tc_"):
+        return "tensor"   # tcgen05 contractions
+    return "hbm"
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_long_bwd_b200 import binding as bb
+
+    cfg = workload(args.workload)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    backward = cfg["passes"] == "fwd+bwd"
+    dt = synth.torch_dtype(cfg["dtype"])
+    B, H, L, bs, r = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"], cfg["r"]
+    nb = L // bs
+
+    inp = synth.make_inputs(cfg, with_grad=backward)
+    att = bb.Attention(B, H, L, bs, r, dt, d=cfg["d"], seed=synth.TABLE_SEED,
+                       device=dev)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    g = inp["dout"].to(dev) if backward else None
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    n_fwd = bb.bb_attn_launch_count(att.desc, 0)
+    n_bwd = bb.bb_attn_launch_count(att.desc, 1) if backward else 0
+    names = ([bb.bb_attn_launch_name(att.desc, 0, i) for i in range(n_fwd)]
+             + [bb.bb_attn_launch_name(att.desc, 1, i) for i in range(n_bwd)])
+    stream = torch.cuda.current_stream()
+
+    def step(ev_f=None, ev_b=None):
+        att.forward(q, k, v, km, out=out, lse=lse, stream=stream, events=ev_f)
+        if backward:
+            att.backward(q, k, v, out, lse, g, km, dq=dq, dk=dk, dv=dv,
+                         stream=stream, events=ev_b)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = bb.bb_attn_check_status(att.ws_fwd)
+    if st != 0:
+        raise SystemExit(f"forward status {bb.bb_status_str(st)}")
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)  # creates the underlying CUDA event
+        return evs
+
+    K = args.steps
+    evf = [new_events(n_fwd + 1) for _ in range(K)]
+    evb = [new_events(n_bwd + 1) for _ in range(K)] if backward else None
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(smi_id(local))
+    sampler.start()
+    time.sleep(0.3)
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for s in range(K):
+        flush.fill_(s & 0xFF)  # outside the step's events: evicts L2
+        step(evf[s], evb[s] if backward else None)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop(t0, t1)
+
+    per_kernel = {n: [] for n in names}
+    step_ms = []
+    for s in range(K):
+        tot = 0.0
+        evs = [(evf[s], names[:n_fwd])]
+        if backward:
+            evs.append((evb[s], names[n_fwd:]))
+        for ev, nm in evs:
+            for i, n in enumerate(nm):
+                t = ev[i].elapsed_time(ev[i + 1])
+                per_kernel[n].append(t)
+            tot += ev[0].elapsed_time(ev[-1])
+        step_ms.append(tot)
+    total_ms = sum(step_ms)
+    if world > 1:
+        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    ms_per_step = total_ms / K
+    tokens = B * L * world
+    value = tokens * K / (total_ms / 1e3)
+
+    # Attended FLOPs over the pattern's pairs (masked keys included).
+    pairs = sum(pairs_per_head(nb, att.table_host[h].numpy())
+                for h in range(H)) * B
+    alg = algorithmic(cfg, pairs)
+    fwd_flops = 4 * pairs * bs * bs * cfg["d"]
+    bwd_flops = 10 * pairs * bs * bs * cfg["d"] if backward else 0
+    avg = {n: sum(v_) / len(v_) for n, v_ in per_kernel.items()}
+    share = {n: sum(per_kernel[n]) / sum(step_ms) for n in names}
+    dom = max(names, key=lambda n: sum(per_kernel[n]))
+    peaks, peak_src = load_peaks()
+    fl, by = alg.get(kernel_kind(dom), (0, 0))
+    dur_s = avg[dom] / 1e3
+    bound = kernel_bound(dom)
+    if bound == "tensor":
+        unit, achieved = "TFLOP/s", fl / dur_s / 1e12
+        peak, how = peaks["bf16_tflops"], "bf16 dense, burst"
+    elif bound == "alu":
+        unit, achieved = "TFLOP/s", fl / dur_s / 1e12
+        # fp32 FFMA: 148 SMs x 128 lanes x 2 FLOP per clock at max SM clock.
+        peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        how = "fp32 FFMA, derived from unit counts and max clock"
+    else:
+        unit, achieved = "GB/s", by / dur_s / 1e9
+        peak, how = peaks["hbm_gbs"], "HBM copy"
+    traffic = None
+    tr = NCU_TRAFFIC.get(dom)
+    if tr is not None and tr[1] == src_hash(os.path.join(
+            ROOT, "block_sparse_long_bwd_b200", "csrc", tr[2])):
+        traffic = tr[0]
+    roofline = {"bound": bound, "achieved": round(achieved, 2),
+                "peak": round(peak, 1), "unit": unit,
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": dom, "peak_source": f"{peak_src}: {how}"}
+    kernels = {n: {"avg_ms": round(avg[n], 5), "share": round(share[n], 4),
+                   "launches": len(per_kernel[n]),
+                   "tflops": (round(alg[kernel_kind(n)][0] / (avg[n] / 1e3)
+                                    / 1e12, 2)
+                              if alg.get(kernel_kind(n), (0, 0))[0] else None),
+                   "gbs": (round(alg[kernel_kind(n)][1] / (avg[n] / 1e3)
+                                 / 1e9, 1)
+                           if alg.get(kernel_kind(n), (0, 0))[1] else None)}
+               for n in names}
+
+    e2e = run_e2e(args, cfg, att, inp, dev, backward, world)
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": cfg["dtype"],
+        "data": "synthetic (seeded N(0,1) inputs, no dataset)",
+        "config": {"workload": args.workload, "B": B, "H": H, "L": L,
+                   "block_size": bs, "d": cfg["d"], "r": r,
+                   "mask": cfg["mask"], "passes": cfg["passes"],
+                   "global_batch": B * world, "seq_len": L,
+                   "parallelism": f"replicas x{world} (independent batches)",
+                   "l2": "flushed between steps (256 MiB write, untimed)"},
+        "attended_tflops": {
+            "fwd": round(fwd_flops * world / (sum(sum(per_kernel[n]) for n in names[:n_fwd]) / K / 1e3) / 1e12, 2),
+            "fwd_bwd": round((fwd_flops + bwd_flops) * world / (ms_per_step / 1e3) / 1e12, 2),
+            "convention": "4*bs^2*d per attended block pair fwd, 10*bs^2*d bwd",
+            "pairs": pairs},
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": K * (n_fwd + n_bwd),
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if rank == 0:
+        result["cpu_baseline"] = cpu_baseline(cfg, att.table_host.numpy(),
+                                              backward, budget_s=12.0)
+        print(json.dumps(result), flush=True)
+
+
+def run_e2e(args, cfg, att, inp, dev, backward, world):
+    """Same metric through the public API from pinned host buffers."""
+    from block_sparse_long_bwd_b200 import binding as bb
+
+    B, H, L, bs, r = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"], cfg["r"]
+    names = ["q", "k", "v"] + (["dout"] if backward else [])
+    host = {n: inp[n].pin_memory() for n in names}
+    km_h = None if inp["key_mask"] is None else inp["key_mask"].pin_memory()
+    devt = {n: torch.empty_like(host[n], device=dev) for n in names}
+    km_d = None if km_h is None else torch.empty_like(km_h, device=dev)
+    tab_d = torch.empty((H, L // bs, r), dtype=torch.int32, device=dev)
+    outs = ["out", "lse"] + (["dq", "dk", "dv"] if backward else [])
+    res_h = {"out": torch.empty_like(host["q"]).pin_memory(),
+             "lse": torch.empty((B, H, L), dtype=torch.float32).pin_memory()}
+    if backward:
+        for n in ("dq", "dk", "dv"):
+            res_h[n] = torch.empty_like(host["q"]).pin_memory()
+    stream = torch.cuda.current_stream()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    h2d += 0 if km_h is None else km_h.numel()
+    h2d += tab_d.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in res_h.values())
+
+    def step():
+        tab = bb.bb_rand_attn_build(synth.TABLE_SEED, H, L // bs, r)
+        tab_d.copy_(tab.pin_memory(), non_blocking=True)
+        for n in names:
+            devt[n].copy_(host[n], non_blocking=True)
+        if km_h is not None:
+            km_d.copy_(km_h, non_blocking=True)
+        o = torch.empty_like(devt["q"])
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+        bb.bb_attn_fwd(att.desc, devt["q"], devt["k"], devt["v"], km_d,
+                       tab_d, o, lse, att.ws_fwd, stream)
+        res = {"out": o, "lse": lse}
+        if backward:
+            dq, dk, dv = (torch.empty_like(devt["q"]) for _ in range(3))
+            bb.bb_attn_bwd(att.desc, devt["q"], devt["k"], devt["v"], o, lse,
+                           devt["dout"], km_d, tab_d, dq, dk, dv, att.ws_bwd,
+                           stream)
+            res.update(dq=dq, dk=dk, dv=dv)
+        for n in outs:
+            res_h[n].copy_(res[n], non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(2):
+        step()
+    n = max(1, args.e2e_steps)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(n):
+        step()
+    torch.cuda.synchronize()
+    el = time.perf_counter() - t0
+    if world > 1:
+        tt = torch.tensor([el], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        el = float(tt.item())
+    return {"value": round(B * L * world * n / el, 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "steps": n, "timing": "host wall clock around synchronised steps"}
+
+
+def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None):
+    """The fp64 oracle, as it stands, on (b, h) slices of the workload until
+    the time budget is spent; scaled to tokens/s of the whole workload
+    (each slice is 1/(B*H) of it)."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()),
+                    default=1)
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    B, H, L, bs = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"]
+    inp = synth.make_inputs(cfg, with_grad=backward, batch_slice=slice(0, 1))
+    f = lambda x, h: x[:, h:h + 1].double().numpy()
+    km = None if inp["key_mask"] is None else inp["key_mask"].numpy()
+    done, t_used = 0, 0.0
+    for h in range(H):
+        t0 = time.perf_counter()
+        oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), km,
+                       table[h:h + 1], bs)
+        if backward:
+            oracle.backward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
+                            f(inp["dout"], h), km, table[h:h + 1], bs)
+        t_used += time.perf_counter() - t0
+        done += 1
+        if t_used >= budget_s or (max_slices and done >= max_slices):
+            break
+    value = (L / H) * done / t_used  # tokens/s of the whole workload
+    return {"value": round(value, 2), "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{done} (b,h) slice(s) of b=0 at full L={L}, "
+                      f"{'fwd+bwd' if backward else 'fwd'}, {t_used:.1f} s; "
+                      f"scaled by B*H={B * H}"}
+
+
+def run_reference(args, world, rank):
+    """The oracle (the only reference implementation for this method) timed
+    on the host cores, one (b, h) slice of the workload per step."""
+    if rank != 0:
+        return
+    import oracle
+    cfg = workload(args.workload)
+    backward = cfg["passes"] == "fwd+bwd"
+    B, H, L, bs, r = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"], cfg["r"]
+    table = oracle.rand_table(synth.TABLE_SEED, H, L // bs, r)
+    inp = synth.make_inputs(cfg, with_grad=backward, batch_slice=slice(0, 1))
+    km = None if inp["key_mask"] is None else inp["key_mask"].numpy()
+    f = lambda x, h: x[:, h:h + 1].double().numpy()
+
+    def step(s):
+        h = s % H
+        oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), km,
+                       table[h:h + 1], bs)
+        if backward:
+            oracle.backward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
+                            f(inp["dout"], h), km, table[h:h + 1], bs)
+
+    for s in range(args.warmup):
+        step(s)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        step(s)
+    el = time.perf_counter() - t0
+    value = (L / H) * args.steps / el
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()),
+                    default=1)
+    except Exception:
+        cores = len(os.sched_getaffinity(0))
+    sample = (f"one (b,h) slice of b=0 per step at full L={L}, "
+              f"{'fwd+bwd' if backward else 'fwd'}; scaled by B*H={B * H}")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 2),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs)",
+        "config": {"workload": args.workload, "B": B, "H": H, "L": L,
+                   "block_size": bs, "d": cfg["d"], "r": r,
+                   "global_batch": B, "seq_len": L},
+        "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
+                         "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = init_dist(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,255 @@
+"""Thin ctypes binding of libbbattn.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of the method: tensors are checked for device, dtype and
+contiguity, their data pointers and sizes are passed through, and a non-OK
+status raises BBError.  The library is loaded on first use; if it is missing
+the call raises (there is no fallback of any kind).
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbbattn.so")
+
+BB_OK = 0
+BB_F32 = 0
+BB_BF16 = 1
+STATUS = {0: "BB_OK", -1: "BB_ERR_INVALID", -2: "BB_ERR_UNSUPPORTED",
+          -3: "BB_ERR_CUDA", -4: "BB_ERR_WORKSPACE", -5: "BB_ERR_TIMEOUT",
+          -6: "BB_ERR_BAD_TABLE"}
+
+
+class BBError(RuntimeError):
+    def __init__(self, code, what):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} "
+                         f"({bb_status_str(code)})")
+
+
+class bb_attn_desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
+                ("d", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("r", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("scale", ctypes.c_float), ("mask_value", ctypes.c_float)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+
+
+def lib():
+    """The loaded library (raises OSError if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m block_sparse_long_bwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.bb_abi_version.restype = ctypes.c_int
+        L.bb_status_str.argtypes = [ctypes.c_int]
+        L.bb_status_str.restype = ctypes.c_char_p
+        L.bb_rand_attn_build.argtypes = [ctypes.c_uint64, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, _P]
+        L.bb_rand_attn_build.restype = ctypes.c_int
+        L.bb_attn_workspace_size.argtypes = [
+            ctypes.POINTER(bb_attn_desc), ctypes.c_int,
+            ctypes.POINTER(ctypes.c_size_t)]
+        L.bb_attn_workspace_size.restype = ctypes.c_int
+        L.bb_attn_fwd.argtypes = [ctypes.POINTER(bb_attn_desc)] + [_P] * 8 + [
+            ctypes.c_size_t, _P]
+        L.bb_attn_fwd.restype = ctypes.c_int
+        L.bb_attn_bwd.argtypes = [ctypes.POINTER(bb_attn_desc)] + [_P] * 12 + [
+            ctypes.c_size_t, _P]
+        L.bb_attn_bwd.restype = ctypes.c_int
+        L.bb_attn_launch_count.argtypes = [ctypes.POINTER(bb_attn_desc),
+                                           ctypes.c_int,
+                                           ctypes.POINTER(ctypes.c_int)]
+        L.bb_attn_launch_count.restype = ctypes.c_int
+        L.bb_attn_launch_name.argtypes = [ctypes.POINTER(bb_attn_desc),
+                                          ctypes.c_int, ctypes.c_int,
+                                          ctypes.POINTER(ctypes.c_char_p)]
+        L.bb_attn_launch_name.restype = ctypes.c_int
+        L.bb_attn_fwd_events.argtypes = (
+            [ctypes.POINTER(bb_attn_desc)] + [_P] * 8
+            + [ctypes.c_size_t, _P, ctypes.POINTER(_P), ctypes.c_int])
+        L.bb_attn_fwd_events.restype = ctypes.c_int
+        L.bb_attn_bwd_events.argtypes = (
+            [ctypes.POINTER(bb_attn_desc)] + [_P] * 12
+            + [ctypes.c_size_t, _P, ctypes.POINTER(_P), ctypes.c_int])
+        L.bb_attn_bwd_events.restype = ctypes.c_int
+        L.bb_attn_check_status.argtypes = [_P, _P]
+        L.bb_attn_check_status.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def bb_status_str(code):
+    return lib().bb_status_str(int(code)).decode()
+
+
+def bb_abi_version():
+    return lib().bb_abi_version()
+
+
+def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0):
+    if isinstance(dtype, torch.dtype):
+        dtype = {torch.float32: BB_F32, torch.bfloat16: BB_BF16}[dtype]
+    return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value)
+
+
+def _check(code, what):
+    if code != BB_OK:
+        raise BBError(code, what)
+
+
+def bb_rand_attn_build(seed, heads, num_blocks, r):
+    """int32 CPU tensor [heads, num_blocks, r] (see include/bb_attn.h)."""
+    out = torch.empty((heads, num_blocks, r), dtype=torch.int32)
+    _check(lib().bb_rand_attn_build(seed, heads, num_blocks, r,
+                                    out.data_ptr() if out.numel() else None),
+           "bb_rand_attn_build")
+    return out
+
+
+def bb_attn_workspace_size(desc, pass_):
+    n = ctypes.c_size_t(0)
+    _check(lib().bb_attn_workspace_size(ctypes.byref(desc), pass_,
+                                        ctypes.byref(n)),
+           "bb_attn_workspace_size")
+    return n.value
+
+
+def bb_attn_launch_count(desc, pass_):
+    n = ctypes.c_int(0)
+    _check(lib().bb_attn_launch_count(ctypes.byref(desc), pass_,
+                                      ctypes.byref(n)),
+           "bb_attn_launch_count")
+    return n.value
+
+
+def bb_attn_launch_name(desc, pass_, index):
+    s = ctypes.c_char_p()
+    _check(lib().bb_attn_launch_name(ctypes.byref(desc), pass_, index,
+                                     ctypes.byref(s)),
+           "bb_attn_launch_name")
+    return s.value.decode()
+
+
+def _event_array(events):
+    """ctypes array of raw cudaEvent_t handles of recorded torch events."""
+    arr = (_P * len(events))()
+    for i, e in enumerate(events):
+        arr[i] = e.cuda_event
+    return arr, len(events)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream_ptr(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _cuda_tensor(t, name, dtype=None):
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}")
+
+
+def desc_for(q, block_size, r, scale=0.0, mask_value=0.0):
+    B, H, L, d = q.shape
+    return make_desc(B, H, L, d, block_size, r, q.dtype, scale, mask_value)
+
+
+def bb_attn_fwd(desc, q, k, v, key_mask, rand_idx, out, lse, workspace,
+                stream=None, events=None):
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _cuda_tensor(t, name, q.dtype)
+    _cuda_tensor(lse, "lse", torch.float32)
+    _cuda_tensor(workspace, "workspace")
+    if key_mask is not None:
+        _cuda_tensor(key_mask, "key_mask", torch.uint8)
+    if rand_idx is not None:
+        _cuda_tensor(rand_idx, "rand_idx", torch.int32)
+    args = (ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(key_mask),
+            _ptr(rand_idx), _ptr(out), _ptr(lse), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if events is None:
+        _check(lib().bb_attn_fwd(*args), "bb_attn_fwd")
+    else:
+        arr, n = _event_array(events)
+        _check(lib().bb_attn_fwd_events(*args, arr, n), "bb_attn_fwd_events")
+
+
+def bb_attn_bwd(desc, q, k, v, out, lse, dout, key_mask, rand_idx, dq, dk, dv,
+                workspace, stream=None, events=None):
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out),
+                    ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+        _cuda_tensor(t, name, q.dtype)
+    _cuda_tensor(lse, "lse", torch.float32)
+    _cuda_tensor(workspace, "workspace")
+    if key_mask is not None:
+        _cuda_tensor(key_mask, "key_mask", torch.uint8)
+    if rand_idx is not None:
+        _cuda_tensor(rand_idx, "rand_idx", torch.int32)
+    args = (ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+            _ptr(lse), _ptr(dout), _ptr(key_mask), _ptr(rand_idx), _ptr(dq),
+            _ptr(dk), _ptr(dv), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if events is None:
+        _check(lib().bb_attn_bwd(*args), "bb_attn_bwd")
+    else:
+        arr, n = _event_array(events)
+        _check(lib().bb_attn_bwd_events(*args, arr, n), "bb_attn_bwd_events")
+
+
+def bb_attn_check_status(workspace, stream=None):
+    return lib().bb_attn_check_status(_ptr(workspace), _stream_ptr(stream))
+
+
+class Attention:
+    """Convenience wrapper holding the table and workspaces for one shape.
+
+    Allocation (workspace, outputs) happens here, with torch, outside the
+    library; every call below goes straight to the C entry points."""
+
+    def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
+                 device="cuda", scale=0.0, mask_value=0.0):
+        self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
+                              mask_value)
+        self.dtype = dtype
+        nb = L // block_size
+        self.table_host = bb_rand_attn_build(seed, H, nb, r)
+        self.table = self.table_host.to(device)
+        self.ws_fwd = torch.empty(bb_attn_workspace_size(self.desc, 0),
+                                  dtype=torch.uint8, device=device)
+        self.ws_bwd = torch.empty(bb_attn_workspace_size(self.desc, 1),
+                                  dtype=torch.uint8, device=device)
+
+    def forward(self, q, k, v, key_mask=None, out=None, lse=None,
+                stream=None, events=None):
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None:
+            lse = torch.empty(q.shape[:3], dtype=torch.float32,
+                              device=q.device)
+        bb_attn_fwd(self.desc, q, k, v, key_mask, self.table, out, lse,
+                    self.ws_fwd, stream, events)
+        return out, lse
+
+    def backward(self, q, k, v, out, lse, dout, key_mask=None, dq=None,
+                 dk=None, dv=None, stream=None, events=None):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        bb_attn_bwd(self.desc, q, k, v, out, lse, dout, key_mask, self.table,
+                    dq, dk, dv, self.ws_bwd, stream, events)
+        return dq, dk, dv

@@ -1,0 +1,138 @@
+// Internal declarations shared by the host API and the kernels of
+// libbbattn.so.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/bb_attn.h"
+
+namespace bb {
+
+constexpr int kHeadDim = 64;       // d supported by this release
+constexpr int kMaxBlocks = 8192;   // nb limit (CSR builder keeps counts in smem)
+constexpr int kMaxRand = 32;       // r limit (attended list fits in smem)
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Everything a kernel needs about one call, passed by value.
+struct Problem {
+  int B, H, L, d, bs, r, nb, dtype;
+  float scale;       // resolved (never 0)
+  float mask_value;  // resolved (never 0)
+  // inputs
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;     // bwd
+  const void* dout;  // bwd
+  const float* lse;  // bwd
+  const uint8_t* key_mask;
+  const int32_t* rand_idx;
+  // outputs
+  void* out;
+  float* lse_out;
+  void* dq;
+  void* dk;
+  void* dv;
+  // workspace pieces
+  int* status;
+  float* D;          // [B*H*L] (bwd)
+  int* csr_offs;     // [H][nb+1] (bwd)
+  int* csr_list;     // [H][csr_cap] (bwd)
+  int csr_cap;
+  float* part;       // split partials (tensor-core path)
+  size_t part_floats;
+};
+
+// Upper bound of attended (query block, key block) pairs per head.
+inline int pair_cap(int nb, int r) { return nb * (7 + r) + 8; }
+
+// Workspace layout, identical for sizing and for carving.
+struct WsLayout {
+  size_t status_off, D_off, offs_off, list_off, part_off, total;
+};
+WsLayout ws_layout(const Problem& p, int pass);
+
+// Records caller-provided timing events between internal launches.
+struct EventMarks {
+  void* const* ev = nullptr;
+  int n = 0;
+  int next = 0;
+  cudaError_t mark(cudaStream_t s) {
+    if (next < n && ev && ev[next]) {
+      cudaError_t e = cudaEventRecord((cudaEvent_t)ev[next], s);
+      ++next;
+      return e;
+    }
+    ++next;
+    return cudaSuccess;
+  }
+};
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_simt_fwd(const Problem& p, cudaStream_t s);
+cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s);
+cudaError_t launch_csr_build(const Problem& p, cudaStream_t s);
+cudaError_t launch_simt_bwd(const Problem& p, cudaStream_t s, EventMarks* marks);
+
+// ---- device helpers -----------------------------------------------------
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+template <typename T>
+__device__ __forceinline__ T from_f(float x);
+template <>
+__device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Record the first non-OK status of a call (integer atomic, not a result).
+__device__ __forceinline__ void set_status(int* status, int code) {
+  atomicCAS(status, 0, code);
+}
+
+// Sorted set A(i) of key blocks for a middle query block i (0 < i < nb-1):
+// {0, i-1, i, i+1, nb-1} U rand row, each once.  Entries outside [-1, nb)
+// are ignored and flagged.  Returns the count written to out (<= 5 + r).
+__device__ __forceinline__ int middle_row_blocks(const int32_t* rand_row,
+                                                 int r, int i, int nb,
+                                                 int* out, int* status) {
+  int n = 0;
+  int base[5] = {0, i - 1, i, i + 1, nb - 1};
+  for (int a = 0; a < 5; ++a) {
+    int j = base[a];
+    bool dup = false;
+    for (int c = 0; c < n; ++c) dup |= (out[c] == j);
+    if (!dup) out[n++] = j;
+  }
+  for (int a = 0; a < r; ++a) {
+    int j = rand_row[a];
+    if (j == -1) continue;
+    if (j < 0 || j >= nb) {
+      set_status(status, BB_ERR_BAD_TABLE);
+      continue;
+    }
+    bool dup = false;
+    for (int c = 0; c < n; ++c) dup |= (out[c] == j);
+    if (!dup) out[n++] = j;
+  }
+  // insertion sort (n is small)
+  for (int a = 1; a < n; ++a) {
+    int x = out[a];
+    int c = a - 1;
+    while (c >= 0 && out[c] > x) {
+      out[c + 1] = out[c];
+      --c;
+    }
+    out[c + 1] = x;
+  }
+  return n;
+}
+
+}  // namespace bb

@@ -1,0 +1,180 @@
+/*
+ * bb_attn.h -- C ABI of libbbattn.so: BigBird ITC block-sparse attention,
+ * forward and backward, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (web page "models 仓库中的 BigBird：线性复杂度稀疏注意力与长序列
+ * 训练的完整实践", blog.gitcode.com, section "BigBird：从二次方注意力到线性稀疏
+ * 注意力"): Q, K and V are cut into blocks of block_size tokens
+ * (nb = L / block_size blocks).  The first and last blocks are global: query
+ * blocks 0 and nb-1 attend every key block, and every query block attends
+ * key blocks 0 and nb-1.  Every other query block i also attends its window
+ * {i-1, i, i+1} and the r random blocks of row i of a per-head table.  The
+ * attended set A(i) is a set (each key block once).  For key token u of an
+ * attended block the score is
+ *     s = scale * <q, k_u> + (key_mask[b][u] ? 0 : mask_value)
+ * and the row softmax over the attended keys weights V.
+ *
+ * Conventions shared by every call:
+ *  - All tensors are dense, row-major, contiguous.  Q, K, V, O, dO, dQ, dK
+ *    and dV are [B][H][L][d] in the descriptor's dtype (fp32 or bf16); the
+ *    blocked view [B][H][nb][block_size][d] of the pages is the same memory.
+ *    lse and the workspace's fp32 arrays are fp32.
+ *  - Pointers named *_host are host memory; every other pointer is device
+ *    memory of the current CUDA device.  The caller owns every buffer; the
+ *    library allocates nothing on the call path and keeps no state between
+ *    calls.  Device pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Compute
+ *    calls validate on the host, enqueue their kernels on `stream` and return
+ *    without synchronising.  Launch errors are returned; faults detected by a
+ *    kernel (a wait that ran out, a corrupt random table) are written to a
+ *    status word at the start of the workspace, read by bb_attn_check_status.
+ *  - Calls are re-entrant and thread-safe (no global mutable state); two
+ *    calls may share a workspace only if they are ordered on the GPU.
+ *  - Results are deterministic run to run: no floating-point atomics.
+ */
+#ifndef BB_ATTN_H_
+#define BB_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BB_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define BB_API __attribute__((visibility("default")))
+#else
+#define BB_API
+#endif
+
+typedef enum {
+  BB_OK = 0,
+  BB_ERR_INVALID = -1,     /* a NULL or misaligned pointer, a bad size */
+  BB_ERR_UNSUPPORTED = -2, /* valid but not built: d != 64, block_size not
+                              in {32, 64, 128}, nb > 8192, r > 32 */
+  BB_ERR_CUDA = -3,        /* a CUDA runtime call failed (launch, copy) */
+  BB_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than required */
+  BB_ERR_TIMEOUT = -5,     /* (status word) a bounded device wait ran out */
+  BB_ERR_BAD_TABLE = -6    /* (status word) a random-table entry outside
+                              [-1, nb) was found and ignored */
+} bb_status;
+
+typedef enum { BB_F32 = 0, BB_BF16 = 1 } bb_dtype;
+
+/* Problem description.  d must be 64; block_size 32, 64 or 128 and a divisor
+ * of L; r >= 0 random blocks per middle row; dtype a bb_dtype.
+ * scale == 0 selects 1/sqrt(d) (key_dim = hidden / heads, as the pages'
+ * layer sets it).  mask_value == 0 selects -10000, the pages' offset for
+ * masked positions.  The scale multiplies <q, k> before the offset is added;
+ * the offset is not scaled. */
+typedef struct {
+  int B, H, L, d, block_size, r;
+  int dtype;
+  float scale;
+  float mask_value;
+} bb_attn_desc;
+
+/* Random block table ([gitcode page] section "随机块掩码是如何生成的": per
+ * head, each middle row draws num_rand_blocks blocks among the middle blocks
+ * outside its own window).  Writes int32 out_host[heads][num_blocks][r]:
+ * rows 0 and num_blocks-1 are all -1; middle row i holds
+ * r_eff = min(r, |cand(i)|) distinct ids from cand(i) = {j in [1, nb-2] :
+ * |j - i| > 1}, sorted ascending, then -1 in the remaining slots.  The draw
+ * is this library's own specification: a SplitMix64 stream (Steele, Lea and
+ * Flood, OOPSLA 2014) seeded with seed ^ ((uint64)h << 32 | i) drives a
+ * partial Fisher-Yates shuffle of cand(i) (slot k swaps with
+ * k + u mod (|cand| - k)).  Deterministic and platform independent; host
+ * only, no CUDA call.  Returns BB_ERR_INVALID for a NULL out_host (unless the
+ * table is empty) or a negative size. */
+BB_API int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
+                       int32_t* out_host);
+
+/* Bytes of device workspace bb_attn_fwd (pass 0) or bb_attn_bwd (pass 1)
+ * needs for `desc`; written to *bytes.  Host only. */
+BB_API int bb_attn_workspace_size(const bb_attn_desc* desc, int pass, size_t* bytes);
+
+/* Forward ([gitcode page] section "BigBird：从二次方注意力到线性稀疏注意力":
+ * five segments first / second / middle / second_last / last, masked keys
+ * offset by -10000, row softmax).
+ *   q, k, v   [B][H][L][d] dtype, device
+ *   key_mask  [B][L] uint8, nonzero = attend; NULL = attend every key
+ *   rand_idx  [H][nb][r] int32, device (as bb_rand_attn_build writes it;
+ *             entries of rows 0 and nb-1 are ignored, -1 is padding, other
+ *             entries outside [0, nb) are ignored and flag BB_ERR_BAD_TABLE)
+ *   out       [B][H][L][d] dtype, device (written)
+ *   lse       [B][H][L] fp32, device (written): natural-log sum of exp of the
+ *             row's attended scores, used by the backward
+ *   workspace device, >= bb_attn_workspace_size(desc, 0) bytes */
+BB_API int bb_attn_fwd(const bb_attn_desc* desc, const void* q, const void* k,
+                const void* v, const uint8_t* key_mask,
+                const int32_t* rand_idx, void* out, float* lse,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward: gradients of the forward's output for upstream gradient dout.
+ * The pages train the layer by autodiff with recomputation (section
+ * "梯度检查点的实现方式"); this computes the same gradient directly,
+ * recomputing the probabilities from lse instead of storing them.
+ *   q, k, v, out, lse, key_mask, rand_idx as produced / used by bb_attn_fwd
+ *   dout      [B][H][L][d] dtype, device
+ *   dq, dk, dv [B][H][L][d] dtype, device (written)
+ *   workspace device, >= bb_attn_workspace_size(desc, 1) bytes; holds the
+ *             transposed block adjacency (query blocks per key block) and
+ *             the per-row D = <dO, O>. */
+BB_API int bb_attn_bwd(const bb_attn_desc* desc, const void* q, const void* k,
+                const void* v, const void* out, const float* lse,
+                const void* dout, const uint8_t* key_mask,
+                const int32_t* rand_idx, void* dq, void* dk, void* dv,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Number of kernel launches bb_attn_fwd (pass 0) or bb_attn_bwd (pass 1)
+ * makes for `desc`, written to *launches.  Host only. */
+BB_API int bb_attn_launch_count(const bb_attn_desc* desc, int pass,
+                                int* launches);
+
+/* Name of internal launch `index` (0-based, < bb_attn_launch_count) of
+ * pass 0 (forward) or 1 (backward) for `desc`, as a static NUL-terminated
+ * string in *name (e.g. "simt_fwd", "bwd_pre").  Host only. */
+BB_API int bb_attn_launch_name(const bb_attn_desc* desc, int pass, int index,
+                               const char** name);
+
+/* Profiling variants of bb_attn_fwd / bb_attn_bwd: same arguments and
+ * results, plus `events`, an array of num_events cudaEvent_t handles created
+ * by the caller.  events[k] is recorded on `stream` just before internal
+ * launch k and events[n] after the last one (n = bb_attn_launch_count);
+ * entries beyond num_events are not recorded.  Lets a caller time each
+ * kernel with CUDA events on the stream it runs on. */
+BB_API int bb_attn_fwd_events(const bb_attn_desc* desc, const void* q,
+                              const void* k, const void* v,
+                              const uint8_t* key_mask,
+                              const int32_t* rand_idx, void* out, float* lse,
+                              void* workspace, size_t workspace_bytes,
+                              void* stream, void* const* events,
+                              int num_events);
+BB_API int bb_attn_bwd_events(const bb_attn_desc* desc, const void* q,
+                              const void* k, const void* v, const void* out,
+                              const float* lse, const void* dout,
+                              const uint8_t* key_mask,
+                              const int32_t* rand_idx, void* dq, void* dk,
+                              void* dv, void* workspace,
+                              size_t workspace_bytes, void* stream,
+                              void* const* events, int num_events);
+
+/* Waits for `stream`, then returns the status word the last call that used
+ * `workspace` left there (BB_OK, BB_ERR_TIMEOUT or BB_ERR_BAD_TABLE), or
+ * BB_ERR_CUDA if the copy itself failed. */
+BB_API int bb_attn_check_status(const void* workspace, void* stream);
+
+/* Static description of a status code (never NULL). */
+BB_API const char* bb_status_str(int status);
+
+/* BB_ABI_VERSION of the loaded library. */
+BB_API int bb_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BB_ATTN_H_ */

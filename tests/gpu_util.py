@@ -1,0 +1,65 @@
+"""Helpers for the GPU parity tests: run the library through the C ABI and
+the oracle on the same seeded inputs."""
+
+import numpy as np
+import torch
+
+import oracle
+from block_sparse_long_bwd_b200 import binding as bb
+from block_sparse_long_bwd_b200 import synth
+
+# Tolerances the problem statement fixes: max-abs error against the fp64
+# oracle, per I/O precision (applied to O, lse, dQ, dK and dV alike).
+ATOL = {"f32": 2e-5, "bf16": 1e-2}
+
+
+def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
+            scale=0.0, mask_value=0.0, table=None):
+    """Forward (and backward) through the C ABI; returns CPU tensors."""
+    dev = torch.device("cuda")
+    B, H, L = cfg["B"], cfg["H"], cfg["L"]
+    att = bb.Attention(B, H, L, cfg["block_size"], cfg["r"],
+                       synth.torch_dtype(cfg["dtype"]), d=cfg["d"],
+                       seed=table_seed, scale=scale, mask_value=mask_value)
+    if table is not None:
+        att.table_host = torch.as_tensor(table, dtype=torch.int32)
+        att.table = att.table_host.to(dev)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+    out, lse = att.forward(q, k, v, km)
+    res = {"out": out, "lse": lse, "table": att.table_host,
+           "status_fwd": bb.bb_attn_check_status(att.ws_fwd)}
+    if backward:
+        dout = inp["dout"].to(dev)
+        dq, dk, dv = att.backward(q, k, v, out, lse, dout, km)
+        res.update(dq=dq, dk=dk, dv=dv,
+                   status_bwd=bb.bb_attn_check_status(att.ws_bwd))
+    torch.cuda.synchronize()
+    return {k_: (v_.float().cpu() if torch.is_tensor(v_) and v_.is_cuda
+                 else v_) for k_, v_ in res.items()}
+
+
+def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
+                 mask_value=oracle.DEFAULT_MASK_VALUE):
+    """Oracle on the (b, h) slice: rows of one (b, h) depend on nothing else."""
+    sl = lambda x: x[b:b + 1, h:h + 1].double().numpy()
+    km = inp["key_mask"]
+    km = None if km is None else km[b:b + 1].numpy()
+    tab = np.asarray(table)[h:h + 1]
+    o, lse = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), km, tab,
+                            cfg["block_size"], scale, mask_value)
+    res = {"out": o[0, 0], "lse": lse[0, 0]}
+    if backward:
+        dq, dk, dv = oracle.backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
+                                     sl(inp["dout"]), km, tab,
+                                     cfg["block_size"], scale, mask_value)
+        res.update(dq=dq[0, 0], dk=dk[0, 0], dv=dv[0, 0])
+    return res
+
+
+def assert_close(gpu, ora, b, h, atol, names):
+    for n in names:
+        g = gpu[n][b, h].double().numpy()
+        err = np.abs(g - ora[n]).max()
+        assert np.isfinite(g).all(), (n, b, h)
+        assert err <= atol, f"{n}[{b},{h}] max-abs err {err:.3e} > {atol}"

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point its header declares, builds the random table bit for bit
+like the oracle's independent generator, and rejects invalid arguments on
+the host before touching the device."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from block_sparse_long_bwd_b200 import binding as bb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f)
+           for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+def _declared():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(bb_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = bb.lib()
+    names = _declared()
+    assert "bb_attn_fwd" in names and "bb_attn_bwd" in names
+    for name in names:
+        assert hasattr(lib, name), name
+    assert bb.bb_abi_version() == 1
+
+
+@pytest.mark.parametrize("seed,H,nb,r", [
+    (0, 12, 64, 3), (0, 16, 64, 3), (0, 12, 256, 3), (0, 2, 16, 3),
+    (123456789, 3, 32, 6), ((1 << 64) - 1, 2, 8, 6), (7, 4, 5, 1),
+    (9, 1, 4, 3), (9, 1, 1, 2), (5, 12, 1024, 6), (2, 3, 33, 0),
+])
+def test_rand_table_bit_exact_vs_oracle(seed, H, nb, r):
+    got = bb.bb_rand_attn_build(seed, H, nb, r).numpy()
+    want = oracle.rand_table(seed, H, nb, r)
+    assert got.dtype == np.int32
+    assert np.array_equal(got, want)
+
+
+def test_rand_table_errors():
+    lib = bb.lib()
+    assert lib.bb_rand_attn_build(0, -1, 4, 3, None) == -1
+    assert lib.bb_rand_attn_build(0, 2, 4, 3, None) == -1
+    assert lib.bb_rand_attn_build(0, 0, 4, 3, None) == 0   # empty table
+
+
+def test_status_strings():
+    for code in (0, -1, -2, -3, -4, -5, -6, 42):
+        assert isinstance(bb.bb_status_str(code), str)
+
+
+def _desc(**kw):
+    base = dict(B=2, H=3, L=512, d=64, block_size=64, r=3, dtype=bb.BB_BF16)
+    base.update(kw)
+    return bb.make_desc(**base)
+
+
+def test_workspace_size_and_validation():
+    n0 = bb.bb_attn_workspace_size(_desc(), 0)
+    n1 = bb.bb_attn_workspace_size(_desc(), 1)
+    assert n0 > 0 and n1 > n0
+    bad = [
+        (dict(L=500), -1), (dict(B=0), -1), (dict(r=-1), -1),
+        (dict(dtype=7), -1), (dict(d=128), -2), (dict(block_size=16), -2),
+        (dict(r=33), -2), (dict(L=64 * 8193), -2),
+    ]
+    lib = bb.lib()
+    for kw, code in bad:
+        n = ctypes.c_size_t(0)
+        got = lib.bb_attn_workspace_size(ctypes.byref(_desc(**kw)), 0,
+                                         ctypes.byref(n))
+        assert got == code, (kw, got)
+    n = ctypes.c_size_t(0)
+    assert lib.bb_attn_workspace_size(None, 0, ctypes.byref(n)) == -1
+    assert lib.bb_attn_workspace_size(ctypes.byref(_desc()), 2,
+                                      ctypes.byref(n)) == -1
+
+
+def test_compute_calls_reject_bad_arguments_on_host():
+    """Fake (never dereferenced) pointers: every case fails validation before
+    any CUDA call is made."""
+    lib = bb.lib()
+    d = _desc()
+    good = 1 << 20  # 16-byte aligned fake address
+    ws_n = bb.bb_attn_workspace_size(d, 0)
+    args = [good] * 8
+    # NULL q
+    assert lib.bb_attn_fwd(ctypes.byref(d), None, *args[1:], ws_n, None) == -1
+    # misaligned v
+    a = list(args)
+    a[2] = good + 2
+    assert lib.bb_attn_fwd(ctypes.byref(d), *a, ws_n, None) == -1
+    # workspace too small / missing
+    assert lib.bb_attn_fwd(ctypes.byref(d), *args, ws_n - 1, None) == -4
+    a = list(args)
+    a[7] = None
+    assert lib.bb_attn_fwd(ctypes.byref(d), *a, ws_n, None) == -4
+    # unsupported desc
+    assert lib.bb_attn_fwd(ctypes.byref(_desc(d=32)), *args, ws_n, None) == -2
+    # r > 0 with no table
+    a = list(args)
+    a[4] = None
+    assert lib.bb_attn_fwd(ctypes.byref(d), *a, ws_n, None) == -1
+    ws_b = bb.bb_attn_workspace_size(d, 1)
+    bargs = [good] * 12
+    assert lib.bb_attn_bwd(ctypes.byref(d), *bargs, ws_b - 16, None) == -4
+    b = list(bargs)
+    b[9] = None  # dk
+    assert lib.bb_attn_bwd(ctypes.byref(d), *b, ws_b, None) == -1
+    assert lib.bb_attn_bwd(None, *bargs, ws_b, None) == -1

@@ -1,0 +1,135 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small shapes are compared element by element over every (b, h); the
+full-size workloads run in the launch configuration the benchmark times and
+are compared on sampled (b, h) slices, which the oracle computes exactly
+(rows of one (b, h) depend on nothing else)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_long_bwd_b200 import synth
+from gpu_util import ATOL, assert_close, oracle_slice, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+FWD = ("out", "lse")
+ALL = ("out", "lse", "dq", "dk", "dv")
+
+
+def _small(B, H, L, bs, r, dtype, mask=None, seed=11):
+    return dict(B=B, H=H, L=L, block_size=bs, d=64, r=r, dtype=dtype,
+                seed=seed, mask=mask, passes="fwd+bwd")
+
+
+def _check_all(cfg, res, inp, names=ALL, **kw):
+    tol = ATOL[cfg["dtype"]]
+    for b in range(cfg["B"]):
+        for h in range(cfg["H"]):
+            ora = oracle_slice(cfg, inp, res["table"], b, h,
+                               backward="dq" in names, **kw)
+            assert_close(res, ora, b, h, tol, names)
+
+
+def test_tiny_fp32_workload_full_compare():
+    cfg = synth.WORKLOADS["tiny_fp32_l1024"]
+    inp = synth.make_inputs(cfg)
+    res = run_gpu(cfg, inp)
+    assert res["status_fwd"] == 0 and res["status_bwd"] == 0
+    _check_all(cfg, res, inp)
+
+
+SMALL = [
+    # B, H, L, bs, r, dtype, mask
+    (1, 1, 64, 64, 3, "bf16", None),        # nb = 1
+    (2, 1, 128, 64, 3, "bf16", "tail"),     # nb = 2
+    (1, 2, 192, 64, 2, "f32", None),        # nb = 3
+    (1, 2, 256, 64, 3, "bf16", "random5"),  # nb = 4: dense
+    (2, 1, 320, 64, 0, "bf16", None),       # nb = 5, r = 0: not dense
+    (1, 3, 448, 64, 1, "f32", "tail"),      # nb = 7
+    (3, 2, 1088, 64, 3, "bf16", "tail"),    # nb = 17
+    (1, 2, 1024, 32, 3, "bf16", "random5"),  # bs = 32
+    (2, 1, 1024, 32, 6, "f32", None),
+    (1, 2, 1024, 128, 6, "bf16", None),     # clamped: fully dense
+    (2, 1, 2048, 128, 3, "bf16", "random5"),
+    (1, 1, 1152, 128, 2, "f32", "tail"),
+    (1, 5, 2112, 64, 6, "bf16", None),
+]
+
+
+@pytest.mark.parametrize("case", SMALL)
+def test_small_shapes_full_compare(case):
+    cfg = _small(*case)
+    inp = synth.make_inputs(cfg)
+    res = run_gpu(cfg, inp)
+    assert res["status_fwd"] == 0 and res["status_bwd"] == 0
+    _check_all(cfg, res, inp)
+
+
+def test_custom_scale_and_mask_value():
+    cfg = _small(1, 2, 640, 64, 2, "f32", "random5", seed=12)
+    inp = synth.make_inputs(cfg)
+    res = run_gpu(cfg, inp, scale=0.2, mask_value=-5.0)
+    _check_all(cfg, res, inp, scale=0.2, mask_value=-5.0)
+
+
+def test_corrupt_table_is_flagged_and_ignored():
+    cfg = _small(1, 2, 768, 64, 3, "bf16", None, seed=13)
+    inp = synth.make_inputs(cfg)
+    nb = cfg["L"] // cfg["block_size"]
+    table = oracle.rand_table(0, 2, nb, 3)
+    table[1, 4, 1] = nb + 7      # out of range: ignored, flagged
+    table[0, 5, 0] = -9          # out of range: ignored, flagged
+    table[0, 6, 2] = 6           # own window: redundant under set union
+    res = run_gpu(cfg, inp, table=table)
+    assert res["status_fwd"] == -6 and res["status_bwd"] == -6
+    clean = table.copy()
+    clean[1, 4, 1] = -1
+    clean[0, 5, 0] = -1
+    res["table"] = clean
+    _check_all(cfg, res, inp)
+
+
+def test_deterministic_bitwise():
+    cfg = _small(2, 3, 2048, 64, 3, "bf16", "tail", seed=14)
+    inp = synth.make_inputs(cfg)
+    a = run_gpu(cfg, inp)
+    b = run_gpu(cfg, inp)
+    for n in ALL:
+        assert torch.equal(a[n], b[n]), n
+
+
+def _full(cfg, samples, backward):
+    inp = synth.make_inputs(cfg, with_grad=backward)
+    res = run_gpu(cfg, inp, backward=backward)
+    assert res["status_fwd"] == 0
+    names = ALL if backward else FWD
+    for b, h in samples:
+        ora = oracle_slice(cfg, inp, res["table"], b, h, backward=backward)
+        assert_close(res, ora, b, h, ATOL[cfg["dtype"]], names)
+    for n in names:
+        assert torch.isfinite(res[n]).all(), n
+
+
+def test_full_base_fwd_l4096():
+    _full(synth.WORKLOADS["base_fwd_l4096"], [(0, 0), (3, 7), (7, 11)], False)
+
+
+def test_full_large_train_l4096():
+    _full(synth.WORKLOADS["large_train_l4096"], [(0, 0), (2, 9), (3, 15)],
+          True)
+
+
+def test_full_long_l16384():
+    _full(synth.WORKLOADS["long_l16384"], [(0, 0), (0, 11)], True)
+
+
+@pytest.mark.parametrize("L,bs,r", [(1024, 128, 6), (32768, 32, 6),
+                                    (32768, 128, 0), (8192, 64, 3),
+                                    (2048, 32, 0)])
+def test_full_sweep_points(L, bs, r):
+    cfg = synth.sweep_point(L, bs, r)
+    B = cfg["B"]
+    _full(cfg, [(0, 0), (B - 1, 11)], True)

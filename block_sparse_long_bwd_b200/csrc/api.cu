@@ -18,6 +18,12 @@ WsLayout ws_layout(const Problem& p, int pass) {
   w.status_off = off;
   off += 256;
   const size_t rows = (size_t)p.B * p.H * p.L;
+  if (pass == 0 && tc_fwd_supported(p)) {
+    w.part_off = off;
+    off = align_up(off + tc_fwd_part_bytes(p), 256);
+    w.total = off;
+    return w;
+  }
   if (pass == 1) {
     w.D_off = off;
     off = align_up(off + rows * sizeof(float), 256);
@@ -187,7 +193,13 @@ static int fwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess)
     return BB_ERR_CUDA;
   if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
-  if (launch_simt_fwd(p, s) != cudaSuccess) return BB_ERR_CUDA;
+  if (tc_fwd_supported(p)) {
+    TensorMaps tm;
+    if (!encode_tensor_maps(p, 0, &tm)) return BB_ERR_CUDA;
+    if (launch_tc_fwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
+  } else {
+    if (launch_simt_fwd(p, s) != cudaSuccess) return BB_ERR_CUDA;
+  }
   if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
   return BB_OK;
 }
@@ -237,6 +249,7 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
 // Names of the launches each pass makes, in order (kept beside the
 // dispatch in fwd_impl / bwd_impl).
 static const char* const kFwdSimt[] = {"simt_fwd"};
+static const char* const kFwdTc[] = {"tc_fwd", "fwd_combine"};
 static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
 
@@ -247,8 +260,9 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
   int st = make_problem(desc, &p);
   if (st != BB_OK) return st;
   if (pass == 0) {
-    *names = kFwdSimt;
-    *n = 1;
+    const bool tc = tc_fwd_supported(p);
+    *names = tc ? kFwdTc : kFwdSimt;
+    *n = tc ? 2 : 1;
   } else {
     *names = kBwdSimt;
     *n = 4;

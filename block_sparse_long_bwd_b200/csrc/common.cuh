@@ -2,6 +2,7 @@
 // libbbattn.so.  Not part of the C ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
@@ -70,6 +71,21 @@ struct EventMarks {
     return cudaSuccess;
   }
 };
+
+// TMA descriptors of the [B*H*L][64] bf16 row views of Q, K, V (and more
+// for the backward), 64 x 64 boxes, 128-byte swizzle.
+struct TensorMaps {
+  CUtensorMap q, k, v, o, dout;
+};
+// Encodes the maps a pass needs; false if the driver entry point or the
+// encode call fails.
+bool encode_tensor_maps(const Problem& p, int pass, TensorMaps* tm);
+
+// Tensor-core path (bf16, block 64, d 64).
+bool tc_fwd_supported(const Problem& p);
+size_t tc_fwd_part_bytes(const Problem& p);
+cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
+                          cudaStream_t s, EventMarks* marks);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_simt_fwd(const Problem& p, cudaStream_t s);

@@ -1,0 +1,568 @@
+// Tensor-core forward of the block-sparse attention (bf16 I/O, block 64,
+// d 64) for sm_100a: TMA tile loads, tcgen05 MMAs with TMEM accumulators and
+// an online softmax, in a persistent warp-specialised kernel.
+//
+// Work item = two query blocks of one (b, h) sharing one 128-row MMA tile:
+//  * middle pair (i, i+1): the key blocks streamed are the union of the two
+//    attended sets A(i) and A(i+1) (window, the two global blocks, random
+//    blocks); each key block carries a 2-bit mask saying which half of the
+//    tile attends it.  Blocks i and i+1, 0 and nb-1 are always shared.
+//  * global chunk: rows 0 and nb-1 (which attend every key block) over a
+//    chunk of kChunk consecutive key blocks; partial (O, m, l) go to the
+//    workspace and fwd_combine_kernel merges the chunks.
+//
+// Roles (192 threads): warp 0 lane 0 issues TMA loads (Q pair once per item,
+// K and V per key block through a kNST-stage ring); warp 1 lane 0 issues the
+// MMAs (S = Q K^T into one of two TMEM S buffers, then O_part = P V with P
+// read from TMEM); warps 2-5 run the softmax, one thread per tile row: load
+// S from TMEM, fold scale, key mask and running max, write P (bf16) back
+// over S, and accumulate O_part into registers with the rescale factor.
+#include "sm100.cuh"
+
+namespace bb {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBS = 64;
+constexpr int kNST = 4;
+constexpr int kMaxT = 32;
+constexpr int kChunk = 8;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTileBytes = kBS * kHeadDim * 2;  // 8 KB
+constexpr int kPartStride = 68;                      // floats per partial row
+
+struct ItemList {
+  int n;
+  int global;   // 1 = global chunk
+  int bh, b;
+  int blk[2];   // query block of half 0 / half 1 (-1: half unused)
+  int chunk;
+  int16_t tile[kMaxT];
+  uint8_t mask[kMaxT];
+};
+
+struct Bars {
+  uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
+  uint64_t kv_full[kNST], kv_empty[kNST];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_full[2], pv_empty[2];
+};
+
+struct FwdArgs {
+  Problem p;
+  int npairs, nchunks, items;
+};
+
+__device__ __forceinline__ void list_add(ItemList& L, int j, int bit) {
+  for (int c = 0; c < L.n; ++c)
+    if (L.tile[c] == j) {
+      L.mask[c] |= (uint8_t)bit;
+      return;
+    }
+  L.tile[L.n] = (int16_t)j;
+  L.mask[L.n] = (uint8_t)bit;
+  ++L.n;
+}
+
+__device__ void build_item(const FwdArgs& a, int item, ItemList& L) {
+  const Problem& p = a.p;
+  const int nb = p.nb;
+  const int per = a.npairs + a.nchunks;
+  const int bh = item / per, loc = item % per;
+  L.n = 0;
+  L.bh = bh;
+  L.b = bh / p.H;
+  const int h = bh % p.H;
+  if (loc < a.nchunks) {
+    L.global = 1;
+    L.chunk = loc;
+    L.blk[0] = 0;
+    L.blk[1] = nb > 1 ? nb - 1 : -1;
+    const int bits = nb > 1 ? 3 : 1;
+    const int j1 = min(nb, (loc + 1) * kChunk);
+    for (int j = loc * kChunk; j < j1; ++j) {
+      L.tile[L.n] = (int16_t)j;
+      L.mask[L.n] = (uint8_t)bits;
+      ++L.n;
+    }
+    return;
+  }
+  L.global = 0;
+  L.chunk = 0;
+  const int i0 = 1 + 2 * (loc - a.nchunks);
+  L.blk[0] = i0;
+  L.blk[1] = (i0 + 1 <= nb - 2) ? i0 + 1 : -1;
+  for (int half = 0; half < 2; ++half) {
+    const int i = L.blk[half];
+    if (i < 0) continue;
+    const int bit = 1 << half;
+    list_add(L, 0, bit);
+    list_add(L, i - 1, bit);
+    list_add(L, i, bit);
+    list_add(L, i + 1, bit);
+    list_add(L, nb - 1, bit);
+    const int32_t* row = p.rand_idx + ((size_t)h * nb + i) * p.r;
+    for (int c = 0; c < p.r; ++c) {
+      const int j = row[c];
+      if (j == -1) continue;
+      if (j < 0 || j >= nb) {
+        set_status(p.status, BB_ERR_BAD_TABLE);
+        continue;
+      }
+      list_add(L, j, bit);
+    }
+  }
+}
+
+// Validity bitmap of the 64 keys of key block j (bit k set = attend).
+__device__ __forceinline__ uint64_t key_bits(const Problem& p, int b, int j) {
+  const uint4* m4 = reinterpret_cast<const uint4*>(p.key_mask + (size_t)b * p.L +
+                                                   (size_t)j * kBS);
+  uint64_t bits = 0;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = __ldg(m4 + c);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int by = 0; by < 4; ++by)
+        if ((ws[e] >> (8 * by)) & 0xFFu) bits |= 1ull << (16 * c + 4 * e + by);
+  }
+  return bits;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    tc_fwd_kernel(const __grid_constant__ FwdArgs a,
+                  const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ Bars bars;
+  __shared__ ItemList lists[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const Problem& p = a.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // 1024-byte aligned operand area: Q[2] (16 KB each), then K/V stages.
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* Qs = base;                       // [2][128][64] bf16
+  uint8_t* KVs = base + 2 * 2 * kTileBytes;  // [kNST][K,V][64][64] bf16
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.list_full[s], 1);
+      mbar_init(&bars.list_empty[s], 5);
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_empty[s], 1);
+      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.pv_full[s], 1);
+      mbar_init(&bars.pv_empty[s], 4);
+    }
+    for (int s = 0; s < kNST; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t tS = tmem;          // 2 S/P buffers: columns [0, 128)
+  const uint32_t tPV = tmem + 128;   // 2 P*V buffers: columns [128, 256)
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t g = 0;
+      int qissued[2] = {0, 0};
+      uint32_t qpar[2] = {0, 0};
+      for (int k = 0, item = blockIdx.x; item < a.items;
+           ++k, item += gridDim.x) {
+        const int slot = k & 1;
+        const uint32_t ph = (k >> 1) & 1;
+        if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
+          break;
+        ItemList& L = lists[slot];
+        build_item(a, item, L);
+        mbar_arrive(&bars.list_full[slot]);
+        if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
+          break;
+        const int row0 = L.bh * p.L;
+        const uint32_t qbytes = (L.blk[1] >= 0 ? 2u : 1u) * kTileBytes;
+        mbar_expect_tx(&bars.q_full[slot], qbytes);
+        uint8_t* q = Qs + slot * 2 * kTileBytes;
+        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.blk[0] * kBS);
+        if (L.blk[1] >= 0)
+          tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
+                      row0 + L.blk[1] * kBS);
+        qissued[slot] = 1;
+        qpar[slot] = ph;
+        bool ok = true;
+        for (int t = 0; t < L.n; ++t) {
+          const int st = g % kNST;
+          const uint32_t kph = (g / kNST) & 1;
+          if (!mbar_wait(&bars.kv_empty[st], kph ^ 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bars.kv_full[st], 2 * kTileBytes);
+          uint8_t* kv = KVs + st * 2 * kTileBytes;
+          const int y = row0 + L.tile[t] * kBS;
+          tma_load_2d(kv, &tmK, &bars.kv_full[st], 0, y);
+          tma_load_2d(kv + kTileBytes, &tmV, &bars.kv_full[st], 0, y);
+          ++g;
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {
+        // Let issued copies land before the CTA's shared memory goes away:
+        // wait (bounded) for the phase of the last load into each buffer.
+        for (uint32_t s = 0; s < (uint32_t)kNST; ++s) {
+          if (g < s + 1) continue;
+          const uint32_t last = g - 1 - ((g - 1 - s) % kNST);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.kv_full[s], (last / kNST) & 1) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+        for (int s = 0; s < 2; ++s) {
+          if (!qissued[s]) continue;
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.q_full[s], qpar[s]) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
+    const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
+    uint32_t g = 0, u = 0;
+    bool ok = true;
+    for (int k = 0, item = blockIdx.x; item < a.items && ok;
+         ++k, item += gridDim.x) {
+      const int slot = k & 1;
+      const uint32_t ph = (k >> 1) & 1;
+      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      const int n = lists[slot].n;
+      if (!mbar_wait(&bars.q_full[slot], ph, &abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t qaddr = smem_u32(Qs + slot * 2 * kTileBytes);
+      auto issue_pv = [&](int t) -> bool {
+        const uint32_t uu = u + t, gg = g + t;
+        const int sb = uu & 1;
+        const uint32_t sph = (uu >> 1) & 1;
+        const int st = gg % kNST;
+        if (!mbar_wait(&bars.p_full[sb], sph, &abort_flag, p.status)) return false;
+        if (!mbar_wait(&bars.pv_empty[sb], sph ^ 1, &abort_flag, p.status))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t vaddr = smem_u32(KVs + st * 2 * kTileBytes + kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tPV + sb * 64, tS + sb * 64 + kk * 8,
+                   sdesc_sw128(vaddr + kk * 2048, 8192), idPV, kk > 0);
+          mma_commit(&bars.pv_full[sb]);
+          mma_commit(&bars.kv_empty[st]);
+          mma_commit(&bars.s_empty[sb]);
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t, gg = g + t;
+        const int sb = uu & 1;
+        const uint32_t sph = (uu >> 1) & 1;
+        const int st = gg % kNST;
+        if (!mbar_wait(&bars.kv_full[st], (gg / kNST) & 1, &abort_flag, p.status) ||
+            !mbar_wait(&bars.s_empty[sb], sph ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tS + sb * 64, sdesc_sw128(qaddr + kk * 32, 16),
+                   sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
+          mma_commit(&bars.s_full[sb]);
+          if (t == n - 1) mma_commit(&bars.q_empty[slot]);
+        }
+        __syncwarp();
+        if (t > 0 && !issue_pv(t - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && n > 0 && !issue_pv(n - 1)) ok = false;
+      g += n;
+      u += n;
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+    }
+  } else {
+    // ---------------- softmax / epilogue (warps 2-5) ----------------
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // TMEM lane = tile row
+    const int half = row >> 6;
+    const int hbit = 1 << half;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float c = p.scale * kLog2e;
+    const float mvl = p.mask_value * kLog2e;
+    uint32_t u = 0;
+    for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
+      const int slot = k & 1;
+      const uint32_t ph = (k >> 1) & 1;
+      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      const ItemList& L = lists[slot];
+      const int n = L.n;
+      float m = -INFINITY, l = 0.f;
+      float O[kHeadDim];
+#pragma unroll
+      for (int e = 0; e < kHeadDim; ++e) O[e] = 0.f;
+      float alpha_prev = 1.f;
+      bool att_prev = false;
+      bool ok = true;
+
+      auto accumulate = [&](int t) -> bool {
+        const uint32_t uu = u + t;
+        const int pb = uu & 1;
+        if (!mbar_wait(&bars.pv_full[pb], (uu >> 1) & 1, &abort_flag, p.status))
+          return false;
+        tc_fence_after();
+        if (att_prev) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tPV + pb * 64 + lane_off, r0);
+          tmem_ld32(tPV + pb * 64 + 32 + lane_off, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            O[e] = fmaf(O[e], alpha_prev, __uint_as_float(r0[e]));
+            O[32 + e] = fmaf(O[32 + e], alpha_prev, __uint_as_float(r1[e]));
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.pv_empty[pb]);
+        return true;
+      };
+
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t;
+        const int sb = uu & 1;
+        if (!mbar_wait(&bars.s_full[sb], (uu >> 1) & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool att = (L.mask[t] & hbit) != 0;
+        const uint32_t taddr = tS + sb * 64 + lane_off;
+        float alpha = 1.f;
+        uint32_t P[32];
+        if (att) {
+          uint32_t s0[32], s1[32];
+          tmem_ld32(taddr, s0);
+          tmem_ld32(taddr + 32, s1);
+          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          tmem_ld_wait();
+          float z[64];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            z[e] = __uint_as_float(s0[e]);
+            z[32 + e] = __uint_as_float(s1[e]);
+          }
+          float mnew;
+          if (kb == ~0ull && c > 0.f) {
+            float mx = z[0];
+#pragma unroll
+            for (int e = 1; e < 64; ++e) mx = fmaxf(mx, z[e]);
+            mnew = fmaxf(m, mx * c);
+            const float nm = -mnew;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) z[e] = fmaf(z[e], c, nm);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              z[e] = fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl);
+            float mx = z[0];
+#pragma unroll
+            for (int e = 1; e < 64; ++e) mx = fmaxf(mx, z[e]);
+            mnew = fmaxf(m, mx);
+#pragma unroll
+            for (int e = 0; e < 64; ++e) z[e] -= mnew;
+          }
+          alpha = ex2(m - mnew);
+          float sum = 0.f;
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const float p0 = ex2(z[e]), p1 = ex2(z[e + 1]);
+            sum += p0 + p1;
+            P[e >> 1] = pack_bf16(p0, p1);
+          }
+          l = fmaf(l, alpha, sum);
+          m = mnew;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) P[e] = 0u;
+        }
+        uint32_t P0[16], P1[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          P0[e] = P[e];
+          P1[e] = P[16 + e];
+        }
+        tmem_st16(taddr, P0);
+        tmem_st16(taddr + 16, P1);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full[sb]);
+        if (t > 0 && !accumulate(t - 1)) {
+          ok = false;
+          break;
+        }
+        alpha_prev = alpha;
+        att_prev = att;
+      }
+      if (ok && n > 0 && !accumulate(n - 1)) ok = false;
+      u += n;
+      if (!ok) break;
+
+      // ---- epilogue ----
+      const int blk = L.blk[half];
+      const int r64 = row & 63;
+      if (blk >= 0) {
+        if (!L.global) {
+          const float inv = 1.f / l;
+          const size_t grow = (size_t)L.bh * p.L + (size_t)blk * kBS + r64;
+          uint4* dst = reinterpret_cast<uint4*>(
+              static_cast<__nv_bfloat16*>(p.out) + grow * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            uint4 w;
+            w.x = pack_bf16(O[8 * v + 0] * inv, O[8 * v + 1] * inv);
+            w.y = pack_bf16(O[8 * v + 2] * inv, O[8 * v + 3] * inv);
+            w.z = pack_bf16(O[8 * v + 4] * inv, O[8 * v + 5] * inv);
+            w.w = pack_bf16(O[8 * v + 6] * inv, O[8 * v + 7] * inv);
+            dst[v] = w;
+          }
+          p.lse_out[grow] = (m + __log2f(l)) * (1.0f / kLog2e);
+        } else {
+          float* dst = p.part +
+                       (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) *
+                           kPartStride;
+#pragma unroll
+          for (int v = 0; v < 16; ++v)
+            reinterpret_cast<float4*>(dst)[v] =
+                make_float4(O[4 * v], O[4 * v + 1], O[4 * v + 2], O[4 * v + 3]);
+          dst[64] = m;
+          dst[65] = l;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge the global rows' split partials: one warp per row, lanes over d.
+__global__ void __launch_bounds__(256) fwd_combine_kernel(const FwdArgs a) {
+  const Problem& p = a.p;
+  const int nhalves = p.nb > 1 ? 2 : 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t grow_id = (size_t)blockIdx.x * 8 + warp;  // over bh x half x 64
+  const size_t total = (size_t)p.B * p.H * nhalves * kBS;
+  if (grow_id >= total) return;
+  const int r64 = grow_id % kBS;
+  const int half = (grow_id / kBS) % nhalves;
+  const size_t bh = grow_id / (kBS * nhalves);
+  const int row = half * 64 + r64;
+  float M = -INFINITY;
+  for (int c = 0; c < a.nchunks; ++c) {
+    const float* src = p.part + ((bh * a.nchunks + c) * 128 + row) * kPartStride;
+    M = fmaxf(M, src[64]);
+  }
+  float L = 0.f, o0 = 0.f, o1 = 0.f;
+  for (int c = 0; c < a.nchunks; ++c) {
+    const float* src = p.part + ((bh * a.nchunks + c) * 128 + row) * kPartStride;
+    const float w = ex2(src[64] - M);
+    L = fmaf(w, src[65], L);
+    const float2 o = reinterpret_cast<const float2*>(src)[lane];
+    o0 = fmaf(w, o.x, o0);
+    o1 = fmaf(w, o.y, o1);
+  }
+  const float inv = 1.f / L;
+  const int blk = half == 0 ? 0 : p.nb - 1;
+  const size_t grow = bh * p.L + (size_t)blk * kBS + r64;
+  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) +
+                              grow * kHeadDim)[lane] =
+      pack_bf16(o0 * inv, o1 * inv);
+  if (lane == 0) p.lse_out[grow] = (M + __log2f(L)) * (1.0f / kLog2e);
+}
+
+}  // namespace
+
+// ---- host side ----------------------------------------------------------
+
+size_t tc_fwd_part_bytes(const Problem& p) {
+  const int nchunks = (p.nb + kChunk - 1) / kChunk;
+  return (size_t)p.B * p.H * nchunks * 128 * kPartStride * sizeof(float);
+}
+
+bool tc_fwd_supported(const Problem& p) {
+  return p.dtype == BB_BF16 && p.bs == kBS && p.d == kHeadDim &&
+         10 + 2 * p.r <= kMaxT && (size_t)p.B * p.H * p.L < (1ull << 31);
+}
+
+cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
+                          cudaStream_t s, EventMarks* marks) {
+  FwdArgs a;
+  a.p = p;
+  a.nchunks = (p.nb + kChunk - 1) / kChunk;
+  a.npairs = p.nb > 2 ? (p.nb - 2 + 1) / 2 : 0;
+  a.items = p.B * p.H * (a.npairs + a.nchunks);
+  const size_t smem = 1024 + (2 * 2 + 2 * kNST) * kTileBytes;
+  cudaError_t e = cudaFuncSetAttribute(
+      tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = min(a.items, 2 * sms);
+  tc_fwd_kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = marks->mark(s);
+  if (e != cudaSuccess) return e;
+  const size_t rows = (size_t)p.B * p.H * (p.nb > 1 ? 2 : 1) * kBS;
+  fwd_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace bb

@@ -1,0 +1,56 @@
+// TMA descriptor encoding through the driver's cuTensorMapEncodeTiled,
+// fetched with cudaGetDriverEntryPoint so the library does not link libcuda.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace bb {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                  void*, const cuuint64_t*, const cuuint64_t*,
+                                  const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// [rows][64] bf16 row view, box 64 x 64, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
+  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool encode_tensor_maps(const Problem& p, int pass, TensorMaps* tm) {
+  const uint64_t rows = (uint64_t)p.B * p.H * p.L;
+  bool ok = encode_rows(&tm->q, p.q, rows) && encode_rows(&tm->k, p.k, rows) &&
+            encode_rows(&tm->v, p.v, rows);
+  if (ok && pass == 1)
+    ok = encode_rows(&tm->o, p.o, rows) && encode_rows(&tm->dout, p.dout, rows);
+  return ok;
+}
+
+}  // namespace bb

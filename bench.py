@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=10)
+    # Profiling runs (ncu) only: leave out the end-to-end and CPU legs.
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
     return ap.parse_args()
 
 
@@ -347,7 +350,8 @@ def run_ours(args, world, rank, local):
                            if alg.get(kernel_kind(n), (0, 0))[1] else None)}
                for n in names}
 
-    e2e = run_e2e(args, cfg, att, inp, dev, backward, world)
+    e2e = None if args.skip_e2e else run_e2e(args, cfg, att, inp, dev,
+                                             backward, world)
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -372,8 +376,8 @@ def run_ours(args, world, rank, local):
         "e2e": e2e,
     }
     if rank == 0:
-        result["cpu_baseline"] = cpu_baseline(cfg, att.table_host.numpy(),
-                                              backward, budget_s=12.0)
+        result["cpu_baseline"] = None if args.skip_cpu else cpu_baseline(
+            cfg, att.table_host.numpy(), backward, budget_s=12.0)
         print(json.dumps(result), flush=True)
 
 

@@ -203,12 +203,15 @@ def algorithmic(cfg, pairs_total):
     }
 
 
+KERNEL_KIND = {"simt_fwd": "fwd", "tc_fwd": "fwd", "simt_dq": "dq",
+               "tc_dq": "dq", "simt_dkdv": "dkdv", "tc_dkdv": "dkdv",
+               "bwd_pre": "bwd_pre", "csr_build": "csr_build"}
+
+
 def kernel_kind(name):
-    """Which algorithmic figure a launch name counts against."""
-    for kind in ("dkdv", "dq", "fwd", "bwd_pre", "csr_build"):
-        if kind in name:
-            return kind
-    return None
+    """Which algorithmic figure a launch name counts against (None for the
+    small merge kernels, which have no figure of their own)."""
+    return KERNEL_KIND.get(name)
 
 
 def kernel_bound(name):

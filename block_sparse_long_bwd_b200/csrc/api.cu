@@ -31,6 +31,12 @@ WsLayout ws_layout(const Problem& p, int pass) {
     off = align_up(off + (size_t)p.H * (p.nb + 1) * sizeof(int), 256);
     w.list_off = off;
     off = align_up(off + (size_t)p.H * pair_cap(p.nb, p.r) * sizeof(int), 256);
+    if (tc_bwd_supported(p)) {
+      w.part_off = off;
+      off = align_up(off + tc_bwd_extra_bytes(p), 256);
+      w.total = off;
+      return w;
+    }
   }
   w.part_off = off;
   w.total = off;
@@ -237,11 +243,19 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   if (cudaMemsetAsync(p.status, 0, sizeof(int), s) != cudaSuccess)
     return BB_ERR_CUDA;
   if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
-  if (launch_bwd_pre(p, s) != cudaSuccess) return BB_ERR_CUDA;
-  if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
-  if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
-  if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
-  if (launch_simt_bwd(p, s, marks) != cudaSuccess) return BB_ERR_CUDA;
+  if (tc_bwd_supported(p)) {
+    TensorMaps tm;
+    if (!encode_tensor_maps(p, 1, &tm)) return BB_ERR_CUDA;
+    if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
+    if (launch_tc_bwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
+  } else {
+    if (launch_bwd_pre(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
+    if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
+    if (launch_simt_bwd(p, s, marks) != cudaSuccess) return BB_ERR_CUDA;
+  }
   if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
   return BB_OK;
 }
@@ -252,6 +266,8 @@ static const char* const kFwdSimt[] = {"simt_fwd"};
 static const char* const kFwdTc[] = {"tc_fwd", "fwd_combine"};
 static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
+static const char* const kBwdTc[] = {"csr_build", "tc_dq", "tc_dkdv",
+                                     "bwd_finish"};
 
 static int launch_plan(const bb_attn_desc* desc, int pass,
                        const char* const** names, int* n) {
@@ -264,7 +280,7 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     *names = tc ? kFwdTc : kFwdSimt;
     *n = tc ? 2 : 1;
   } else {
-    *names = kBwdSimt;
+    *names = tc_bwd_supported(p) ? kBwdTc : kBwdSimt;
     *n = 4;
   }
   return BB_OK;

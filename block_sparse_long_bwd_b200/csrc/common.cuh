@@ -87,6 +87,11 @@ size_t tc_fwd_part_bytes(const Problem& p);
 cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);
 
+bool tc_bwd_supported(const Problem& p);
+size_t tc_bwd_extra_bytes(const Problem& p);
+cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
+                          cudaStream_t s, EventMarks* marks);
+
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_simt_fwd(const Problem& p, cudaStream_t s);
 cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s);

@@ -1,0 +1,886 @@
+// Tensor-core backward of the block-sparse attention (bf16 I/O, block 64,
+// d 64) for sm_100a.  Probabilities are recomputed from the forward's lse
+// (P = exp(S - lse)), so nothing of size pairs x bs^2 is stored.
+//
+// tc_dq_kernel: query-side items (as in the forward: middle query-block pairs
+//   and chunks of the global rows).  Per key block j of the item:
+//   S = Q K_j^T and dP = dO V_j^T into TMEM; one thread per row forms
+//   dS = P (dP - D) (D = <dO, O> of the row, computed at the start of the
+//   item and also written to the workspace with -lse*log2(e) for the next
+//   kernel); dS (bf16) goes back to TMEM and dQ += dS K_j accumulates in
+//   TMEM across the item.  Global rows write fp32 partials per chunk.
+// tc_dkdv_kernel: key-side items pair two key blocks (j, j+1) in one
+//   128-row tile and walk the union of their transposed adjacency lists (the
+//   query blocks that attend them, from the CSR); the global key blocks
+//   (0, nb-1), attended by every query block, are split into chunks of query
+//   blocks.  Per query block i: S^T = K_pair Q_i^T and dP^T = V_pair dO_i^T;
+//   P^T and dS^T (bf16) back to TMEM; dV += P^T dO_i and dK += dS^T Q_i
+//   accumulate in TMEM.  Each key row is owned by exactly one item (or one
+//   chunk partial), so there are no atomics.
+// bwd_finish_kernel: sums the chunk partials of the global query rows (dQ)
+//   and of the global key blocks (dK, dV) in a fixed order.
+#include "tc_common.cuh"
+
+namespace bb {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr int kKvStages = 3;
+constexpr int kQStages = 3;
+constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // Q, dO, NL, D
+
+struct BwdArgs {
+  PairArgs qa;       // query-side items (dq)
+  int kpairs;        // middle key-block pairs
+  int kchunks;       // query-block chunks of the global key blocks
+  int kitems;        // key-side items (dkdv)
+  float* D;          // [B*H*L]
+  float* NL;         // [B*H*L]: -lse * log2(e)
+  float* dqpart;     // [B*H][nchunks][128][64]
+  float* kvpart;     // [B*H][kchunks][128][128] (dK | dV)
+};
+
+__device__ __forceinline__ void ld_bf16x8_as_f(const __nv_bfloat16* p,
+                                               float (&f)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(p);
+  const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    f[2 * e] = __uint_as_float(ws[e] << 16);
+    f[2 * e + 1] = __uint_as_float(ws[e] & 0xFFFF0000u);
+  }
+}
+
+// ======================= dQ =======================
+
+struct DqBars {
+  uint64_t list_full[2], list_empty[2];
+  uint64_t q_full, q_empty;
+  uint64_t kv_full[kKvStages], kv_empty[kKvStages];
+  uint64_t s_full, s_empty, p_full, dq_full, dq_empty;
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    tc_dq_kernel(const __grid_constant__ BwdArgs ba,
+                 const __grid_constant__ CUtensorMap tmQ,
+                 const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmG) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ DqBars bars;
+  __shared__ ItemList lists[2];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const PairArgs& a = ba.qa;
+  const Problem& p = a.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* Qs = base;                          // [128][64] Q pair
+  uint8_t* Gs = base + 2 * kTileBytes;         // [128][64] dO pair
+  uint8_t* KVs = base + 4 * kTileBytes;        // [stage][K, V]
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.list_full[s], 1);
+      mbar_init(&bars.list_empty[s], 5);
+    }
+    mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_empty, 1);
+    for (int s = 0; s < kKvStages; ++s) {
+      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
+    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, 1);
+    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.dq_full, 1);
+    mbar_init(&bars.dq_empty, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmG);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t tDQ = tmem, tS = tmem + 64, tDP = tmem + 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t g = 0;
+      int q_issued = 0;
+      uint32_t q_par = 0;
+      for (int k = 0, item = blockIdx.x; item < a.items;
+           ++k, item += gridDim.x) {
+        const int slot = k & 1;
+        if (!mbar_wait(&bars.list_empty[slot], ((k >> 1) & 1) ^ 1, &abort_flag,
+                       p.status))
+          break;
+        ItemList& L = lists[slot];
+        build_pair_item(a, item, L);
+        mbar_arrive(&bars.list_full[slot]);
+        if (!mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        const int row0 = L.bh * p.L;
+        const int nh = L.blk[1] >= 0 ? 2 : 1;
+        mbar_expect_tx(&bars.q_full, 2u * nh * kTileBytes);
+        for (int hh = 0; hh < nh; ++hh) {
+          const int y = row0 + L.blk[hh] * kBS;
+          tma_load_2d(Qs + hh * kTileBytes, &tmQ, &bars.q_full, 0, y);
+          tma_load_2d(Gs + hh * kTileBytes, &tmG, &bars.q_full, 0, y);
+        }
+        q_issued = 1;
+        q_par = k & 1;
+        bool ok = true;
+        for (int t = 0; t < L.n; ++t) {
+          const int st = g % kKvStages;
+          if (!mbar_wait(&bars.kv_empty[st], ((g / kKvStages) & 1) ^ 1,
+                         &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&bars.kv_full[st], 2 * kTileBytes);
+          uint8_t* kv = KVs + st * 2 * kTileBytes;
+          const int y = row0 + L.tile[t] * kBS;
+          tma_load_2d(kv, &tmK, &bars.kv_full[st], 0, y);
+          tma_load_2d(kv + kTileBytes, &tmV, &bars.kv_full[st], 0, y);
+          ++g;
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {
+        for (uint32_t s = 0; s < (uint32_t)kKvStages; ++s) {
+          if (g < s + 1) continue;
+          const uint32_t last = g - 1 - ((g - 1 - s) % kKvStages);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.kv_full[s], (last / kKvStages) & 1) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+        if (q_issued) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.q_full, q_par) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+    const uint32_t idDQ = idesc_bf16(128, 64, 0, 1);
+    const uint32_t qaddr = smem_u32(Qs), gaddr = smem_u32(Gs);
+    uint32_t g = 0, u = 0;
+    bool ok = true;
+    for (int k = 0, item = blockIdx.x; item < a.items && ok;
+         ++k, item += gridDim.x) {
+      const int slot = k & 1;
+      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
+        break;
+      const int n = lists[slot].n;
+      if (!mbar_wait(&bars.q_full, k & 1, &abort_flag, p.status)) break;
+      tc_fence_after();
+      for (int t = 0; t < n; ++t, ++g, ++u) {
+        const int st = g % kKvStages;
+        if (!mbar_wait(&bars.kv_full[st], (g / kKvStages) & 1, &abort_flag,
+                       p.status) ||
+            !mbar_wait(&bars.s_empty, (u & 1) ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
+        const uint32_t vaddr = kaddr + kTileBytes;
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tS, sdesc_sw128(qaddr + kk * 32, 16),
+                   sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tDP, sdesc_sw128(gaddr + kk * 32, 16),
+                   sdesc_sw128(vaddr + kk * 32, 16), idS, kk > 0);
+          mma_commit(&bars.s_full);
+        }
+        __syncwarp();
+        if (!mbar_wait(&bars.p_full, u & 1, &abort_flag, p.status) ||
+            (t == 0 &&
+             !mbar_wait(&bars.dq_empty, (k & 1) ^ 1, &abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tDQ, tS + kk * 8, sdesc_sw128(kaddr + kk * 2048, 8192), idDQ,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.kv_empty[st]);
+          mma_commit(&bars.s_empty);
+          if (t == n - 1) {
+            mma_commit(&bars.dq_full);
+            mma_commit(&bars.q_empty);
+          }
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int half = row >> 6, hbit = 1 << half, r64 = row & 63;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float c = p.scale * kLog2e;
+    const float mvl = p.mask_value * kLog2e;
+    uint32_t u = 0;
+    for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
+      const int slot = k & 1;
+      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
+        break;
+      const ItemList& L = lists[slot];
+      const int n = L.n;
+      const int blk = L.blk[half];
+      const size_t grow = (size_t)L.bh * p.L + (size_t)(blk < 0 ? 0 : blk) * kBS + r64;
+      float nl2 = 0.f, Dr = 0.f;
+      if (blk >= 0) {
+        nl2 = -p.lse[grow] * kLog2e;
+        const __nv_bfloat16* Or = static_cast<const __nv_bfloat16*>(p.o) + grow * kHeadDim;
+        const __nv_bfloat16* Gr = static_cast<const __nv_bfloat16*>(p.dout) + grow * kHeadDim;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          float fo[8], fg[8];
+          ld_bf16x8_as_f(Or + 8 * v, fo);
+          ld_bf16x8_as_f(Gr + 8 * v, fg);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) Dr = fmaf(fo[e], fg[e], Dr);
+        }
+        if (!L.global || L.chunk == 0) {
+          ba.D[grow] = Dr;
+          ba.NL[grow] = nl2;
+        }
+      }
+      bool ok = true;
+      for (int t = 0; t < n; ++t, ++u) {
+        if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool att = (L.mask[t] & hbit) != 0;
+        uint32_t dS[32];
+        if (att) {
+          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t s[32], dp[32];
+            tmem_ld32(tS + hc * 32 + lane_off, s);
+            tmem_ld32(tDP + hc * 32 + lane_off, dp);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const int col = hc * 32 + e;
+              const float off0 = ((kb >> col) & 1ull) ? 0.f : mvl;
+              const float off1 = ((kb >> (col + 1)) & 1ull) ? 0.f : mvl;
+              const float p0 = ex2(fmaf(__uint_as_float(s[e]), c, nl2 + off0));
+              const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), c, nl2 + off1));
+              const float d0 = p0 * (__uint_as_float(dp[e]) - Dr);
+              const float d1 = p1 * (__uint_as_float(dp[e + 1]) - Dr);
+              dS[(col >> 1)] = pack_bf16(d0, d1);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) dS[e] = 0u;
+        }
+        uint32_t d0[16], d1[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          d0[e] = dS[e];
+          d1[e] = dS[16 + e];
+        }
+        tmem_st16(tS + lane_off, d0);
+        tmem_st16(tS + 16 + lane_off, d1);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full);
+      }
+      if (!ok) break;
+      if (!mbar_wait(&bars.dq_full, k & 1, &abort_flag, p.status)) break;
+      tc_fence_after();
+      uint32_t q0[32], q1[32];
+      tmem_ld32(tDQ + lane_off, q0);
+      tmem_ld32(tDQ + 32 + lane_off, q1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.dq_empty);
+      if (blk >= 0) {
+        if (!L.global) {
+          uint4* dst = reinterpret_cast<uint4*>(
+              static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint32_t* src = v < 4 ? q0 + 8 * v : q1 + 8 * (v - 4);
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(src[0]) * p.scale, __uint_as_float(src[1]) * p.scale);
+            w.y = pack_bf16(__uint_as_float(src[2]) * p.scale, __uint_as_float(src[3]) * p.scale);
+            w.z = pack_bf16(__uint_as_float(src[4]) * p.scale, __uint_as_float(src[5]) * p.scale);
+            w.w = pack_bf16(__uint_as_float(src[6]) * p.scale, __uint_as_float(src[7]) * p.scale);
+            dst[v] = w;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(
+              ba.dqpart + (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) * 64);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(q0[4 * v]), __uint_as_float(q0[4 * v + 1]),
+                                 __uint_as_float(q0[4 * v + 2]), __uint_as_float(q0[4 * v + 3]));
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[8 + v] = make_float4(__uint_as_float(q1[4 * v]), __uint_as_float(q1[4 * v + 1]),
+                                     __uint_as_float(q1[4 * v + 2]), __uint_as_float(q1[4 * v + 3]));
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ======================= dK / dV =======================
+
+// Key-side item decoding and the walk over attending query blocks.  Every
+// role of the kernel runs its own copy of this iterator; all copies see the
+// same sequence.
+struct KeyItem {
+  int bh, b;
+  int kb[2];          // key block of half 0 / 1 (-1: unused)
+  int global, chunk;
+  // walk state
+  const int* la;
+  const int* lb;
+  int na, nbb, ia, ib;
+  int cur, end, bits;
+
+  __device__ void init(const BwdArgs& ba, int item) {
+    const Problem& p = ba.qa.p;
+    const int nb = p.nb;
+    const int per = ba.kpairs + ba.kchunks;
+    bh = item / per;
+    b = bh / p.H;
+    const int h = bh % p.H;
+    const int loc = item % per;
+    ia = ib = na = nbb = 0;
+    la = lb = nullptr;
+    if (loc < ba.kchunks) {
+      global = 1;
+      chunk = loc;
+      kb[0] = 0;
+      kb[1] = nb > 1 ? nb - 1 : -1;
+      bits = nb > 1 ? 3 : 1;
+      cur = loc * kChunk;
+      end = min(nb, cur + kChunk);
+      return;
+    }
+    global = 0;
+    chunk = 0;
+    const int j0 = 1 + 2 * (loc - ba.kchunks);
+    kb[0] = j0;
+    kb[1] = (j0 + 1 <= nb - 2) ? j0 + 1 : -1;
+    const int* offs = p.csr_offs + (size_t)h * (nb + 1);
+    const int* list = p.csr_list + (size_t)h * p.csr_cap;
+    la = list + offs[j0];
+    na = offs[j0 + 1] - offs[j0];
+    if (kb[1] >= 0) {
+      lb = list + offs[j0 + 1];
+      nbb = offs[j0 + 2] - offs[j0 + 1];
+    }
+  }
+  // Next attending query block i and its half mask; false at the end.
+  __device__ bool next(int& i, int& mask) {
+    if (global) {
+      if (cur >= end) return false;
+      i = cur++;
+      mask = bits;
+      return true;
+    }
+    const int va = ia < na ? la[ia] : 0x7FFFFFFF;
+    const int vb = ib < nbb ? lb[ib] : 0x7FFFFFFF;
+    if (va == 0x7FFFFFFF && vb == 0x7FFFFFFF) return false;
+    if (va < vb) {
+      i = va;
+      mask = 1;
+      ++ia;
+    } else if (vb < va) {
+      i = vb;
+      mask = 2;
+      ++ib;
+    } else {
+      i = va;
+      mask = 3;
+      ++ia;
+      ++ib;
+    }
+    return true;
+  }
+};
+
+struct KvBars {
+  uint64_t kp_full, kp_empty;
+  uint64_t qt_full[kQStages], qt_empty[kQStages];
+  uint64_t s_full, s_empty, p_full, acc_full, acc_empty;
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    tc_dkdv_kernel(const __grid_constant__ BwdArgs ba,
+                   const __grid_constant__ CUtensorMap tmQ,
+                   const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmG) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ KvBars bars;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const Problem& p = ba.qa.p;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* Ks = base;                      // [128][64] K pair
+  uint8_t* Vs = base + 2 * kTileBytes;     // [128][64] V pair
+  uint8_t* QT = base + 4 * kTileBytes;     // [stage][Q | dO | NL[64] | D[64]]
+
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&bars.kp_full, 1);
+    mbar_init(&bars.kp_empty, 1);
+    for (int s = 0; s < kQStages; ++s) {
+      mbar_init(&bars.qt_full[s], 1);
+      mbar_init(&bars.qt_empty[s], 1);
+    }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_empty, 1);
+    mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.acc_full, 1);
+    mbar_init(&bars.acc_empty, 4);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmG);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t tDK = tmem, tDV = tmem + 64, tS = tmem + 128, tDP = tmem + 192;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t g = 0;
+      int kp_issued = 0;
+      uint32_t kp_par = 0;
+      for (int k = 0, item = blockIdx.x; item < ba.kitems;
+           ++k, item += gridDim.x) {
+        KeyItem it;
+        it.init(ba, item);
+        if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        const int row0 = it.bh * p.L;
+        const int nh = it.kb[1] >= 0 ? 2 : 1;
+        mbar_expect_tx(&bars.kp_full, 2u * nh * kTileBytes);
+        for (int hh = 0; hh < nh; ++hh) {
+          const int y = row0 + it.kb[hh] * kBS;
+          tma_load_2d(Ks + hh * kTileBytes, &tmK, &bars.kp_full, 0, y);
+          tma_load_2d(Vs + hh * kTileBytes, &tmV, &bars.kp_full, 0, y);
+        }
+        kp_issued = 1;
+        kp_par = k & 1;
+        int i, mask;
+        bool ok = true;
+        while (it.next(i, mask)) {
+          const int st = g % kQStages;
+          if (!mbar_wait(&bars.qt_empty[st], ((g / kQStages) & 1) ^ 1,
+                         &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* q = QT + st * kQStageBytes;
+          mbar_expect_tx(&bars.qt_full[st], 2 * kTileBytes + 512);
+          const int y = row0 + i * kBS;
+          tma_load_2d(q, &tmQ, &bars.qt_full[st], 0, y);
+          tma_load_2d(q + kTileBytes, &tmG, &bars.qt_full[st], 0, y);
+          bulk_load(q + 2 * kTileBytes, ba.NL + y, 256, &bars.qt_full[st]);
+          bulk_load(q + 2 * kTileBytes + 256, ba.D + y, 256, &bars.qt_full[st]);
+          ++g;
+        }
+        if (!ok) break;
+      }
+      if (abort_flag) {
+        for (uint32_t s = 0; s < (uint32_t)kQStages; ++s) {
+          if (g < s + 1) continue;
+          const uint32_t last = g - 1 - ((g - 1 - s) % kQStages);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.qt_full[s], (last / kQStages) & 1) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+        if (kp_issued) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.kp_full, kp_par) &&
+                 globaltimer() - t0 < 100000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+    const uint32_t idAcc = idesc_bf16(128, 64, 0, 1);
+    const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
+    uint32_t g = 0, u = 0;
+    bool ok = true;
+    for (int k = 0, item = blockIdx.x; item < ba.kitems && ok;
+         ++k, item += gridDim.x) {
+      KeyItem it;
+      it.init(ba, item);
+      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
+      tc_fence_after();
+      int i, mask, t = 0;
+      while (it.next(i, mask)) {
+        const int st = g % kQStages;
+        if (!mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
+                       p.status) ||
+            !mbar_wait(&bars.s_empty, (u & 1) ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
+        const uint32_t gaddr = qaddr + kTileBytes;
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tS, sdesc_sw128(kaddr + kk * 32, 16),
+                   sdesc_sw128(qaddr + kk * 32, 16), idS, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tDP, sdesc_sw128(vaddr + kk * 32, 16),
+                   sdesc_sw128(gaddr + kk * 32, 16), idS, kk > 0);
+          mma_commit(&bars.s_full);
+        }
+        __syncwarp();
+        if (!mbar_wait(&bars.p_full, u & 1, &abort_flag, p.status) ||
+            (t == 0 &&
+             !mbar_wait(&bars.acc_empty, (k & 1) ^ 1, &abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tDV, tS + kk * 8, sdesc_sw128(gaddr + kk * 2048, 8192), idAcc,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tDK, tDP + kk * 8, sdesc_sw128(qaddr + kk * 2048, 8192), idAcc,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.qt_empty[st]);
+          mma_commit(&bars.s_empty);
+        }
+        __syncwarp();
+        ++g;
+        ++u;
+        ++t;
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(&bars.acc_full);
+        mma_commit(&bars.kp_empty);
+      }
+      __syncwarp();
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int half = row >> 6, hbit = 1 << half, r64 = row & 63;
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const float c = p.scale * kLog2e;
+    const float mvl = p.mask_value * kLog2e;
+    uint32_t g = 0, u = 0;
+    for (int k = 0, item = blockIdx.x; item < ba.kitems; ++k, item += gridDim.x) {
+      KeyItem it;
+      it.init(ba, item);
+      const int kblk = it.kb[half];
+      const size_t krow = (size_t)it.bh * p.L + (size_t)(kblk < 0 ? 0 : kblk) * kBS + r64;
+      float off = 0.f;
+      if (kblk >= 0 && p.key_mask)
+        off = p.key_mask[(size_t)it.b * p.L + (size_t)kblk * kBS + r64] ? 0.f : mvl;
+      int i, mask;
+      bool ok = true;
+      while (it.next(i, mask)) {
+        const int st = g % kQStages;
+        if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool att = (mask & hbit) != 0;
+        uint32_t P[32], dS[32];
+        // The stage's NL / D arrived by bulk copy: observe its barrier too.
+        if (att && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
+                              p.status)) {
+          ok = false;
+          break;
+        }
+        if (att) {
+          const float* NLs = reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
+          const float* Ds = NLs + 64;
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
+            uint32_t s[32], dp[32];
+            tmem_ld32(tS + hc * 32 + lane_off, s);
+            tmem_ld32(tDP + hc * 32 + lane_off, dp);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              const int col = hc * 32 + e;
+              const float4 nl = *reinterpret_cast<const float4*>(NLs + col);
+              const float4 dd = *reinterpret_cast<const float4*>(Ds + col);
+              const float nls[4] = {nl.x, nl.y, nl.z, nl.w};
+              const float dds[4] = {dd.x, dd.y, dd.z, dd.w};
+              float pv[4], dv[4];
+#pragma unroll
+              for (int x = 0; x < 4; ++x) {
+                pv[x] = ex2(fmaf(__uint_as_float(s[e + x]), c, nls[x] + off));
+                dv[x] = pv[x] * (__uint_as_float(dp[e + x]) - dds[x]);
+              }
+              P[col >> 1] = pack_bf16(pv[0], pv[1]);
+              P[(col >> 1) + 1] = pack_bf16(pv[2], pv[3]);
+              dS[col >> 1] = pack_bf16(dv[0], dv[1]);
+              dS[(col >> 1) + 1] = pack_bf16(dv[2], dv[3]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            P[e] = 0u;
+            dS[e] = 0u;
+          }
+        }
+        {
+          uint32_t a0[16], a1[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            a0[e] = P[e];
+            a1[e] = P[16 + e];
+          }
+          tmem_st16(tS + lane_off, a0);
+          tmem_st16(tS + 16 + lane_off, a1);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            a0[e] = dS[e];
+            a1[e] = dS[16 + e];
+          }
+          tmem_st16(tDP + lane_off, a0);
+          tmem_st16(tDP + 16 + lane_off, a1);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.p_full);
+        ++g;
+        ++u;
+      }
+      if (!ok) break;
+      if (!mbar_wait(&bars.acc_full, k & 1, &abort_flag, p.status)) break;
+      tc_fence_after();
+      uint32_t k0[32], k1[32], v0[32], v1[32];
+      tmem_ld32(tDK + lane_off, k0);
+      tmem_ld32(tDK + 32 + lane_off, k1);
+      tmem_ld32(tDV + lane_off, v0);
+      tmem_ld32(tDV + 32 + lane_off, v1);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.acc_empty);
+      if (kblk >= 0) {
+        if (!it.global) {
+          uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + krow * kHeadDim);
+          uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + krow * kHeadDim);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint32_t* sk = v < 4 ? k0 + 8 * v : k1 + 8 * (v - 4);
+            const uint32_t* sv = v < 4 ? v0 + 8 * v : v1 + 8 * (v - 4);
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(sk[0]) * p.scale, __uint_as_float(sk[1]) * p.scale);
+            w.y = pack_bf16(__uint_as_float(sk[2]) * p.scale, __uint_as_float(sk[3]) * p.scale);
+            w.z = pack_bf16(__uint_as_float(sk[4]) * p.scale, __uint_as_float(sk[5]) * p.scale);
+            w.w = pack_bf16(__uint_as_float(sk[6]) * p.scale, __uint_as_float(sk[7]) * p.scale);
+            dk[v] = w;
+            w.x = pack_bf16(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
+            w.y = pack_bf16(__uint_as_float(sv[2]), __uint_as_float(sv[3]));
+            w.z = pack_bf16(__uint_as_float(sv[4]), __uint_as_float(sv[5]));
+            w.w = pack_bf16(__uint_as_float(sv[6]), __uint_as_float(sv[7]));
+            dv[v] = w;
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(
+              ba.kvpart + (((size_t)it.bh * ba.kchunks + it.chunk) * 128 + row) * 128);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            dst[v] = make_float4(__uint_as_float(k0[4 * v]), __uint_as_float(k0[4 * v + 1]),
+                                 __uint_as_float(k0[4 * v + 2]), __uint_as_float(k0[4 * v + 3]));
+            dst[8 + v] = make_float4(__uint_as_float(k1[4 * v]), __uint_as_float(k1[4 * v + 1]),
+                                     __uint_as_float(k1[4 * v + 2]), __uint_as_float(k1[4 * v + 3]));
+            dst[16 + v] = make_float4(__uint_as_float(v0[4 * v]), __uint_as_float(v0[4 * v + 1]),
+                                      __uint_as_float(v0[4 * v + 2]), __uint_as_float(v0[4 * v + 3]));
+            dst[24 + v] = make_float4(__uint_as_float(v1[4 * v]), __uint_as_float(v1[4 * v + 1]),
+                                      __uint_as_float(v1[4 * v + 2]), __uint_as_float(v1[4 * v + 3]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// One warp per row of a global block (query rows for dQ, key rows for
+// dK/dV); lanes over d.  Chunks are summed in a fixed order.
+__global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
+  const Problem& p = ba.qa.p;
+  const int nhalves = p.nb > 1 ? 2 : 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t id = (size_t)blockIdx.x * 8 + warp;
+  const size_t total = (size_t)p.B * p.H * nhalves * kBS;
+  if (id >= total) return;
+  const int r64 = id % kBS;
+  const int half = (id / kBS) % nhalves;
+  const size_t bh = id / (kBS * nhalves);
+  const int row = half * 64 + r64;
+  const int blk = half == 0 ? 0 : p.nb - 1;
+  const size_t grow = bh * p.L + (size_t)blk * kBS + r64;
+  float q0 = 0.f, q1 = 0.f;
+  for (int c = 0; c < ba.qa.nchunks; ++c) {
+    const float2 x = reinterpret_cast<const float2*>(
+        ba.dqpart + ((bh * ba.qa.nchunks + c) * 128 + row) * 64)[lane];
+    q0 += x.x;
+    q1 += x.y;
+  }
+  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  for (int c = 0; c < ba.kchunks; ++c) {
+    const float* src = ba.kvpart + ((bh * ba.kchunks + c) * 128 + row) * 128;
+    const float2 xk = reinterpret_cast<const float2*>(src)[lane];
+    const float2 xv = reinterpret_cast<const float2*>(src + 64)[lane];
+    k0 += xk.x;
+    k1 += xk.y;
+    v0 += xv.x;
+    v1 += xv.y;
+  }
+  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim)[lane] =
+      pack_bf16(q0 * p.scale, q1 * p.scale);
+  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dk) + grow * kHeadDim)[lane] =
+      pack_bf16(k0 * p.scale, k1 * p.scale);
+  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dv) + grow * kHeadDim)[lane] =
+      pack_bf16(v0, v1);
+}
+
+BwdArgs make_bwd_args(const Problem& p) {
+  BwdArgs ba;
+  ba.qa = make_pair_args(p);
+  ba.kchunks = ba.qa.nchunks;
+  ba.kpairs = ba.qa.npairs;
+  ba.kitems = p.B * p.H * (ba.kpairs + ba.kchunks);
+  return ba;
+}
+
+}  // namespace
+
+bool tc_bwd_supported(const Problem& p) { return tc_shape_ok(p); }
+
+// D, NL: rows floats each; dq partials; dK/dV partials.
+size_t tc_bwd_extra_bytes(const Problem& p) {
+  const size_t rows = (size_t)p.B * p.H * p.L;
+  const int nch = (p.nb + kChunk - 1) / kChunk;
+  return rows * 4 /* NL */ + (size_t)p.B * p.H * nch * 128 * 64 * 4 +
+         (size_t)p.B * p.H * nch * 128 * 128 * 4 + 3 * 256;
+}
+
+cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
+                          cudaStream_t s, EventMarks* marks) {
+  BwdArgs ba = make_bwd_args(p);
+  const size_t rows = (size_t)p.B * p.H * p.L;
+  const int nch = ba.qa.nchunks;
+  auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+  uint8_t* x = reinterpret_cast<uint8_t*>(p.part);
+  ba.D = p.D;
+  ba.NL = reinterpret_cast<float*>(x);
+  x += al(rows * 4);
+  ba.dqpart = reinterpret_cast<float*>(x);
+  x += al((size_t)p.B * p.H * nch * 128 * 64 * 4);
+  ba.kvpart = reinterpret_cast<float*>(x);
+
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+  const size_t smem_dq = 1024 + (4 + 2 * kKvStages) * kTileBytes;
+  cudaError_t e = cudaFuncSetAttribute(
+      tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
+  if (e != cudaSuccess) return e;
+  tc_dq_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_dq, s>>>(
+      ba, tm.q, tm.k, tm.v, tm.dout);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = marks->mark(s);
+  if (e != cudaSuccess) return e;
+
+  const size_t smem_kv = 1024 + 4 * kTileBytes + kQStages * kQStageBytes;
+  e = cudaFuncSetAttribute(tc_dkdv_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
+  if (e != cudaSuccess) return e;
+  tc_dkdv_kernel<<<min(ba.kitems, 2 * sms), kThreads, smem_kv, s>>>(
+      ba, tm.q, tm.k, tm.v, tm.dout);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = marks->mark(s);
+  if (e != cudaSuccess) return e;
+
+  const size_t frows = (size_t)p.B * p.H * (p.nb > 1 ? 2 : 1) * kBS;
+  bwd_finish_kernel<<<(unsigned)((frows + 7) / 8), 256, 0, s>>>(ba);
+  return cudaGetLastError();
+}
+
+}  // namespace bb

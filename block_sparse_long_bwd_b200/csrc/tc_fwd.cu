@@ -17,31 +17,16 @@
 // read from TMEM); warps 2-5 run the softmax, one thread per tile row: load
 // S from TMEM, fold scale, key mask and running max, write P (bf16) back
 // over S, and accumulate O_part into registers with the rescale factor.
-#include "sm100.cuh"
+#include "tc_common.cuh"
 
 namespace bb {
 namespace {
 
 using namespace sm100;
 
-constexpr int kBS = 64;
 constexpr int kNST = 4;
-constexpr int kMaxT = 32;
-constexpr int kChunk = 8;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTileBytes = kBS * kHeadDim * 2;  // 8 KB
-constexpr int kPartStride = 68;                      // floats per partial row
-
-struct ItemList {
-  int n;
-  int global;   // 1 = global chunk
-  int bh, b;
-  int blk[2];   // query block of half 0 / half 1 (-1: half unused)
-  int chunk;
-  int16_t tile[kMaxT];
-  uint8_t mask[kMaxT];
-};
 
 struct Bars {
   uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
@@ -49,92 +34,8 @@ struct Bars {
   uint64_t s_full[2], s_empty[2], p_full[2], pv_full[2], pv_empty[2];
 };
 
-struct FwdArgs {
-  Problem p;
-  int npairs, nchunks, items;
-};
-
-__device__ __forceinline__ void list_add(ItemList& L, int j, int bit) {
-  for (int c = 0; c < L.n; ++c)
-    if (L.tile[c] == j) {
-      L.mask[c] |= (uint8_t)bit;
-      return;
-    }
-  L.tile[L.n] = (int16_t)j;
-  L.mask[L.n] = (uint8_t)bit;
-  ++L.n;
-}
-
-__device__ void build_item(const FwdArgs& a, int item, ItemList& L) {
-  const Problem& p = a.p;
-  const int nb = p.nb;
-  const int per = a.npairs + a.nchunks;
-  const int bh = item / per, loc = item % per;
-  L.n = 0;
-  L.bh = bh;
-  L.b = bh / p.H;
-  const int h = bh % p.H;
-  if (loc < a.nchunks) {
-    L.global = 1;
-    L.chunk = loc;
-    L.blk[0] = 0;
-    L.blk[1] = nb > 1 ? nb - 1 : -1;
-    const int bits = nb > 1 ? 3 : 1;
-    const int j1 = min(nb, (loc + 1) * kChunk);
-    for (int j = loc * kChunk; j < j1; ++j) {
-      L.tile[L.n] = (int16_t)j;
-      L.mask[L.n] = (uint8_t)bits;
-      ++L.n;
-    }
-    return;
-  }
-  L.global = 0;
-  L.chunk = 0;
-  const int i0 = 1 + 2 * (loc - a.nchunks);
-  L.blk[0] = i0;
-  L.blk[1] = (i0 + 1 <= nb - 2) ? i0 + 1 : -1;
-  for (int half = 0; half < 2; ++half) {
-    const int i = L.blk[half];
-    if (i < 0) continue;
-    const int bit = 1 << half;
-    list_add(L, 0, bit);
-    list_add(L, i - 1, bit);
-    list_add(L, i, bit);
-    list_add(L, i + 1, bit);
-    list_add(L, nb - 1, bit);
-    const int32_t* row = p.rand_idx + ((size_t)h * nb + i) * p.r;
-    for (int c = 0; c < p.r; ++c) {
-      const int j = row[c];
-      if (j == -1) continue;
-      if (j < 0 || j >= nb) {
-        set_status(p.status, BB_ERR_BAD_TABLE);
-        continue;
-      }
-      list_add(L, j, bit);
-    }
-  }
-}
-
-// Validity bitmap of the 64 keys of key block j (bit k set = attend).
-__device__ __forceinline__ uint64_t key_bits(const Problem& p, int b, int j) {
-  const uint4* m4 = reinterpret_cast<const uint4*>(p.key_mask + (size_t)b * p.L +
-                                                   (size_t)j * kBS);
-  uint64_t bits = 0;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 w = __ldg(m4 + c);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-#pragma unroll
-      for (int by = 0; by < 4; ++by)
-        if ((ws[e] >> (8 * by)) & 0xFFu) bits |= 1ull << (16 * c + 4 * e + by);
-  }
-  return bits;
-}
-
 __global__ void __launch_bounds__(kThreads, 2)
-    tc_fwd_kernel(const __grid_constant__ FwdArgs a,
+    tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
@@ -200,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
         ItemList& L = lists[slot];
-        build_item(a, item, L);
+        build_pair_item(a, item, L);
         mbar_arrive(&bars.list_full[slot]);
         if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
@@ -492,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // Merge the global rows' split partials: one warp per row, lanes over d.
-__global__ void __launch_bounds__(256) fwd_combine_kernel(const FwdArgs a) {
+__global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
   const Problem& p = a.p;
   const int nhalves = p.nb > 1 ? 2 : 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -535,18 +436,11 @@ size_t tc_fwd_part_bytes(const Problem& p) {
   return (size_t)p.B * p.H * nchunks * 128 * kPartStride * sizeof(float);
 }
 
-bool tc_fwd_supported(const Problem& p) {
-  return p.dtype == BB_BF16 && p.bs == kBS && p.d == kHeadDim &&
-         10 + 2 * p.r <= kMaxT && (size_t)p.B * p.H * p.L < (1ull << 31);
-}
+bool tc_fwd_supported(const Problem& p) { return tc_shape_ok(p); }
 
 cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
-  FwdArgs a;
-  a.p = p;
-  a.nchunks = (p.nb + kChunk - 1) / kChunk;
-  a.npairs = p.nb > 2 ? (p.nb - 2 + 1) / 2 : 0;
-  a.items = p.B * p.H * (a.npairs + a.nchunks);
+  const PairArgs a = make_pair_args(p);
   const size_t smem = 1024 + (2 * 2 + 2 * kNST) * kTileBytes;
   cudaError_t e = cudaFuncSetAttribute(
       tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -25,18 +25,23 @@ namespace {
 using namespace sm100;
 
 constexpr int kNST = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 256;
 // Rescale threshold of the lazy running max (log2 units): the max used for
-// the exponent is only moved when a row's true max exceeds it by more than
+// the exponent only moves when a row's true max exceeds it by more than
 // this, so probabilities stay below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.0f;
+
+// TMEM columns: S[2] (fp32, 64 each), P[2] (bf16 pairs, 32 each), O (fp32).
+// S, P and O are separate so the next S can be computed as soon as the
+// softmax has read the current one, and P V accumulates straight into O.
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct Bars {
   uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
   uint64_t kv_full[kNST], kv_empty[kNST];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
-  uint64_t o_empty, xch_full[2];
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t pv_done, o_empty;
 };
 
 __device__ __forceinline__ float max8(const float* z) {
@@ -53,7 +58,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ ItemList lists[2];
-  __shared__ float2 xch[2][128];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -68,15 +72,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.list_full[s], 1);
-      mbar_init(&bars.list_empty[s], 9);
+      mbar_init(&bars.list_empty[s], 5);
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
       mbar_init(&bars.s_full[s], 1);
-      mbar_init(&bars.s_empty[s], 1);
+      mbar_init(&bars.s_empty[s], 4);
       mbar_init(&bars.p_full[s], 4);
-      mbar_init(&bars.pv_done[s], 1);
-      mbar_init(&bars.xch_full[s], 4);
+      mbar_init(&bars.p_empty[s], 1);
     }
+    mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_empty, 4);
     for (int s = 0; s < kNST; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -97,8 +101,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tS = tmem;         // S/P of group 0 / 1: columns [0, 128)
-  const uint32_t tO = tmem + 128;   // O of group 0 / 1: columns [128, 256)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -168,8 +170,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---------------- MMA issuer ----------------
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
-    uint32_t g = 0;
-    uint32_t cnt[2] = {0, 0};
+    uint32_t g = 0, u = 0;  // K/V stage counter, tile counter
     bool ok = true;
     for (int k = 0, item = blockIdx.x; item < a.items && ok;
          ++k, item += gridDim.x) {
@@ -180,12 +181,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!mbar_wait(&bars.q_full[slot], ph, &abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t qaddr = smem_u32(Qs + slot * 2 * kTileBytes);
-      uint32_t pend_c = 0;
-      // P V of tile t (group t & 1) into that group's O accumulator.
-      auto issue_pv = [&](int t, uint32_t c) -> bool {
-        const int gg = t & 1;
+      // P V of tile t into O.
+      auto issue_pv = [&](int t) -> bool {
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
         const int st = (g + t) % kNST;
-        if (!mbar_wait(&bars.p_full[gg], c & 1, &abort_flag, p.status)) return false;
+        if (!mbar_wait(&bars.p_full[b2], (uu >> 1) & 1, &abort_flag, p.status))
+          return false;
         if (t == 0 && !mbar_wait(&bars.o_empty, (k & 1) ^ 1, &abort_flag, p.status))
           return false;
         tc_fence_after();
@@ -193,23 +195,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t vaddr = smem_u32(KVs + st * 2 * kTileBytes + kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tO + gg * 64, tS + gg * 64 + kk * 8,
+            mma_ts(tmem + kColO, tmem + kColP + b2 * 32 + kk * 8,
                    sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
-                   (t >= 2 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars.pv_done[gg]);
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.pv_done);
+          mma_commit(&bars.p_empty[b2]);
           mma_commit(&bars.kv_empty[st]);
-          mma_commit(&bars.s_empty[gg]);
         }
         __syncwarp();
         return true;
       };
       for (int t = 0; t < n; ++t) {
-        const int gg = t & 1;
-        const uint32_t c = cnt[gg]++;
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
         const int st = (g + t) % kNST;
         if (!mbar_wait(&bars.kv_full[st], ((g + t) / kNST) & 1, &abort_flag,
                        p.status) ||
-            !mbar_wait(&bars.s_empty[gg], (c & 1) ^ 1, &abort_flag, p.status)) {
+            !mbar_wait(&bars.s_empty[b2], ((uu >> 1) & 1) ^ 1, &abort_flag,
+                       p.status)) {
           ok = false;
           break;
         }
@@ -218,35 +221,33 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tS + gg * 64, sdesc_sw128(qaddr + kk * 32, 16),
+            mma_ss(tmem + kColS + b2 * 64, sdesc_sw128(qaddr + kk * 32, 16),
                    sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
-          mma_commit(&bars.s_full[gg]);
+          mma_commit(&bars.s_full[b2]);
           if (t == n - 1) mma_commit(&bars.q_empty[slot]);
         }
         __syncwarp();
-        if (t > 0 && !issue_pv(t - 1, pend_c)) {
+        if (t > 0 && !issue_pv(t - 1)) {
           ok = false;
           break;
         }
-        pend_c = c;
       }
-      if (ok && n > 0 && !issue_pv(n - 1, pend_c)) ok = false;
+      if (ok && n > 0 && !issue_pv(n - 1)) ok = false;
       g += n;
+      u += n;
       if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
     }
   } else {
-    // ------------- softmax groups: warps 2-5 (group 0), 6-9 (group 1) -------------
-    const int grp = (warp - 2) >> 2;
+    // ---------------- softmax / epilogue (warps 2-5) ----------------
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // TMEM lane = tile row
     const int half = row >> 6;
     const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tSg = tS + grp * 64 + lane_off;
-    const uint32_t tOg = tO + grp * 64 + lane_off;
+    const uint32_t tO = tmem + kColO + lane_off;
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
-    uint32_t cnt = 0;
+    uint32_t u = 0;  // tile counter (same sequence as the MMA warp)
     for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
@@ -254,52 +255,66 @@ __global__ void __launch_bounds__(kThreads, 2)
       const ItemList& L = lists[slot];
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
-      int nt = 0;
       bool ok = true;
-      for (int t = grp; t < n; t += 2, ++cnt, ++nt) {
-        if (!mbar_wait(&bars.s_full[grp], cnt & 1, &abort_flag, p.status)) {
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
+        const uint32_t par = (uu >> 1) & 1;
+        const bool att = (L.mask[t] & hbit) != 0;
+        if (!mbar_wait(&bars.s_full[b2], par, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const bool att = (L.mask[t] & hbit) != 0;
+        float z[64];
         if (att) {
-          // Two passes over the S tile in TMEM, 16 columns at a time, so
-          // few registers stay live: pass 1 takes the row max, pass 2 the
-          // exponentials, their sum and the bf16 P written back over S.
-          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
-          const bool plain = (kb == ~0ull) && c > 0.f;
-          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t s0[32], s1[32];
+          tmem_ld32(tmem + kColS + b2 * 64 + lane_off, s0);
+          tmem_ld32(tmem + kColS + b2 * 64 + 32 + lane_off, s1);
+          tmem_ld_wait();
 #pragma unroll
-          for (int q16 = 0; q16 < 4; ++q16) {
-            uint32_t r[16];
-            tmem_ld16(tSg + q16 * 16, r);
-            tmem_ld_wait();
-            if (plain) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e)
-                mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(r[e]));
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int col = q16 * 16 + e;
-                mx4[e & 3] = fmaxf(mx4[e & 3],
-                                   fmaf(__uint_as_float(r[e]), c,
-                                        ((kb >> col) & 1ull) ? 0.f : mvl));
-              }
-            }
+          for (int e = 0; e < 32; ++e) {
+            z[e] = __uint_as_float(s0[e]);
+            z[32 + e] = __uint_as_float(s1[e]);
           }
-          float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-          if (plain) mx *= c;
-          // Lazy running max: move it only when the row's max exceeds it by
+        }
+        // S is in registers: its buffer may take the next tile's scores.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_empty[b2]);
+        // P buffer b2 is free once the P V two tiles back has completed.
+        if (!mbar_wait(&bars.p_empty[b2], par ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
+        if (att) {
+          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          float mx;
+          if (kb == ~0ull && c > 0.f) {
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
+            mx = max8(mx8) * c;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              z[e] = fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl);
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
+            mx = max8(mx8);
+          }
+          const bool scaled = !(kb == ~0ull && c > 0.f);
+          // Lazy running max: move it only when the row max exceeds it by
           // more than the threshold (or on the row's first attended tile).
           const bool first = (m == -INFINITY);
           const bool need = !first && mx > m + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
-            // O holds this group's earlier tiles: wait for the last P V,
-            // then scale O by 2^(m_old - m_new) on the rows that move.
-            if (!mbar_wait(&bars.pv_done[grp], (cnt - 1) & 1, &abort_flag,
-                           p.status)) {
+            // O holds earlier tiles: wait for the last P V, then scale O by
+            // 2^(m_old - m_new) on the rows that move.
+            if (!mbar_wait(&bars.pv_done, (uu - 1) & 1, &abort_flag, p.status)) {
               ok = false;
               break;
             }
@@ -308,12 +323,12 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int q16 = 0; q16 < 4; ++q16) {
               uint32_t o[16];
-              tmem_ld16(tOg + q16 * 16, o);
+              tmem_ld16(tO + q16 * 16, o);
               tmem_ld_wait();
 #pragma unroll
               for (int e = 0; e < 16; ++e)
                 o[e] = __float_as_uint(__uint_as_float(o[e]) * al);
-              tmem_st16(tOg + q16 * 16, o);
+              tmem_st16(tO + q16 * 16, o);
             }
             tmem_st_wait();
             if (need) {
@@ -322,115 +337,87 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
           if (first) m = mx;
+          float sum8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+          const float cc = scaled ? 1.f : c;
           const float nm = -m;
-          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int q16 = 0; q16 < 4; ++q16) {
-            uint32_t r[16], Pq[8];
-            tmem_ld16(tSg + q16 * 16, r);
-            tmem_ld_wait();
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t Ph[16];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              float z0, z1;
-              if (plain) {
-                z0 = fmaf(__uint_as_float(r[e]), c, nm);
-                z1 = fmaf(__uint_as_float(r[e + 1]), c, nm);
-              } else {
-                const int col = q16 * 16 + e;
-                z0 = fmaf(__uint_as_float(r[e]), c,
-                          (((kb >> col) & 1ull) ? 0.f : mvl) + nm);
-                z1 = fmaf(__uint_as_float(r[e + 1]), c,
-                          (((kb >> (col + 1)) & 1ull) ? 0.f : mvl) + nm);
-              }
-              const float p0 = ex2(z0), p1 = ex2(z1);
-              sum4[(e >> 1) & 3] += p0 + p1;
-              Pq[e >> 1] = pack_bf16(p0, p1);
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2(fmaf(z[32 * hh + e], cc, nm));
+              const float p1 = ex2(fmaf(z[32 * hh + e + 1], cc, nm));
+              sum8[(e >> 1) & 7] += p0 + p1;
+              Ph[e >> 1] = pack_bf16(p0, p1);
             }
-            tmem_st8(tSg + q16 * 8, Pq);
+            tmem_st16(tP + 16 * hh, Ph);
           }
-          l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+          l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+               ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         } else {
           uint32_t Z[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) Z[e] = 0u;
-          tmem_st16(tSg, Z);
-          tmem_st16(tSg + 16, Z);
+          tmem_st16(tP, Z);
+          tmem_st16(tP + 16, Z);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[grp]);
+        if (lane == 0) mbar_arrive(&bars.p_full[b2]);
       }
       if (!ok) break;
-      // Wait for this group's last P V to land in its O accumulator.
-      if (nt > 0 &&
-          !mbar_wait(&bars.pv_done[grp], (cnt - 1) & 1, &abort_flag, p.status))
-        break;
+      u += n;
+      // Wait for the item's last P V, then normalise O and write it.
+      if (!mbar_wait(&bars.pv_done, (u - 1) & 1, &abort_flag, p.status)) break;
       tc_fence_after();
-      if (grp == 1) {
-        xch[slot][row] = make_float2(m, l);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.xch_full[slot]);
-      } else {
-        if (!mbar_wait(&bars.xch_full[slot], ph, &abort_flag, p.status)) break;
-        tc_fence_after();
-        const float2 ml1 = xch[slot][row];
-        const bool use0 = l > 0.f;
-        const bool use1 = n >= 2 && ml1.y > 0.f;
-        const float M = fmaxf(use0 ? m : -INFINITY, use1 ? ml1.x : -INFINITY);
-        const float w0 = use0 ? ex2(m - M) : 0.f;
-        const float w1 = use1 ? ex2(ml1.x - M) : 0.f;
-        const float Ls = l * w0 + ml1.y * w1;
-        const int blk = L.blk[half];
-        const int r64 = row & 63;
-        const bool write = blk >= 0;
-        const float inv = L.global ? 1.f : 1.f / Ls;
-        const float a0 = w0 * inv, a1 = w1 * inv;
-        const size_t grow = (size_t)L.bh * p.L + (size_t)(write ? blk : 0) * kBS + r64;
-        float* part = p.part + (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) *
-                                   kPartStride;
+      const int blk = L.blk[half];
+      const int r64 = row & 63;
+      const bool write = blk >= 0;
+      const float inv = L.global ? 1.f : 1.f / l;
+      const size_t grow = (size_t)L.bh * p.L + (size_t)(write ? blk : 0) * kBS + r64;
+      float* part = p.part +
+                    (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) * kPartStride;
 #pragma unroll
-        for (int q16 = 0; q16 < 4; ++q16) {
-          uint32_t o0[16], o1[16];
-          tmem_ld16(tO + lane_off + q16 * 16, o0);
-          if (n >= 2) tmem_ld16(tO + 64 + lane_off + q16 * 16, o1);
-          tmem_ld_wait();
+      for (int q16 = 0; q16 < 4; ++q16) {
+        uint32_t o[16];
+        tmem_ld16(tO + q16 * 16, o);
+        tmem_ld_wait();
+        if (write) {
           float v[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            v[e] = (use0 ? __uint_as_float(o0[e]) * a0 : 0.f) +
-                   (use1 ? __uint_as_float(o1[e]) * a1 : 0.f);
-          if (write) {
-            if (!L.global) {
-              uint4* dst = reinterpret_cast<uint4*>(
-                  static_cast<__nv_bfloat16*>(p.out) + grow * kHeadDim + q16 * 16);
-              dst[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                  pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-              dst[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                                  pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
-            } else {
-              float4* dst = reinterpret_cast<float4*>(part + q16 * 16);
-#pragma unroll
-              for (int e = 0; e < 4; ++e)
-                dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.o_empty);
-        if (write) {
+          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(o[e]) * inv;
           if (!L.global) {
-            p.lse_out[grow] = (M + __log2f(Ls)) * (1.0f / kLog2e);
+            uint4* dst = reinterpret_cast<uint4*>(
+                static_cast<__nv_bfloat16*>(p.out) + grow * kHeadDim + q16 * 16);
+            dst[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            dst[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                                pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
           } else {
-            part[64] = M;
-            part[65] = Ls;
+            float4* dst = reinterpret_cast<float4*>(part + q16 * 16);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
           }
         }
       }
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+      if (lane == 0) {
+        mbar_arrive(&bars.o_empty);
+        mbar_arrive(&bars.list_empty[slot]);
+      }
+      if (write) {
+        if (!L.global) {
+          p.lse_out[grow] = (m + __log2f(l)) * (1.0f / kLog2e);
+        } else {
+          part[64] = m;
+          part[65] = l;
+        }
+      }
     }
   }
 

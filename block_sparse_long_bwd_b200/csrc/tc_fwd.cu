@@ -24,28 +24,33 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kNST = 2;           // K/V stages
+constexpr int kNST = 4;
 constexpr int kThreads = 192;
-constexpr int kCtasPerSm = 4;
-constexpr uint32_t kTmemCols = 128;
+constexpr uint32_t kTmemCols = 256;
 // Rescale threshold of the lazy running max (log2 units): the max used for
 // the exponent only moves when a row's true max exceeds it by more than
 // this, so probabilities stay below 2^8 and O is rarely rescaled.
 constexpr float kRescaleThreshold = 8.0f;
 
-// TMEM columns: S (fp32, 64) with P (bf16 pairs, 32) written over its first
-// half once read, and O (fp32, 64) accumulated by the P V MMAs.  A CTA keeps
-// one tile in flight; four CTAs per SM overlap each other's MMA, softmax and
-// load latencies.
-constexpr uint32_t kColS = 0, kColO = 64;
+// TMEM columns: S[2] (fp32, 64 each), P[2] (bf16 pairs, 32 each), O (fp32).
+// S, P and O are separate so the next S can be computed as soon as the
+// softmax has read the current one, and P V accumulates straight into O.
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct Bars {
-  uint64_t list_full[2], list_empty[2], q_full, q_empty;
+  uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
   uint64_t kv_full[kNST], kv_empty[kNST];
-  uint64_t s_full, s_free, p_full, pv_done, o_empty;
+  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
+  uint64_t pv_done, o_empty;
 };
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+__device__ __forceinline__ float max8(const float* z) {
+  const float a = fmaxf(z[0], z[1]), b = fmaxf(z[2], z[3]);
+  const float c = fmaxf(z[4], z[5]), d = fmaxf(z[6], z[7]);
+  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
     tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK,
@@ -60,26 +65,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* Qs = base;                    // [128][64] bf16
-  uint8_t* KVs = base + 2 * kTileBytes;  // [kNST][K, V][64][64] bf16
+  uint8_t* Qs = base;                        // [2][128][64] bf16
+  uint8_t* KVs = base + 2 * 2 * kTileBytes;  // [kNST][K, V][64][64] bf16
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.list_full[s], 1);
       mbar_init(&bars.list_empty[s], 5);
+      mbar_init(&bars.q_full[s], 1);
+      mbar_init(&bars.q_empty[s], 1);
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_empty[s], 4);
+      mbar_init(&bars.p_full[s], 4);
+      mbar_init(&bars.p_empty[s], 1);
     }
-    mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_empty, 1);
+    mbar_init(&bars.pv_done, 1);
+    mbar_init(&bars.o_empty, 4);
     for (int s = 0; s < kNST; ++s) {
       mbar_init(&bars.kv_full[s], 1);
       mbar_init(&bars.kv_empty[s], 1);
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_free, 1);
-    mbar_init(&bars.p_full, 4);
-    mbar_init(&bars.pv_done, 1);
-    mbar_init(&bars.o_empty, 4);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -100,8 +106,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       uint32_t g = 0;
-      int qissued = 0;
-      uint32_t qpar = 0;
+      int qissued[2] = {0, 0};
+      uint32_t qpar[2] = {0, 0};
       for (int k = 0, item = blockIdx.x; item < a.items;
            ++k, item += gridDim.x) {
         const int slot = k & 1;
@@ -111,16 +117,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         ItemList& L = lists[slot];
         build_pair_item(a, item, L);
         mbar_arrive(&bars.list_full[slot]);
-        if (!mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
+          break;
         const int row0 = L.bh * p.L;
         const uint32_t qbytes = (L.blk[1] >= 0 ? 2u : 1u) * kTileBytes;
-        mbar_expect_tx(&bars.q_full, qbytes);
-        tma_load_2d(Qs, &tmQ, &bars.q_full, 0, row0 + L.blk[0] * kBS);
+        mbar_expect_tx(&bars.q_full[slot], qbytes);
+        uint8_t* q = Qs + slot * 2 * kTileBytes;
+        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.blk[0] * kBS);
         if (L.blk[1] >= 0)
-          tma_load_2d(Qs + kTileBytes, &tmQ, &bars.q_full, 0,
+          tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
                       row0 + L.blk[1] * kBS);
-        qissued = 1;
-        qpar = k & 1;
+        qissued[slot] = 1;
+        qpar[slot] = ph;
         bool ok = true;
         for (int t = 0; t < L.n; ++t) {
           const int st = g % kNST;
@@ -149,9 +157,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                  globaltimer() - t0 < 100000000ull) {
           }
         }
-        if (qissued) {
+        for (int s = 0; s < 2; ++s) {
+          if (!qissued[s]) continue;
           const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(&bars.q_full, qpar) &&
+          while (!mbar_try_wait(&bars.q_full[s], qpar[s]) &&
                  globaltimer() - t0 < 100000000ull) {
           }
         }
@@ -159,58 +168,89 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
+    // Two cursors over the stream of tiles (items back to back): S runs up
+    // to two tiles ahead of P V, so S(u + 2) is issued as soon as the
+    // softmax has read S(u), and P V(u) as soon as P(u) is written.  S may
+    // run into the next item (its list and Q are double-buffered) but never
+    // two items ahead, whose list slot is still held by the P V cursor.
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
-    const uint32_t qaddr = smem_u32(Qs);
-    uint32_t g = 0, u = 0;  // K/V stage counter, tile counter
+    int kS = 0, itemS = blockIdx.x, tS = 0, nS = -1;  // S cursor
+    int kP = 0, tP = 0;                               // P V cursor
+    uint32_t uS = 0, uP = 0;                          // global tile indices
     bool ok = true;
-    for (int k = 0, item = blockIdx.x; item < a.items && ok;
-         ++k, item += gridDim.x) {
-      const int slot = k & 1;
-      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
-        break;
-      const int n = lists[slot].n;
-      if (!mbar_wait(&bars.q_full, k & 1, &abort_flag, p.status)) break;
-      tc_fence_after();
-      for (int t = 0; t < n; ++t, ++g, ++u) {
-        const int st = g % kNST;
-        // S may be overwritten once the previous tile's P V has consumed P.
-        if (!mbar_wait(&bars.kv_full[st], (g / kNST) & 1, &abort_flag, p.status) ||
-            !mbar_wait(&bars.s_free, (u & 1) ^ 1, &abort_flag, p.status)) {
+    while (ok) {
+      // ---- S for as many tiles as allowed ----
+      while (ok && uS < uP + 2 && itemS < a.items && kS <= kP + 1) {
+        const int slot = kS & 1;
+        if (tS == 0) {
+          if (!mbar_wait(&bars.list_full[slot], (kS >> 1) & 1, &abort_flag, p.status) ||
+              !mbar_wait(&bars.q_full[slot], (kS >> 1) & 1, &abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
+          nS = lists[slot].n;
+        }
+        const int b2 = uS & 1;
+        const int st = uS % kNST;
+        if (!mbar_wait(&bars.kv_full[st], (uS / kNST) & 1, &abort_flag, p.status) ||
+            !mbar_wait(&bars.s_empty[b2], ((uS >> 1) & 1) ^ 1, &abort_flag,
+                       p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
         if (lane == 0) {
+          const uint32_t qaddr = smem_u32(Qs + slot * 2 * kTileBytes);
+          const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kColS, sdesc_sw128(qaddr + kk * 32, 16),
+            mma_ss(tmem + kColS + b2 * 64, sdesc_sw128(qaddr + kk * 32, 16),
                    sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
-          mma_commit(&bars.s_full);
-          if (t == n - 1) mma_commit(&bars.q_empty);
+          mma_commit(&bars.s_full[b2]);
+          if (tS == nS - 1) mma_commit(&bars.q_empty[slot]);
         }
         __syncwarp();
-        if (!mbar_wait(&bars.p_full, u & 1, &abort_flag, p.status) ||
-            (t == 0 &&
-             !mbar_wait(&bars.o_empty, (k & 1) ^ 1, &abort_flag, p.status))) {
+        ++uS;
+        if (++tS == nS) {
+          tS = 0;
+          ++kS;
+          itemS += gridDim.x;
+        }
+      }
+      if (!ok || uP == uS) break;  // nothing left for P V
+      // ---- P V of tile uP ----
+      {
+        const int slot = kP & 1;
+        const int nP = lists[slot].n;
+        const int b2 = uP & 1;
+        const int st = uP % kNST;
+        if (!mbar_wait(&bars.p_full[b2], (uP >> 1) & 1, &abort_flag, p.status) ||
+            (tP == 0 &&
+             !mbar_wait(&bars.o_empty, (kP & 1) ^ 1, &abort_flag, p.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
+          const uint32_t vaddr = smem_u32(KVs + st * 2 * kTileBytes + kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + kColO, tmem + kColS + kk * 8,
-                   sdesc_sw128(kaddr + kTileBytes + kk * 2048, 8192), idPV,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + kColO, tmem + kColP + b2 * 32 + kk * 8,
+                   sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
+                   (tP > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.pv_done);
-          mma_commit(&bars.s_free);
+          mma_commit(&bars.p_empty[b2]);
           mma_commit(&bars.kv_empty[st]);
         }
         __syncwarp();
+        ++uP;
+        if (++tP == nP) {
+          tP = 0;
+          if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+          ++kP;
+        }
       }
-      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
     }
   } else {
     // ---------------- softmax / epilogue (warps 2-5) ----------------
@@ -219,68 +259,81 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int half = row >> 6;
     const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-    const uint32_t tS = tmem + kColS + lane_off;
     const uint32_t tO = tmem + kColO + lane_off;
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;  // tile counter (same sequence as the MMA warp)
     for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
       const int slot = k & 1;
-      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
-        break;
+      const uint32_t ph = (k >> 1) & 1;
+      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
       const ItemList& L = lists[slot];
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
-      for (int t = 0; t < n; ++t, ++u) {
-        if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
+        const uint32_t par = (uu >> 1) & 1;
+        const bool att = (L.mask[t] & hbit) != 0;
+        if (!mbar_wait(&bars.s_full[b2], par, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const bool att = (L.mask[t] & hbit) != 0;
+        float z[64];
         if (att) {
-          // Two passes over S in TMEM, 16 columns at a time (few live
-          // registers): the row max, then the exponentials, their sum and
-          // the bf16 P written back over the first half of S.
-          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
-          const bool plain = (kb == ~0ull) && c > 0.f;
-          float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t s0[32], s1[32];
+          tmem_ld32(tmem + kColS + b2 * 64 + lane_off, s0);
+          tmem_ld32(tmem + kColS + b2 * 64 + 32 + lane_off, s1);
+          tmem_ld_wait();
 #pragma unroll
-          for (int q32 = 0; q32 < 2; ++q32) {
-            uint32_t r0[16], r1[16];
-            tmem_ld16(tS + q32 * 32, r0);
-            tmem_ld16(tS + q32 * 32 + 16, r1);
-            tmem_ld_wait();
-            if (plain) {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                mx4[e & 3] = fmaxf(mx4[e & 3], __uint_as_float(r0[e]));
-                mx4[(e + 2) & 3] = fmaxf(mx4[(e + 2) & 3], __uint_as_float(r1[e]));
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const int col = q32 * 32 + e;
-                mx4[e & 3] = fmaxf(mx4[e & 3],
-                                   fmaf(__uint_as_float(r0[e]), c,
-                                        ((kb >> col) & 1ull) ? 0.f : mvl));
-                mx4[(e + 2) & 3] =
-                    fmaxf(mx4[(e + 2) & 3],
-                          fmaf(__uint_as_float(r1[e]), c,
-                               ((kb >> (col + 16)) & 1ull) ? 0.f : mvl));
-              }
-            }
+          for (int e = 0; e < 32; ++e) {
+            z[e] = __uint_as_float(s0[e]);
+            z[32 + e] = __uint_as_float(s1[e]);
           }
-          float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-          if (plain) mx *= c;
+        }
+        // S is in registers: its buffer may take the next tile's scores.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_empty[b2]);
+        // P buffer b2 is free once the P V two tiles back has completed.
+        if (!mbar_wait(&bars.p_empty[b2], par ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
+        if (att) {
+          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          float mx;
+          if (kb == ~0ull && c > 0.f) {
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
+            mx = max8(mx8) * c;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              z[e] = fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl);
+            float mx8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
+            mx = max8(mx8);
+          }
+          const bool scaled = !(kb == ~0ull && c > 0.f);
           // Lazy running max: move it only when the row max exceeds it by
           // more than the threshold (or on the row's first attended tile).
-          // O is complete up to the previous tile (its P V finished before
-          // this tile's S was computed), so it can be rescaled in place.
           const bool first = (m == -INFINITY);
           const bool need = !first && mx > m + kRescaleThreshold;
           if (__any_sync(0xffffffffu, need)) {
+            // O holds earlier tiles: wait for the last P V, then scale O by
+            // 2^(m_old - m_new) on the rows that move.
+            if (!mbar_wait(&bars.pv_done, (uu - 1) & 1, &abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             const float al = need ? ex2(m - mx) : 1.f;
 #pragma unroll
             for (int q16 = 0; q16 < 4; ++q16) {
@@ -299,46 +352,39 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
           }
           if (first) m = mx;
+          float sum8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+          const float cc = scaled ? 1.f : c;
           const float nm = -m;
-          float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int q16 = 0; q16 < 4; ++q16) {
-            uint32_t r[16], Pq[8];
-            tmem_ld16(tS + q16 * 16, r);
-            tmem_ld_wait();
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t Ph[16];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              float z0, z1;
-              if (plain) {
-                z0 = fmaf(__uint_as_float(r[e]), c, nm);
-                z1 = fmaf(__uint_as_float(r[e + 1]), c, nm);
-              } else {
-                const int col = q16 * 16 + e;
-                z0 = fmaf(__uint_as_float(r[e]), c,
-                          (((kb >> col) & 1ull) ? 0.f : mvl) + nm);
-                z1 = fmaf(__uint_as_float(r[e + 1]), c,
-                          (((kb >> (col + 1)) & 1ull) ? 0.f : mvl) + nm);
-              }
-              const float p0 = ex2(z0), p1 = ex2(z1);
-              sum4[(e >> 1) & 3] += p0 + p1;
-              Pq[e >> 1] = pack_bf16(p0, p1);
+            for (int e = 0; e < 32; e += 2) {
+              const float p0 = ex2(fmaf(z[32 * hh + e], cc, nm));
+              const float p1 = ex2(fmaf(z[32 * hh + e + 1], cc, nm));
+              sum8[(e >> 1) & 7] += p0 + p1;
+              Ph[e >> 1] = pack_bf16(p0, p1);
             }
-            tmem_st8(tS + q16 * 8, Pq);
+            tmem_st16(tP + 16 * hh, Ph);
           }
-          l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+          l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+               ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
         } else {
           uint32_t Z[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) Z[e] = 0u;
-          tmem_st16(tS, Z);
-          tmem_st16(tS + 16, Z);
+          tmem_st16(tP, Z);
+          tmem_st16(tP + 16, Z);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full);
+        if (lane == 0) mbar_arrive(&bars.p_full[b2]);
       }
       if (!ok) break;
+      u += n;
       // Wait for the item's last P V, then normalise O and write it.
       if (!mbar_wait(&bars.pv_done, (u - 1) & 1, &abort_flag, p.status)) break;
       tc_fence_after();
@@ -447,14 +493,14 @@ bool tc_fwd_supported(const Problem& p) { return tc_shape_ok(p); }
 cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
   const PairArgs a = make_pair_args(p);
-  const size_t smem = 1024 + (2 + 2 * kNST) * kTileBytes;
+  const size_t smem = 1024 + (2 * 2 + 2 * kNST) * kTileBytes;
   cudaError_t e = cudaFuncSetAttribute(
       tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = min(a.items, kCtasPerSm * sms);
+  const int grid = min(a.items, 2 * sms);
   tc_fwd_kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

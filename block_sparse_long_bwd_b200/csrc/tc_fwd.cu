@@ -41,7 +41,10 @@ struct Bars {
   uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
   uint64_t kv_full[kNST], kv_empty[kNST];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
-  uint64_t pv_done, o_empty;
+  // One P V completion barrier per P buffer: P V(u) commits to
+  // pv_done[u & 1], so a wait for P V(u) by parity is never confused with
+  // P V(u - 1), which may still be in flight.
+  uint64_t pv_done[2], o_empty;
 };
 
 __device__ __forceinline__ float max8(const float* z) {
@@ -79,8 +82,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.s_empty[s], 4);
       mbar_init(&bars.p_full[s], 4);
       mbar_init(&bars.p_empty[s], 1);
+      mbar_init(&bars.pv_done[s], 1);
     }
-    mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_empty, 4);
     for (int s = 0; s < kNST; ++s) {
       mbar_init(&bars.kv_full[s], 1);
@@ -239,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             mma_ts(tmem + kColO, tmem + kColP + b2 * 32 + kk * 8,
                    sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
                    (tP > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars.pv_done);
+          mma_commit(&bars.pv_done[b2]);
           mma_commit(&bars.p_empty[b2]);
           mma_commit(&bars.kv_empty[st]);
         }
@@ -329,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (__any_sync(0xffffffffu, need)) {
             // O holds earlier tiles: wait for the last P V, then scale O by
             // 2^(m_old - m_new) on the rows that move.
-            if (!mbar_wait(&bars.pv_done, (uu - 1) & 1, &abort_flag, p.status)) {
+            if (!mbar_wait(&bars.pv_done[(uu - 1) & 1], ((uu - 1) >> 1) & 1,
+                           &abort_flag, p.status)) {
               ok = false;
               break;
             }
@@ -386,7 +390,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!ok) break;
       u += n;
       // Wait for the item's last P V, then normalise O and write it.
-      if (!mbar_wait(&bars.pv_done, (u - 1) & 1, &abort_flag, p.status)) break;
+      if (!mbar_wait(&bars.pv_done[(u - 1) & 1], ((u - 1) >> 1) & 1, &abort_flag,
+                     p.status))
+        break;
       tc_fence_after();
       const int blk = L.blk[half];
       const int r64 = row & 63;

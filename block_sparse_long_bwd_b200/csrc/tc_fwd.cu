@@ -213,11 +213,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     // Two cursors over the stream of tiles (items back to back): S(u + 2)
-    // is issued as soon as the softmax has read S(u) (the S buffer is free
-    // then; P lives elsewhere), even before P V(u) is issued, and P V(u) as
-    // soon as P(u) is written.  S may run into the next item (its list and
-    // Q are double-buffered) but never two items ahead, whose list slot is
-    // still held by the P V cursor.
+    // is issued right after P V(u), and P V(u) as soon as P(u) is written.
+    // (An MMA issue blocks while the tensor core's queue is full, so S is
+    // kept only one batch ahead: running it further ahead delays the P V the
+    // softmax waits on.)  S may run into the next item (its list and Q are
+    // double-buffered) but never two items ahead, whose list slot is still
+    // held by the P V cursor.
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
     int kS = 0, itemS = blockIdx.x, tS = 0, nS = -1;  // S cursor
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
     while (ok) {
       // ---- S for as many tiles as allowed ----
-      while (ok && uS < uP + 3 && itemS < a.items && kS <= kP + 1) {
+      while (ok && uS < uP + 2 && itemS < a.items && kS <= kP + 1) {
         const int slot = kS & 1;
         if (tS == 0) {
           if (!mbar_wait(&bars.list_full[slot], (kS >> 1) & 1, &abort_flag, p.status) ||

@@ -39,10 +39,7 @@ constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct Bars {
   uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
-  // K and V tiles sit in separate rings: a K stage is freed when its S
-  // MMA completes, a V stage when its P V completes, so K loads run ahead
-  // of the P V chain.
-  uint64_t k_full[kNST], k_empty[kNST], v_full[kNST], v_empty[kNST];
+  uint64_t kv_full[kNST], kv_empty[kNST];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   // One P V completion barrier per P buffer: P V(u) commits to
   // pv_done[u & 1], so a wait for P V(u) by parity is never confused with
@@ -72,8 +69,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* Qs = base;                        // [2][128][64] bf16
-  uint8_t* Ks = base + 2 * 2 * kTileBytes;        // [kNST][64][64] bf16
-  uint8_t* Vs = Ks + kNST * kTileBytes;             // [kNST][64][64] bf16
+  uint8_t* KVs = base + 2 * 2 * kTileBytes;  // [kNST][K, V][64][64] bf16
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
@@ -90,10 +86,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     mbar_init(&bars.o_empty, 4);
     for (int s = 0; s < kNST; ++s) {
-      mbar_init(&bars.k_full[s], 1);
-      mbar_init(&bars.k_empty[s], 1);
-      mbar_init(&bars.v_full[s], 1);
-      mbar_init(&bars.v_empty[s], 1);
+      mbar_init(&bars.kv_full[s], 1);
+      mbar_init(&bars.kv_empty[s], 1);
     }
     fence_mbar_init();
   }
@@ -113,92 +107,57 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
-    // Two cursors: K loads run up to two tiles ahead of V loads (and at
-    // most one item ahead, whose list slot is still held otherwise).
     if (lane == 0) {
-      int kK = 0, itemK = blockIdx.x, tK = 0, nK = 0, row0K = 0;
-      int kV = 0, tV = 0;
-      uint32_t uK = 0, uV = 0;
+      uint32_t g = 0;
       int qissued[2] = {0, 0};
       uint32_t qpar[2] = {0, 0};
-      bool ok = true;
-      while (ok) {
-        while (ok && uK < uV + 3 && itemK < a.items && kK <= kV + 1) {
-          const int slot = kK & 1;
-          const uint32_t ph = (kK >> 1) & 1;
-          if (tK == 0) {
-            if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            ItemList& L = lists[slot];
-            build_pair_item(a, itemK, L);
-            mbar_arrive(&bars.list_full[slot]);
-            nK = L.n;
-            row0K = L.bh * p.L;
-            if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t qbytes = (L.blk[1] >= 0 ? 2u : 1u) * kTileBytes;
-            mbar_expect_tx(&bars.q_full[slot], qbytes);
-            uint8_t* q = Qs + slot * 2 * kTileBytes;
-            tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0K + L.blk[0] * kBS);
-            if (L.blk[1] >= 0)
-              tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
-                          row0K + L.blk[1] * kBS);
-            qissued[slot] = 1;
-            qpar[slot] = ph;
-          }
-          const int st = uK % kNST;
-          if (!mbar_wait(&bars.k_empty[st], ((uK / kNST) & 1) ^ 1, &abort_flag,
-                         p.status)) {
+      for (int k = 0, item = blockIdx.x; item < a.items;
+           ++k, item += gridDim.x) {
+        const int slot = k & 1;
+        const uint32_t ph = (k >> 1) & 1;
+        if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
+          break;
+        ItemList& L = lists[slot];
+        build_pair_item(a, item, L);
+        mbar_arrive(&bars.list_full[slot]);
+        if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
+          break;
+        const int row0 = L.bh * p.L;
+        const uint32_t qbytes = (L.blk[1] >= 0 ? 2u : 1u) * kTileBytes;
+        mbar_expect_tx(&bars.q_full[slot], qbytes);
+        uint8_t* q = Qs + slot * 2 * kTileBytes;
+        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.blk[0] * kBS);
+        if (L.blk[1] >= 0)
+          tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
+                      row0 + L.blk[1] * kBS);
+        qissued[slot] = 1;
+        qpar[slot] = ph;
+        bool ok = true;
+        for (int t = 0; t < L.n; ++t) {
+          const int st = g % kNST;
+          const uint32_t kph = (g / kNST) & 1;
+          if (!mbar_wait(&bars.kv_empty[st], kph ^ 1, &abort_flag, p.status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&bars.k_full[st], kTileBytes);
-          tma_load_2d(Ks + st * kTileBytes, &tmK, &bars.k_full[st], 0,
-                      row0K + lists[slot].tile[tK] * kBS);
-          ++uK;
-          if (++tK == nK) {
-            tK = 0;
-            ++kK;
-            itemK += gridDim.x;
-          }
+          mbar_expect_tx(&bars.kv_full[st], 2 * kTileBytes);
+          uint8_t* kv = KVs + st * 2 * kTileBytes;
+          const int y = row0 + L.tile[t] * kBS;
+          tma_load_2d(kv, &tmK, &bars.kv_full[st], 0, y);
+          tma_load_2d(kv + kTileBytes, &tmV, &bars.kv_full[st], 0, y);
+          ++g;
         }
-        if (!ok || uV == uK) break;
-        const int slot = kV & 1;
-        const ItemList& L = lists[slot];
-        const int st = uV % kNST;
-        if (!mbar_wait(&bars.v_empty[st], ((uV / kNST) & 1) ^ 1, &abort_flag,
-                       p.status))
-          break;
-        mbar_expect_tx(&bars.v_full[st], kTileBytes);
-        tma_load_2d(Vs + st * kTileBytes, &tmV, &bars.v_full[st], 0,
-                    L.bh * p.L + L.tile[tV] * kBS);
-        ++uV;
-        if (++tV == L.n) {
-          tV = 0;
-          ++kV;
-        }
+        if (!ok) break;
       }
       if (abort_flag) {
         // Let issued copies land before the CTA's shared memory goes away:
         // wait (bounded) for the phase of the last load into each buffer.
         for (uint32_t s = 0; s < (uint32_t)kNST; ++s) {
-          if (uK >= s + 1) {
-            const uint32_t last = uK - 1 - ((uK - 1 - s) % kNST);
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(&bars.k_full[s], (last / kNST) & 1) &&
-                   globaltimer() - t0 < 100000000ull) {
-            }
-          }
-          if (uV >= s + 1) {
-            const uint32_t last = uV - 1 - ((uV - 1 - s) % kNST);
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(&bars.v_full[s], (last / kNST) & 1) &&
-                   globaltimer() - t0 < 100000000ull) {
-            }
+          if (g < s + 1) continue;
+          const uint32_t last = g - 1 - ((g - 1 - s) % kNST);
+          const uint64_t t0 = globaltimer();
+          while (!mbar_try_wait(&bars.kv_full[s], (last / kNST) & 1) &&
+                 globaltimer() - t0 < 100000000ull) {
           }
         }
         for (int s = 0; s < 2; ++s) {
@@ -212,93 +171,74 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
-    // Two cursors over the stream of tiles (items back to back): S(u + 2)
-    // is issued right after P V(u), and P V(u) as soon as P(u) is written.
-    // (An MMA issue blocks while the tensor core's queue is full, so S is
-    // kept only one batch ahead: running it further ahead delays the P V the
-    // softmax waits on.)  S may run into the next item (its list and Q are
-    // double-buffered) but never two items ahead, whose list slot is still
-    // held by the P V cursor.
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
-    int kS = 0, itemS = blockIdx.x, tS = 0, nS = -1;  // S cursor
-    int kP = 0, tP = 0;                               // P V cursor
-    uint32_t uS = 0, uP = 0;                          // global tile indices
+    uint32_t g = 0, u = 0;  // K/V stage counter, tile counter
     bool ok = true;
-    while (ok) {
-      // ---- S for as many tiles as allowed ----
-      while (ok && uS < uP + 2 && itemS < a.items && kS <= kP + 1) {
-        const int slot = kS & 1;
-        if (tS == 0) {
-          if (!mbar_wait(&bars.list_full[slot], (kS >> 1) & 1, &abort_flag, p.status) ||
-              !mbar_wait(&bars.q_full[slot], (kS >> 1) & 1, &abort_flag, p.status)) {
-            ok = false;
-            break;
-          }
-          nS = lists[slot].n;
+    for (int k = 0, item = blockIdx.x; item < a.items && ok;
+         ++k, item += gridDim.x) {
+      const int slot = k & 1;
+      const uint32_t ph = (k >> 1) & 1;
+      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      const int n = lists[slot].n;
+      if (!mbar_wait(&bars.q_full[slot], ph, &abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t qaddr = smem_u32(Qs + slot * 2 * kTileBytes);
+      // P V of tile t into O.
+      auto issue_pv = [&](int t) -> bool {
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
+        const int st = (g + t) % kNST;
+        if (!mbar_wait(&bars.p_full[b2], (uu >> 1) & 1, &abort_flag, p.status))
+          return false;
+        if (t == 0 && !mbar_wait(&bars.o_empty, (k & 1) ^ 1, &abort_flag, p.status))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t vaddr = smem_u32(KVs + st * 2 * kTileBytes + kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tmem + kColO, tmem + kColP + b2 * 32 + kk * 8,
+                   sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.pv_done[b2]);
+          mma_commit(&bars.p_empty[b2]);
+          mma_commit(&bars.kv_empty[st]);
         }
-        const int b2 = uS & 1;
-        const int st = uS % kNST;
-        if (!mbar_wait(&bars.k_full[st], (uS / kNST) & 1, &abort_flag, p.status) ||
-            !mbar_wait(&bars.s_empty[b2], ((uS >> 1) & 1) ^ 1, &abort_flag,
+        __syncwarp();
+        return true;
+      };
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t;
+        const int b2 = uu & 1;
+        const int st = (g + t) % kNST;
+        if (!mbar_wait(&bars.kv_full[st], ((g + t) / kNST) & 1, &abort_flag,
+                       p.status) ||
+            !mbar_wait(&bars.s_empty[b2], ((uu >> 1) & 1) ^ 1, &abort_flag,
                        p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t qaddr = smem_u32(Qs + slot * 2 * kTileBytes);
-          const uint32_t kaddr = smem_u32(Ks + st * kTileBytes);
+          const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tmem + kColS + b2 * 64, sdesc_sw128(qaddr + kk * 32, 16),
                    sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
           mma_commit(&bars.s_full[b2]);
-          mma_commit(&bars.k_empty[st]);
-          if (tS == nS - 1) mma_commit(&bars.q_empty[slot]);
+          if (t == n - 1) mma_commit(&bars.q_empty[slot]);
         }
         __syncwarp();
-        ++uS;
-        if (++tS == nS) {
-          tS = 0;
-          ++kS;
-          itemS += gridDim.x;
-        }
-      }
-      if (!ok || uP == uS) break;  // nothing left for P V
-      // ---- P V of tile uP ----
-      {
-        const int slot = kP & 1;
-        const int nP = lists[slot].n;
-        const int b2 = uP & 1;
-        const int st = uP % kNST;
-        if (!mbar_wait(&bars.p_full[b2], (uP >> 1) & 1, &abort_flag, p.status) ||
-            !mbar_wait(&bars.v_full[st], (uP / kNST) & 1, &abort_flag, p.status) ||
-            (tP == 0 &&
-             !mbar_wait(&bars.o_empty, (kP & 1) ^ 1, &abort_flag, p.status))) {
+        if (t > 0 && !issue_pv(t - 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t vaddr = smem_u32(Vs + st * kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tmem + kColO, tmem + kColP + b2 * 32 + kk * 8,
-                   sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
-                   (tP > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars.pv_done[b2]);
-          mma_commit(&bars.p_empty[b2]);
-          mma_commit(&bars.v_empty[st]);
-        }
-        __syncwarp();
-        ++uP;
-        if (++tP == nP) {
-          tP = 0;
-          if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
-          ++kP;
-        }
       }
+      if (ok && n > 0 && !issue_pv(n - 1)) ok = false;
+      g += n;
+      u += n;
+      if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
     }
   } else {
     // ---------------- softmax / epilogue (warps 2-5) ----------------

@@ -44,10 +44,16 @@ PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
                   "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 
-# DRAM bytes per launch from one ncu capture, keyed by kernel name, with the
-# sha256 of the source file the kernel was built from when captured.  A
-# mismatch (the kernel changed since) reports traffic as null.
-NCU_TRAFFIC = {}
+# DRAM bytes per launch from one ncu capture, keyed by kernel name: (bytes,
+# sha256 prefix of the kernel's source file when captured, that file, the
+# workload captured).  Another workload or a changed source reports null.
+NCU_TRAFFIC = {
+    # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, 1 launch)
+    "tc_dq": (168891136 + 33869312, "ad3192932ce3b04f", "tc_bwd.cu",
+               "large_train_l4096"),
+    "tc_dkdv": (136520960 + 62859264, "ad3192932ce3b04f", "tc_bwd.cu",
+                "large_train_l4096"),
+}
 
 
 def parse():
@@ -336,8 +342,9 @@ def run_ours(args, world, rank, local):
         peak, how = peaks["hbm_gbs"], "HBM copy"
     traffic = None
     tr = NCU_TRAFFIC.get(dom)
-    if tr is not None and tr[1] == src_hash(os.path.join(
-            ROOT, "block_sparse_long_bwd_b200", "csrc", tr[2])):
+    if (tr is not None and args.workload == tr[3] and
+            tr[1] == src_hash(os.path.join(ROOT, "block_sparse_long_bwd_b200",
+                                           "csrc", tr[2]))):
         traffic = tr[0]
     roofline = {"bound": bound, "achieved": round(achieved, 2),
                 "peak": round(peak, 1), "unit": unit,

@@ -81,6 +81,9 @@ def lib():
             [ctypes.POINTER(bb_attn_desc)] + [_P] * 12
             + [ctypes.c_size_t, _P, ctypes.POINTER(_P), ctypes.c_int])
         L.bb_attn_bwd_events.restype = ctypes.c_int
+        L.bb_attn_fwd_noalloc.argtypes = [ctypes.POINTER(bb_attn_desc)] + [
+            _P] * 8
+        L.bb_attn_fwd_noalloc.restype = ctypes.c_int
         L.bb_attn_check_status.argtypes = [_P, _P]
         L.bb_attn_check_status.restype = ctypes.c_int
         _lib = L
@@ -187,6 +190,24 @@ def bb_attn_fwd(desc, q, k, v, key_mask, rand_idx, out, lse, workspace,
     else:
         arr, n = _event_array(events)
         _check(lib().bb_attn_fwd_events(*args, arr, n), "bb_attn_fwd_events")
+
+
+def bb_attn_fwd_noalloc(desc, q, k, v, key_mask, rand_idx, out, lse,
+                        stream=None):
+    """Forward using the library's built-in scratch instead of a workspace
+    (for callers that cannot allocate; see include/bb_attn.h)."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _cuda_tensor(t, name, q.dtype)
+    _cuda_tensor(lse, "lse", torch.float32)
+    if key_mask is not None:
+        _cuda_tensor(key_mask, "key_mask", torch.uint8)
+    if rand_idx is not None:
+        _cuda_tensor(rand_idx, "rand_idx", torch.int32)
+    _check(lib().bb_attn_fwd_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k),
+                                     _ptr(v), _ptr(key_mask), _ptr(rand_idx),
+                                     _ptr(out), _ptr(lse),
+                                     _stream_ptr(stream)),
+           "bb_attn_fwd_noalloc")
 
 
 def bb_attn_bwd(desc, q, k, v, out, lse, dout, key_mask, rand_idx, dq, dk, dv,

@@ -162,6 +162,31 @@ BB_API int bb_attn_bwd_events(const bb_attn_desc* desc, const void* q,
                               size_t workspace_bytes, void* stream,
                               void* const* events, int num_events);
 
+/* Forward without a workspace, for callers that cannot allocate device
+ * memory (a runtime that reserves its whole memory budget at start-up and
+ * forbids later cudaMalloc, a plugin that must not bypass its host
+ * framework's allocator, a C caller with no spare buffer to lend).  The
+ * pages have no counterpart of this call: it is an interface convenience.
+ * Same arguments, results and kernels as bb_attn_fwd, except that the
+ * workspace is a 32 MiB scratch array built into the library, which every
+ * device that loads the library keeps until the process exits.  The caller
+ * still provides q, k, v, key_mask, rand_idx, out and lse.
+ *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating routine.
+ *  - The first call on a device looks up the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Returns BB_ERR_WORKSPACE, without launching anything, when the problem
+ *    needs more than 32 MiB of workspace (bb_attn_workspace_size(desc, 0)).
+ *  - Every call shares the one scratch array, which keeps the last call's
+ *    contents: calls that overlap on the GPU (other streams, other threads
+ *    on the same device) race; order them on one stream.  The device status
+ *    word lives in the scratch and is not reported by this call. */
+BB_API int bb_attn_fwd_noalloc(const bb_attn_desc* desc, const void* q,
+                               const void* k, const void* v,
+                               const uint8_t* key_mask,
+                               const int32_t* rand_idx, void* out, float* lse,
+                               void* stream);
+
 /* Waits for `stream`, then returns the status word the last call that used
  * `workspace` left there (BB_OK, BB_ERR_TIMEOUT or BB_ERR_BAD_TABLE), or
  * BB_ERR_CUDA if the copy itself failed. */

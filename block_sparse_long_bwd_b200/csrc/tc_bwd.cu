@@ -60,7 +60,7 @@ struct DqBars {
   uint64_t list_full[2], list_empty[2];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kKvStages], kv_empty[kKvStages];
-  uint64_t s_full, s_empty, p_full, dq_full, dq_empty;
+  uint64_t s_full, p_full, dq_full, dq_empty;
 };
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -97,7 +97,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.kv_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 1);
     mbar_init(&bars.p_full, 4);
     mbar_init(&bars.dq_full, 1);
     mbar_init(&bars.dq_empty, 4);
@@ -194,9 +193,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       for (int t = 0; t < n; ++t, ++g, ++u) {
         const int st = g % kKvStages;
+        // S and dP of this tile overwrite the previous tile's buffers (dS
+        // lives over S).  The previous dQ MMA, which reads that dS, was
+        // issued earlier by this thread, and MMAs from one thread execute in
+        // order, so there is no need to wait for it to complete.
         if (!mbar_wait(&bars.kv_full[st], (g / kKvStages) & 1, &abort_flag,
-                       p.status) ||
-            !mbar_wait(&bars.s_empty, (u & 1) ^ 1, &abort_flag, p.status)) {
+                       p.status)) {
           ok = false;
           break;
         }
@@ -228,7 +230,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             mma_ts(tDQ, tS + kk * 8, sdesc_sw128(kaddr + kk * 2048, 8192), idDQ,
                    (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.kv_empty[st]);
-          mma_commit(&bars.s_empty);
           if (t == n - 1) {
             mma_commit(&bars.dq_full);
             mma_commit(&bars.q_empty);
@@ -449,7 +450,7 @@ struct KeyItem {
 struct KvBars {
   uint64_t kp_full, kp_empty;
   uint64_t qt_full[kQStages], qt_empty[kQStages];
-  uint64_t s_full, s_empty, p_full, acc_full, acc_empty;
+  uint64_t s_full, p_full, acc_full, acc_empty;
 };
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -480,7 +481,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.qt_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_empty, 1);
     mbar_init(&bars.p_full, 4);
     mbar_init(&bars.acc_full, 1);
     mbar_init(&bars.acc_empty, 4);
@@ -574,9 +574,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       int i, mask, t = 0;
       while (it.next(i, mask)) {
         const int st = g % kQStages;
+        // S^T and dP^T overwrite the buffers that hold the previous tile's
+        // P^T and dS^T; the dV / dK MMAs reading those were issued earlier by
+        // this thread and execute first (in-order), so no completion wait.
         if (!mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
-                       p.status) ||
-            !mbar_wait(&bars.s_empty, (u & 1) ^ 1, &abort_flag, p.status)) {
+                       p.status)) {
           ok = false;
           break;
         }
@@ -612,7 +614,6 @@ __global__ void __launch_bounds__(kThreads, 2)
             mma_ts(tDK, tDP + kk * 8, sdesc_sw128(qaddr + kk * 2048, 8192), idAcc,
                    (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.qt_empty[st]);
-          mma_commit(&bars.s_empty);
         }
         __syncwarp();
         ++g;

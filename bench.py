@@ -67,6 +67,11 @@ def parse():
     # Profiling runs (ncu) only: leave out the end-to-end and CPU legs.
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    # Sweep mode: one line per (L, block, r) point of the length / block /
+    # random-count sweep (B*L = 32768 tokens, H = 12), then the linear-in-L
+    # check; not the headline line.
+    ap.add_argument("--sweep", action="store_true")
+    ap.add_argument("--sweep-steps", type=int, default=20)
     return ap.parse_args()
 
 
@@ -542,8 +547,83 @@ def run_reference(args, world, rank):
     }), flush=True)
 
 
+def run_sweep(args):
+    """fwd+bwd tokens/s and attended TFLOP/s per sweep point (device-timed,
+    CUDA events around each step, L2 flushed between steps), then the
+    linear-in-L check: at fixed (block, r), tokens/s within +-15 % of its
+    median over L."""
+    from block_sparse_long_bwd_b200 import binding as bb
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, _ = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for bs in synth.SWEEP_BS:
+        for r in synth.SWEEP_R:
+            for L in synth.SWEEP_L:
+                cfg = synth.sweep_point(L, bs, r)
+                B, H = cfg["B"], cfg["H"]
+                inp = synth.make_inputs(cfg)
+                att = bb.Attention(B, H, L, bs, r, torch.bfloat16, device=dev)
+                q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
+                out = torch.empty_like(q)
+                lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+                dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+
+                def step():
+                    att.forward(q, k, v, None, out=out, lse=lse)
+                    att.backward(q, k, v, out, lse, g, None, dq=dq, dk=dk, dv=dv)
+
+                for _ in range(3):
+                    step()
+                tot = 0.0
+                for s_ in range(args.sweep_steps):
+                    flush.fill_(s_ & 0xFF)
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    step()
+                    e1.record()
+                    e1.synchronize()
+                    tot += e0.elapsed_time(e1)
+                ms = tot / args.sweep_steps
+                pairs = sum(pairs_per_head(L // bs, att.table_host[h].numpy())
+                            for h in range(H)) * B
+                # FLOPs by the FlashAttention convention: 4 (fwd) + 10 (bwd)
+                # bs^2 d per attended pair.
+                counted = (4 + 10) * pairs * bs * bs * cfg["d"]
+                names = [bb.bb_attn_launch_name(att.desc, 0, 0)]
+                row = {"L": L, "block_size": bs, "r": r, "B": B,
+                       "ms": round(ms, 4),
+                       "tokens_per_s": round(B * L / (ms / 1e3), 1),
+                       "attended_tflops": round(counted / (ms / 1e3) / 1e12, 2),
+                       "frac_of_peak": round(counted / (ms / 1e3) / 1e12
+                                             / peaks["bf16_tflops"], 4),
+                       "path": "tensor" if names[0].startswith("tc_") else
+                               "cuda-core"}
+                rows.append(row)
+                print(json.dumps(row), flush=True)
+                del q, k, v, g, out, lse, dq, dk, dv, att
+                torch.cuda.empty_cache()
+    checks = []
+    for bs in synth.SWEEP_BS:
+        for r in synth.SWEEP_R:
+            tp = [x["tokens_per_s"] for x in rows
+                  if x["block_size"] == bs and x["r"] == r]
+            med = statistics.median(tp)
+            dev_ = max(abs(t / med - 1) for t in tp)
+            checks.append({"block_size": bs, "r": r,
+                           "max_dev_from_median": round(dev_, 3),
+                           "linear_in_L": dev_ <= 0.15})
+    print(json.dumps({"sweep_linear_in_L": checks}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     world, rank, local = init_dist(args)
     try:
         if args.impl == "reference":

@@ -198,6 +198,22 @@ def init_dist(args):
     return world, rank, local
 
 
+def max_over_ranks(value, world, device=None):
+    """Largest `value` over all ranks (the slowest rank's time); identity on
+    one rank.  Works with the nccl (CUDA tensors) or gloo (CPU) backend."""
+    if world <= 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(tokens_per_rank, steps, max_total_ms, world):
+    """Whole-job throughput: tokens of all ranks over the slowest rank's
+    device time (weak scaling: every rank runs its own batch)."""
+    return tokens_per_rank * world * steps / (max_total_ms / 1e3)
+
+
 def algorithmic(cfg, pairs_total):
     """Algorithmic FLOPs and bytes per launch of each kernel kind."""
     B, H, L, d, bs = cfg["B"], cfg["H"], cfg["L"], cfg["d"], cfg["block_size"]
@@ -312,14 +328,9 @@ def run_ours(args, world, rank, local):
                 per_kernel[n].append(t)
             tot += ev[0].elapsed_time(ev[-1])
         step_ms.append(tot)
-    total_ms = sum(step_ms)
-    if world > 1:
-        tt = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / K
-    tokens = B * L * world
-    value = tokens * K / (total_ms / 1e3)
+    value = aggregate_tokens_per_s(B * L, K, total_ms, world)
 
     # Attended FLOPs over the pattern's pairs (masked keys included).
     pairs = sum(pairs_per_head(nb, att.table_host[h].numpy())
@@ -449,11 +460,7 @@ def run_e2e(args, cfg, att, inp, dev, backward, world):
     for _ in range(n):
         step()
     torch.cuda.synchronize()
-    el = time.perf_counter() - t0
-    if world > 1:
-        tt = torch.tensor([el], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        el = float(tt.item())
+    el = max_over_ranks(time.perf_counter() - t0, world, dev)
     return {"value": round(B * L * world * n / el, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": n, "timing": "host wall clock around synchronised steps"}

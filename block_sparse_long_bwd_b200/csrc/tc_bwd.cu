@@ -2,18 +2,18 @@
 // d 64) for sm_100a.  Probabilities are recomputed from the forward's lse
 // (P = exp(S - lse)), so nothing of size pairs x bs^2 is stored.
 //
-// tc_dq_kernel: query-side items (as in the forward: middle query-block pairs
-//   and chunks of the global rows).  Per key block j of the item:
+// tc_dq_kernel: query-side items (as in the forward: middle 128-row windows
+//   and chunks of the global rows; see tc_common.cuh).  Per key block j of the item:
 //   S = Q K_j^T and dP = dO V_j^T into TMEM; one thread per row forms
 //   dS = P (dP - D) (D = <dO, O> of the row, computed at the start of the
 //   item and also written to the workspace with -lse*log2(e) for the next
 //   kernel); dS (bf16) goes back to TMEM and dQ += dS K_j accumulates in
 //   TMEM across the item.  Global rows write fp32 partials per chunk.
-// tc_dkdv_kernel: key-side items pair two key blocks (j, j+1) in one
-//   128-row tile and walk the union of their transposed adjacency lists (the
-//   query blocks that attend them, from the CSR); the global key blocks
-//   (0, nb-1), attended by every query block, are split into chunks of query
-//   blocks.  Per query block i: S^T = K_pair Q_i^T and dP^T = V_pair dO_i^T;
+// tc_dkdv_kernel: key-side items take 128 key rows (a middle window of two
+//   key tiles) and walk the merged transposed adjacency lists (the query
+//   blocks that attend their key blocks, from the CSR), as query tiles with
+//   a group/half mask; the global key blocks, attended by every query block,
+//   are split into chunks of query tiles.  Per query block i: S^T = K_pair Q_i^T and dP^T = V_pair dO_i^T;
 //   P^T and dS^T (bf16) back to TMEM; dV += P^T dO_i and dK += dS^T Q_i
 //   accumulate in TMEM.  Each key row is owned by exactly one item (or one
 //   chunk partial), so there are no atomics.
@@ -33,14 +33,11 @@ constexpr int kQStages = 3;
 constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // Q, dO, NL, D
 
 struct BwdArgs {
-  PairArgs qa;       // query-side items (dq)
-  int kpairs;        // middle key-block pairs
-  int kchunks;       // query-block chunks of the global key blocks
-  int kitems;        // key-side items (dkdv)
+  PairArgs qa;       // items: query side (dq) and, mirrored, key side (dkdv)
   float* D;          // [B*H*L]
   float* NL;         // [B*H*L]: -lse * log2(e)
-  float* dqpart;     // [B*H][nchunks][128][64]
-  float* kvpart;     // [B*H][kchunks][128][128] (dK | dV)
+  float* dqpart;     // [B*H][n_git][nchunks][128][64]
+  float* kvpart;     // [B*H][n_git][nchunks][128][128] (dK | dV)
 };
 
 __device__ __forceinline__ void ld_bf16x8_as_f(const __nv_bfloat16* p,
@@ -134,10 +131,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&bars.list_full[slot]);
         if (!mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = L.bh * p.L;
-        const int nh = L.blk[1] >= 0 ? 2 : 1;
+        const int nh = L.t[1] >= 0 ? 2 : 1;
         mbar_expect_tx(&bars.q_full, 2u * nh * kTileBytes);
         for (int hh = 0; hh < nh; ++hh) {
-          const int y = row0 + L.blk[hh] * kBS;
+          const int y = row0 + L.t[hh] * kTile;
           tma_load_2d(Qs + hh * kTileBytes, &tmQ, &bars.q_full, 0, y);
           tma_load_2d(Gs + hh * kTileBytes, &tmG, &bars.q_full, 0, y);
         }
@@ -153,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           mbar_expect_tx(&bars.kv_full[st], 2 * kTileBytes);
           uint8_t* kv = KVs + st * 2 * kTileBytes;
-          const int y = row0 + L.tile[t] * kBS;
+          const int y = row0 + L.tile[t] * kTile;
           tma_load_2d(kv, &tmK, &bars.kv_full[st], 0, y);
           tma_load_2d(kv + kTileBytes, &tmV, &bars.kv_full[st], 0, y);
           ++g;
@@ -242,7 +239,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int half = row >> 6, hbit = 1 << half, r64 = row & 63;
+    const int half = row >> 6, r64 = row & 63;
+    const int gshift = 2 * quarter;  // this warp's row group = its quarter
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
@@ -253,10 +251,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         break;
       const ItemList& L = lists[slot];
       const int n = L.n;
-      const int blk = L.blk[half];
-      const size_t grow = (size_t)L.bh * p.L + (size_t)(blk < 0 ? 0 : blk) * kBS + r64;
+      const bool rvalid = (L.gvalid >> quarter) & 1;
+      const size_t grow = (size_t)L.bh * p.L + (size_t)(rvalid ? L.t[half] : 0) * kTile + r64;
       float nl2 = 0.f, Dr = 0.f;
-      if (blk >= 0) {
+      if (rvalid) {
         nl2 = -p.lse[grow] * kLog2e;
         const __nv_bfloat16* Or = static_cast<const __nv_bfloat16*>(p.o) + grow * kHeadDim;
         const __nv_bfloat16* Gr = static_cast<const __nv_bfloat16*>(p.dout) + grow * kHeadDim;
@@ -280,12 +278,17 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-        const bool att = (L.mask[t] & hbit) != 0;
+        const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
         uint32_t dS[32];
-        if (att) {
+        if (m2) {
           const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
+            if (!((m2 >> hc) & 1)) {  // keys outside the attended blocks
+#pragma unroll
+              for (int e = 0; e < 16; ++e) dS[hc * 16 + e] = 0u;
+              continue;
+            }
             uint32_t s[32], dp[32];
             tmem_ld32(tS + hc * 32 + lane_off, s);
             tmem_ld32(tDP + hc * 32 + lane_off, dp);
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.dq_empty);
-      if (blk >= 0) {
+      if (rvalid) {
         if (!L.global) {
           uint4* dst = reinterpret_cast<uint4*>(
               static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim);
@@ -345,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(
-              ba.dqpart + (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) * 64);
+              ba.dqpart + ((((size_t)L.bh * a.geo.n_git + L.gi) * a.geo.nchunks + L.chunk) *
+                               128 + row) * 64);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             dst[v] = make_float4(__uint_as_float(q0[4 * v]), __uint_as_float(q0[4 * v + 1]),
@@ -370,82 +374,6 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ======================= dK / dV =======================
-
-// Key-side item decoding and the walk over attending query blocks.  Every
-// role of the kernel runs its own copy of this iterator; all copies see the
-// same sequence.
-struct KeyItem {
-  int bh, b;
-  int kb[2];          // key block of half 0 / 1 (-1: unused)
-  int global, chunk;
-  // walk state
-  const int* la;
-  const int* lb;
-  int na, nbb, ia, ib;
-  int cur, end, bits;
-
-  __device__ void init(const BwdArgs& ba, int item) {
-    const Problem& p = ba.qa.p;
-    const int nb = p.nb;
-    const int per = ba.kpairs + ba.kchunks;
-    bh = item / per;
-    b = bh / p.H;
-    const int h = bh % p.H;
-    const int loc = item % per;
-    ia = ib = na = nbb = 0;
-    la = lb = nullptr;
-    if (loc < ba.kchunks) {
-      global = 1;
-      chunk = loc;
-      kb[0] = 0;
-      kb[1] = nb > 1 ? nb - 1 : -1;
-      bits = nb > 1 ? 3 : 1;
-      cur = loc * kChunk;
-      end = min(nb, cur + kChunk);
-      return;
-    }
-    global = 0;
-    chunk = 0;
-    const int j0 = 1 + 2 * (loc - ba.kchunks);
-    kb[0] = j0;
-    kb[1] = (j0 + 1 <= nb - 2) ? j0 + 1 : -1;
-    const int* offs = p.csr_offs + (size_t)h * (nb + 1);
-    const int* list = p.csr_list + (size_t)h * p.csr_cap;
-    la = list + offs[j0];
-    na = offs[j0 + 1] - offs[j0];
-    if (kb[1] >= 0) {
-      lb = list + offs[j0 + 1];
-      nbb = offs[j0 + 2] - offs[j0 + 1];
-    }
-  }
-  // Next attending query block i and its half mask; false at the end.
-  __device__ bool next(int& i, int& mask) {
-    if (global) {
-      if (cur >= end) return false;
-      i = cur++;
-      mask = bits;
-      return true;
-    }
-    const int va = ia < na ? la[ia] : 0x7FFFFFFF;
-    const int vb = ib < nbb ? lb[ib] : 0x7FFFFFFF;
-    if (va == 0x7FFFFFFF && vb == 0x7FFFFFFF) return false;
-    if (va < vb) {
-      i = va;
-      mask = 1;
-      ++ia;
-    } else if (vb < va) {
-      i = vb;
-      mask = 2;
-      ++ib;
-    } else {
-      i = va;
-      mask = 3;
-      ++ia;
-      ++ib;
-    }
-    return true;
-  }
-};
 
 struct KvBars {
   uint64_t kp_full, kp_empty;
@@ -507,16 +435,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int kp_issued = 0;
       uint32_t kp_par = 0;
-      for (int k = 0, item = blockIdx.x; item < ba.kitems;
+      for (int k = 0, item = blockIdx.x; item < ba.qa.items;
            ++k, item += gridDim.x) {
-        KeyItem it;
-        it.init(ba, item);
+        KeyWalk it;
+        it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
         if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = it.bh * p.L;
-        const int nh = it.kb[1] >= 0 ? 2 : 1;
+        const int nh = it.t[1] >= 0 ? 2 : 1;
         mbar_expect_tx(&bars.kp_full, 2u * nh * kTileBytes);
         for (int hh = 0; hh < nh; ++hh) {
-          const int y = row0 + it.kb[hh] * kBS;
+          const int y = row0 + it.t[hh] * kTile;
           tma_load_2d(Ks + hh * kTileBytes, &tmK, &bars.kp_full, 0, y);
           tma_load_2d(Vs + hh * kTileBytes, &tmV, &bars.kp_full, 0, y);
         }
@@ -533,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           uint8_t* q = QT + st * kQStageBytes;
           mbar_expect_tx(&bars.qt_full[st], 2 * kTileBytes + 512);
-          const int y = row0 + i * kBS;
+          const int y = row0 + i * kTile;
           tma_load_2d(q, &tmQ, &bars.qt_full[st], 0, y);
           tma_load_2d(q + kTileBytes, &tmG, &bars.qt_full[st], 0, y);
           bulk_load(q + 2 * kTileBytes, ba.NL + y, 256, &bars.qt_full[st]);
@@ -565,10 +493,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
     uint32_t g = 0, u = 0;
     bool ok = true;
-    for (int k = 0, item = blockIdx.x; item < ba.kitems && ok;
+    for (int k = 0, item = blockIdx.x; item < ba.qa.items && ok;
          ++k, item += gridDim.x) {
-      KeyItem it;
-      it.init(ba, item);
+      KeyWalk it;
+      it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
       if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       int i, mask, t = 0;
@@ -630,19 +558,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else {
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int half = row >> 6, hbit = 1 << half, r64 = row & 63;
+    const int half = row >> 6, r64 = row & 63;
+    const int gshift = 2 * quarter;  // this warp's key-row group = its quarter
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t g = 0, u = 0;
-    for (int k = 0, item = blockIdx.x; item < ba.kitems; ++k, item += gridDim.x) {
-      KeyItem it;
-      it.init(ba, item);
-      const int kblk = it.kb[half];
-      const size_t krow = (size_t)it.bh * p.L + (size_t)(kblk < 0 ? 0 : kblk) * kBS + r64;
+    for (int k = 0, item = blockIdx.x; item < ba.qa.items; ++k, item += gridDim.x) {
+      KeyWalk it;
+      it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
+      const bool rvalid = (it.gvalid >> quarter) & 1;
+      const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
+      const size_t krow = (size_t)it.bh * p.L + ktok;
       float off = 0.f;
-      if (kblk >= 0 && p.key_mask)
-        off = p.key_mask[(size_t)it.b * p.L + (size_t)kblk * kBS + r64] ? 0.f : mvl;
+      if (rvalid && p.key_mask)
+        off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
       int i, mask;
       bool ok = true;
       while (it.next(i, mask)) {
@@ -652,7 +582,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
-        const bool att = (mask & hbit) != 0;
+        const int m2 = (mask >> gshift) & 3;  // attending query-column halves
+        const bool att = m2 != 0;
         uint32_t P[32], dS[32];
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
         if (att && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
@@ -665,6 +596,14 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float* Ds = NLs + 64;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
+            if (!((m2 >> hc) & 1)) {  // query rows outside attending blocks
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                P[hc * 16 + e] = 0u;
+                dS[hc * 16 + e] = 0u;
+              }
+              continue;
+            }
             uint32_t s[32], dp[32];
             tmem_ld32(tS + hc * 32 + lane_off, s);
             tmem_ld32(tDP + hc * 32 + lane_off, dp);
@@ -731,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty);
-      if (kblk >= 0) {
+      if (rvalid) {
         if (!it.global) {
           uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + krow * kHeadDim);
           uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + krow * kHeadDim);
@@ -753,7 +692,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(
-              ba.kvpart + (((size_t)it.bh * ba.kchunks + it.chunk) * 128 + row) * 128);
+              ba.kvpart + ((((size_t)it.bh * ba.qa.geo.n_git + it.gi) * ba.qa.geo.nchunks +
+                            it.chunk) * 128 + row) * 128);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             dst[v] = make_float4(__uint_as_float(k0[4 * v]), __uint_as_float(k0[4 * v + 1]),
@@ -778,31 +718,31 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// One warp per row of a global block (query rows for dQ, key rows for
-// dK/dV); lanes over d.  Chunks are summed in a fixed order.
+// One warp per row of a global item (query rows for dQ, key rows for
+// dK / dV: both sides use the same tiles); lanes over d.  Chunks are summed
+// in a fixed order; rows outside the global blocks are skipped.
 __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
   const Problem& p = ba.qa.p;
-  const int nhalves = p.nb > 1 ? 2 : 1;
+  const Geom& g = ba.qa.geo;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t id = (size_t)blockIdx.x * 8 + warp;
-  const size_t total = (size_t)p.B * p.H * nhalves * kBS;
+  const size_t id = (size_t)blockIdx.x * 8 + warp;  // over bh x gi x 128
+  const size_t total = (size_t)p.B * p.H * g.n_git * 128;
   if (id >= total) return;
-  const int r64 = id % kBS;
-  const int half = (id / kBS) % nhalves;
-  const size_t bh = id / (kBS * nhalves);
-  const int row = half * 64 + r64;
-  const int blk = half == 0 ? 0 : p.nb - 1;
-  const size_t grow = bh * p.L + (size_t)blk * kBS + r64;
-  float q0 = 0.f, q1 = 0.f;
-  for (int c = 0; c < ba.qa.nchunks; ++c) {
+  const int row = id % 128;
+  const int gi = (id / 128) % g.n_git;
+  const size_t bh = id / (128 * g.n_git);
+  int t[2], gvalid;
+  item_rows(g, true, gi, t, gvalid);
+  if (!((gvalid >> (row >> 5)) & 1)) return;
+  const size_t grow = bh * p.L + (size_t)t[row >> 6] * kTile + (row & 63);
+  const size_t ib = (bh * g.n_git + gi) * g.nchunks;
+  float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  for (int c = 0; c < g.nchunks; ++c) {
     const float2 x = reinterpret_cast<const float2*>(
-        ba.dqpart + ((bh * ba.qa.nchunks + c) * 128 + row) * 64)[lane];
+        ba.dqpart + ((ib + c) * 128 + row) * 64)[lane];
     q0 += x.x;
     q1 += x.y;
-  }
-  float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
-  for (int c = 0; c < ba.kchunks; ++c) {
-    const float* src = ba.kvpart + ((bh * ba.kchunks + c) * 128 + row) * 128;
+    const float* src = ba.kvpart + ((ib + c) * 128 + row) * 128;
     const float2 xk = reinterpret_cast<const float2*>(src)[lane];
     const float2 xv = reinterpret_cast<const float2*>(src + 64)[lane];
     k0 += xk.x;
@@ -821,9 +761,6 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
 BwdArgs make_bwd_args(const Problem& p) {
   BwdArgs ba;
   ba.qa = make_pair_args(p);
-  ba.kchunks = ba.qa.nchunks;
-  ba.kpairs = ba.qa.npairs;
-  ba.kitems = p.B * p.H * (ba.kpairs + ba.kchunks);
   return ba;
 }
 
@@ -834,23 +771,23 @@ bool tc_bwd_supported(const Problem& p) { return tc_shape_ok(p); }
 // D, NL: rows floats each; dq partials; dK/dV partials.
 size_t tc_bwd_extra_bytes(const Problem& p) {
   const size_t rows = (size_t)p.B * p.H * p.L;
-  const int nch = (p.nb + kChunk - 1) / kChunk;
-  return rows * 4 /* NL */ + (size_t)p.B * p.H * nch * 128 * 64 * 4 +
-         (size_t)p.B * p.H * nch * 128 * 128 * 4 + 3 * 256;
+  const Geom g = make_geom(p.L, p.bs);
+  const size_t units = (size_t)p.B * p.H * g.n_git * g.nchunks * 128;
+  return rows * 4 /* NL */ + units * 64 * 4 + units * 128 * 4 + 3 * 256;
 }
 
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
   BwdArgs ba = make_bwd_args(p);
   const size_t rows = (size_t)p.B * p.H * p.L;
-  const int nch = ba.qa.nchunks;
+  const size_t units = (size_t)p.B * p.H * ba.qa.geo.n_git * ba.qa.geo.nchunks * 128;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   uint8_t* x = reinterpret_cast<uint8_t*>(p.part);
   ba.D = p.D;
   ba.NL = reinterpret_cast<float*>(x);
   x += al(rows * 4);
   ba.dqpart = reinterpret_cast<float*>(x);
-  x += al((size_t)p.B * p.H * nch * 128 * 64 * 4);
+  x += al(units * 64 * 4);
   ba.kvpart = reinterpret_cast<float*>(x);
 
   int dev = 0, sms = 148;
@@ -872,14 +809,14 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   e = cudaFuncSetAttribute(tc_dkdv_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
   if (e != cudaSuccess) return e;
-  tc_dkdv_kernel<<<min(ba.kitems, 2 * sms), kThreads, smem_kv, s>>>(
+  tc_dkdv_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_kv, s>>>(
       ba, tm.q, tm.k, tm.v, tm.dout);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = marks->mark(s);
   if (e != cudaSuccess) return e;
 
-  const size_t frows = (size_t)p.B * p.H * (p.nb > 1 ? 2 : 1) * kBS;
+  const size_t frows = (size_t)p.B * p.H * ba.qa.geo.n_git * 128;
   bwd_finish_kernel<<<(unsigned)((frows + 7) / 8), 256, 0, s>>>(ba);
   return cudaGetLastError();
 }

@@ -1,118 +1,356 @@
-// Work-item description shared by the tensor-core kernels.
+// Work items shared by the tensor-core kernels.
 //
-// A query-side item pairs two query blocks of one (b, h) in one 128-row MMA
-// tile (rows 0-63: half 0, rows 64-127: half 1):
-//  * middle pair (i, i+1), i = 1, 3, 5, ...: the key blocks visited are the
-//    union of the two attended sets A(i), A(i+1) ({0, i-1, i, i+1, nb-1} and
-//    the row's random blocks); each carries a 2-bit mask of the halves that
-//    attend it.  The last pair has an empty half when nb - 2 is odd.
-//  * global chunk c: query blocks 0 and nb-1, which attend every key block,
-//    over key blocks [c * kChunk, (c + 1) * kChunk); the kernels write
+// The kernels work in 64-token tiles (one 64 x 64 bf16 TMA box) whatever the
+// block size (32, 64 or 128).  An item is one 128-row MMA tile made of two
+// 64-row tiles ("halves"), split into four 32-row groups g = 0..3 (group g =
+// TMEM lane quarter g, so each softmax warp owns one group).  A group lies in
+// a single block of the pattern (blocks are >= 32 tokens).  Each tile an
+// item visits (a key tile on the query side, a query tile on the key side)
+// carries an 8-bit mask: bit 2g + c says "row group g attends the 32
+// columns c of this tile" (c = 0: columns 0-31, c = 1: columns 32-63).
+//
+// Query-side items (forward and dQ):
+//  * middle window w: rows [128 w, 128 w + 128) (query tiles 2w, 2w + 1);
+//    every group whose block is a middle block (1 .. nb - 2) visits the key
+//    tiles of its attended set A(i) = {0, i-1, i, i+1, nb-1} U rand(i);
+//    groups of the global blocks, or past L, are masked off.  Only windows
+//    that hold a middle block are items.
+//  * global item gi, chunk c: the 64-row tiles holding the global blocks 0
+//    and nb-1 (at most four, paired two per item) over key tiles
+//    [8c, 8c + 8); those rows attend every key, so the kernels write
 //    per-chunk partials that a second kernel merges.
+// Key-side items (dK / dV) mirror this with key and query swapped: a middle
+// window walks the merged transposed-adjacency lists of its key blocks; the
+// global key blocks are split over chunks of query tiles.
 #pragma once
 
 #include "sm100.cuh"
 
 namespace bb {
 
-constexpr int kBS = 64;                               // block size (tokens)
-constexpr int kMaxT = 32;                             // key blocks per item
-constexpr int kChunk = 8;                             // key blocks per chunk
-constexpr uint32_t kTileBytes = kBS * kHeadDim * 2;   // one 64 x 64 bf16 tile
-constexpr int kPartStride = 68;                       // floats per partial row
+constexpr int kTile = 64;                             // tokens per tile
+constexpr int kMaxT = 64;                             // tiles per item
+constexpr int kChunk = 8;                             // tiles per chunk
+constexpr uint32_t kTileBytes = kTile * kHeadDim * 2; // one 64 x 64 bf16 tile
+constexpr int kPartStride = 68;                       // floats per fwd partial row
+
+// Geometry of the tiled problem (host and device).
+struct Geom {
+  int bs, nb, nt;       // block size, blocks, 64-token tiles
+  int w_first, n_mid;   // middle windows
+  int ngt;              // tiles holding global blocks (ascending in gt)
+  int gt[4];
+  int n_git;            // global items = ceil(ngt / 2)
+  int nchunks;          // chunks of the tile range [0, nt)
+  int per_bh;           // items per (b, h): n_mid + n_git * nchunks
+};
+
+__host__ __device__ inline Geom make_geom(int L, int bs) {
+  Geom g;
+  g.bs = bs;
+  g.nb = L / bs;
+  g.nt = L / kTile;
+  // Windows intersecting the middle tokens [bs, L - bs).
+  if (g.nb >= 3) {
+    g.w_first = bs / 128;
+    const int w_last = (L - bs - 1) / 128;
+    g.n_mid = w_last - g.w_first + 1;
+  } else {
+    g.w_first = 0;
+    g.n_mid = 0;
+  }
+  // Tiles holding rows of blocks 0 and nb - 1.
+  g.ngt = 0;
+  const int tpb = bs >= kTile ? bs / kTile : 1;  // tiles per block
+  for (int t = 0; t < tpb; ++t) g.gt[g.ngt++] = t;
+  for (int t = g.nt - tpb; t < g.nt; ++t) {
+    bool dup = false;
+    for (int c = 0; c < g.ngt; ++c) dup |= (g.gt[c] == t);
+    if (!dup && t >= 0) g.gt[g.ngt++] = t;
+  }
+  g.n_git = (g.ngt + 1) / 2;
+  g.nchunks = (g.nt + kChunk - 1) / kChunk;
+  g.per_bh = g.n_mid + g.n_git * g.nchunks;
+  return g;
+}
+
+// Block of token row `tok`.
+__host__ __device__ inline int block_of(const Geom& g, int tok) {
+  return tok / g.bs;
+}
+
+// Tiles covering block j and the column halves of each it spans:
+// bs 32 -> one tile, one half; 64 -> one tile, both halves; 128 -> two tiles.
+template <typename F>
+__host__ __device__ __forceinline__ void for_block_tiles(const Geom& g, int j, F f) {
+  if (g.bs == 32) {
+    f(j >> 1, 1 << (j & 1));
+  } else if (g.bs == 64) {
+    f(j, 3);
+  } else {
+    f(2 * j, 3);
+    f(2 * j + 1, 3);
+  }
+}
 
 struct ItemList {
   int n;
-  int global;   // 1 = global chunk
+  int global;   // 1 = global item
   int bh, b;
-  int blk[2];   // query block of half 0 / half 1 (-1: half unused)
-  int chunk;
+  int t[2];     // row tile of half 0 / 1 (-1: absent)
+  int gvalid;   // 4-bit: groups whose rows this item produces
+  int gi, chunk;
   int16_t tile[kMaxT];
   uint8_t mask[kMaxT];
 };
 
 struct PairArgs {
   Problem p;
-  int npairs, nchunks, items;
+  Geom geo;
+  int items;
 };
 
 inline PairArgs make_pair_args(const Problem& p) {
   PairArgs a;
   a.p = p;
-  a.nchunks = (p.nb + kChunk - 1) / kChunk;
-  a.npairs = p.nb > 2 ? (p.nb - 1) / 2 : 0;
-  a.items = p.B * p.H * (a.npairs + a.nchunks);
+  a.geo = make_geom(p.L, p.bs);
+  a.items = p.B * p.H * a.geo.per_bh;
   return a;
 }
 
-__device__ __forceinline__ void list_add(ItemList& L, int j, int bit) {
+__host__ __device__ __forceinline__ void list_add(ItemList& L, int tile, int bits) {
   for (int c = 0; c < L.n; ++c)
-    if (L.tile[c] == j) {
-      L.mask[c] |= (uint8_t)bit;
+    if (L.tile[c] == tile) {
+      L.mask[c] |= (uint8_t)bits;
       return;
     }
-  L.tile[L.n] = (int16_t)j;
-  L.mask[L.n] = (uint8_t)bit;
+  if (L.n >= kMaxT) return;  // host validation keeps lists within kMaxT
+  L.tile[L.n] = (int16_t)tile;
+  L.mask[L.n] = (uint8_t)bits;
   ++L.n;
 }
 
-// Fills L for query-side item `item` (items are (b, h)-major; within one
-// (b, h) the global chunks come first, then the middle pairs).
-__device__ inline void build_pair_item(const PairArgs& a, int item,
-                                       ItemList& L) {
+// Row tiles and valid groups of a window / global item.
+__host__ __device__ __forceinline__ void item_rows(const Geom& g, bool global, int w_or_gi,
+                                          int (&t)[2], int& gvalid) {
+  if (!global) {
+    t[0] = 2 * w_or_gi;
+    t[1] = 2 * w_or_gi + 1 < g.nt ? 2 * w_or_gi + 1 : -1;
+  } else {
+    t[0] = g.gt[2 * w_or_gi];
+    t[1] = 2 * w_or_gi + 1 < g.ngt ? g.gt[2 * w_or_gi + 1] : -1;
+  }
+  gvalid = 0;
+  for (int gr = 0; gr < 4; ++gr) {
+    const int tt = t[gr >> 1];
+    if (tt < 0) continue;
+    const int blk = block_of(g, tt * kTile + 32 * (gr & 1));
+    const bool is_global = (blk == 0 || blk == g.nb - 1);
+    if (global == is_global) gvalid |= 1 << gr;
+  }
+}
+
+// Expand a 4-bit group set into mask bits for column halves `halves`.
+__host__ __device__ __forceinline__ int expand_groups(int groups, int halves) {
+  int m = 0;
+  for (int gr = 0; gr < 4; ++gr)
+    if (groups & (1 << gr)) m |= halves << (2 * gr);
+  return m;
+}
+
+// Fills L for query-side item `item` ((b, h)-major; within one (b, h) the
+// global items' chunks come first, then the middle windows).
+__host__ __device__ inline void build_pair_item(const PairArgs& a, int item,
+                                                ItemList& L) {
   const Problem& p = a.p;
-  const int nb = p.nb;
-  const int per = a.npairs + a.nchunks;
-  const int bh = item / per, loc = item % per;
+  const Geom& g = a.geo;
+  const int bh = item / g.per_bh, loc = item % g.per_bh;
   L.n = 0;
   L.bh = bh;
   L.b = bh / p.H;
   const int h = bh % p.H;
-  if (loc < a.nchunks) {
+  const int nglob = g.n_git * g.nchunks;
+  if (loc < nglob) {
     L.global = 1;
-    L.chunk = loc;
-    L.blk[0] = 0;
-    L.blk[1] = nb > 1 ? nb - 1 : -1;
-    const int bits = nb > 1 ? 3 : 1;
-    const int j1 = min(nb, (loc + 1) * kChunk);
-    for (int j = loc * kChunk; j < j1; ++j) {
+    L.gi = loc / g.nchunks;
+    L.chunk = loc % g.nchunks;
+    item_rows(g, true, L.gi, L.t, L.gvalid);
+    const int m = expand_groups(L.gvalid, 3);
+    const int j1 = g.nt < (L.chunk + 1) * kChunk ? g.nt : (L.chunk + 1) * kChunk;
+    for (int j = L.chunk * kChunk; j < j1; ++j) {
       L.tile[L.n] = (int16_t)j;
-      L.mask[L.n] = (uint8_t)bits;
+      L.mask[L.n] = (uint8_t)m;
       ++L.n;
     }
     return;
   }
   L.global = 0;
+  L.gi = 0;
   L.chunk = 0;
-  const int i0 = 1 + 2 * (loc - a.nchunks);
-  L.blk[0] = i0;
-  L.blk[1] = (i0 + 1 <= nb - 2) ? i0 + 1 : -1;
-  for (int half = 0; half < 2; ++half) {
-    const int i = L.blk[half];
-    if (i < 0) continue;
-    const int bit = 1 << half;
-    list_add(L, 0, bit);
-    list_add(L, i - 1, bit);
-    list_add(L, i, bit);
-    list_add(L, i + 1, bit);
-    list_add(L, nb - 1, bit);
+  const int w = g.w_first + (loc - nglob);
+  item_rows(g, false, w, L.t, L.gvalid);
+  const int nb = g.nb;
+  int last_blk = -1;
+  for (int gr = 0; gr < 4; ++gr) {
+    if (!(L.gvalid & (1 << gr))) continue;
+    const int i = block_of(g, L.t[gr >> 1] * kTile + 32 * (gr & 1));
+    const int gbits = 1 << (2 * gr);
+    auto add_block = [&](int j) {
+      for_block_tiles(g, j, [&](int tile, int halves) {
+        list_add(L, tile, halves * gbits);
+      });
+    };
+    add_block(0);
+    add_block(i - 1);
+    add_block(i);
+    add_block(i + 1);
+    add_block(nb - 1);
     const int32_t* row = p.rand_idx + ((size_t)h * nb + i) * p.r;
     for (int c = 0; c < p.r; ++c) {
       const int j = row[c];
       if (j == -1) continue;
       if (j < 0 || j >= nb) {
-        set_status(p.status, BB_ERR_BAD_TABLE);
+#ifdef __CUDA_ARCH__
+        if (i != last_blk) set_status(p.status, BB_ERR_BAD_TABLE);
+#endif
         continue;
       }
-      list_add(L, j, bit);
+      add_block(j);
     }
+    last_blk = i;
   }
 }
 
-// Validity bitmap of the 64 keys of key block j (bit k set = attend).
+// Walk of one key-side item over the query tiles that attend it, with the
+// 8-bit mask (bit 2g + c: key group g is attended by query rows of column
+// half c of the query tile).  Every role of the dK/dV kernel runs its own
+// copy; all copies see the same sequence.
+struct KeyWalk {
+  int bh, b;
+  int t[2];       // key tile of half 0 / 1 (-1: absent)
+  int gvalid;
+  int global, gi, chunk;
+  // global: query tiles [cur, end)
+  int cur, end, gmask;
+  // middle: up to four sorted CSR lists (one per distinct key block)
+  int nl;
+  const int* lp[4];
+  int ln[4], li[4], lg[4];
+  int bs;
+  int pend_tile, pend_mask;  // block 128: second tile of a query block
+
+  __host__ __device__ void init(const PairArgs& a, const int* csr_offs,
+                       const int* csr_list, int csr_cap, int item) {
+    const Problem& p = a.p;
+    const Geom& g = a.geo;
+    bh = item / g.per_bh;
+    b = bh / p.H;
+    const int h = bh % p.H;
+    const int loc = item % g.per_bh;
+    const int nglob = g.n_git * g.nchunks;
+    bs = g.bs;
+    pend_tile = -1;
+    pend_mask = 0;
+    nl = 0;
+    if (loc < nglob) {
+      global = 1;
+      gi = loc / g.nchunks;
+      chunk = loc % g.nchunks;
+      item_rows(g, true, gi, t, gvalid);
+      gmask = expand_groups(gvalid, 3);
+      cur = chunk * kChunk;
+      end = g.nt < cur + kChunk ? g.nt : cur + kChunk;
+      return;
+    }
+    global = 0;
+    gi = 0;
+    chunk = 0;
+    item_rows(g, false, g.w_first + (loc - nglob), t, gvalid);
+    const int* offs = csr_offs + (size_t)h * (g.nb + 1);
+    const int* list = csr_list + (size_t)h * csr_cap;
+    for (int gr = 0; gr < 4; ++gr) {
+      if (!(gvalid & (1 << gr))) continue;
+      const int j = block_of(g, t[gr >> 1] * kTile + 32 * (gr & 1));
+      int x = 0;
+      while (x < nl && lp[x] != list + offs[j]) ++x;
+      if (x == nl) {
+        lp[nl] = list + offs[j];
+        ln[nl] = offs[j + 1] - offs[j];
+        li[nl] = 0;
+        lg[nl] = 0;
+        ++nl;
+      }
+      lg[x] |= 1 << gr;
+    }
+  }
+
+  // Smallest unconsumed query block over the lists (INT_MAX when done) and
+  // the groups whose lists hold it.
+  __host__ __device__ __forceinline__ int peek(int& groups) const {
+    int qb = 0x7FFFFFFF;
+    groups = 0;
+    for (int x = 0; x < nl; ++x)
+      if (li[x] < ln[x]) {
+        const int v = lp[x][li[x]];
+        if (v < qb) {
+          qb = v;
+          groups = lg[x];
+        } else if (v == qb) {
+          groups |= lg[x];
+        }
+      }
+    return qb;
+  }
+  __host__ __device__ __forceinline__ void consume(int qb) {
+    for (int x = 0; x < nl; ++x)
+      if (li[x] < ln[x] && lp[x][li[x]] == qb) ++li[x];
+  }
+
+  // Next query tile and its mask; false at the end.
+  __host__ __device__ bool next(int& tile, int& mask) {
+    if (global) {
+      if (cur >= end) return false;
+      tile = cur++;
+      mask = gmask;
+      return true;
+    }
+    if (pend_tile >= 0) {
+      tile = pend_tile;
+      mask = pend_mask;
+      pend_tile = -1;
+      return true;
+    }
+    int groups;
+    const int qb = peek(groups);
+    if (qb == 0x7FFFFFFF) return false;
+    consume(qb);
+    if (bs == 32) {
+      tile = qb >> 1;
+      mask = expand_groups(groups, 1 << (qb & 1));
+      // the other block of the same query tile, if attended too
+      int g2;
+      const int qb2 = peek(g2);
+      if (qb2 != 0x7FFFFFFF && (qb2 >> 1) == tile) {
+        consume(qb2);
+        mask |= expand_groups(g2, 1 << (qb2 & 1));
+      }
+    } else if (bs == 64) {
+      tile = qb;
+      mask = expand_groups(groups, 3);
+    } else {
+      tile = 2 * qb;
+      mask = expand_groups(groups, 3);
+      pend_tile = 2 * qb + 1;
+      pend_mask = mask;
+    }
+    return true;
+  }
+};
+
+// Validity bitmap of the 64 keys of key tile j (bit k set = attend).
 __device__ __forceinline__ uint64_t key_bits(const Problem& p, int b, int j) {
   const uint4* m4 = reinterpret_cast<const uint4*>(
-      p.key_mask + (size_t)b * p.L + (size_t)j * kBS);
+      p.key_mask + (size_t)b * p.L + (size_t)j * kTile);
   uint64_t bits = 0;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {
@@ -127,10 +365,23 @@ __device__ __forceinline__ uint64_t key_bits(const Problem& p, int b, int j) {
   return bits;
 }
 
-// TMA/tcgen05 path conditions shared by forward and backward.
+// Column-validity bitmap of a tile from its two mask bits for one group
+// (bit k set = column k belongs to an attended block).
+__device__ __forceinline__ uint64_t half_bits(int m2) {
+  return ((m2 & 1) ? 0x00000000FFFFFFFFull : 0ull) |
+         ((m2 & 2) ? 0xFFFFFFFF00000000ull : 0ull);
+}
+
+// Tensor-core path conditions shared by forward and backward.
 inline bool tc_shape_ok(const Problem& p) {
-  return p.dtype == BB_BF16 && p.bs == kBS && p.d == kHeadDim &&
-         10 + 2 * p.r <= kMaxT && (size_t)p.B * p.H * p.L < (1ull << 31);
+  if (p.dtype != BB_BF16 || p.d != kHeadDim) return false;
+  if (p.bs != 32 && p.bs != 64 && p.bs != 128) return false;
+  if (p.L % kTile != 0) return false;
+  if ((size_t)p.B * p.H * p.L >= (1ull << 31)) return false;
+  // tiles per middle item: 4 groups x (5 + r) blocks, each one tile (32),
+  // or 2 blocks per item x (5 + r) tiles (64), or (5 + r) x 2 tiles (128)
+  const int per = p.bs == 32 ? 4 * (5 + p.r) : 2 * (5 + p.r);
+  return per <= kMaxT;
 }
 
 }  // namespace bb

@@ -2,14 +2,12 @@
 // d 64) for sm_100a: TMA tile loads, tcgen05 MMAs with TMEM accumulators and
 // an online softmax, in a persistent warp-specialised kernel.
 //
-// Work item = two query blocks of one (b, h) sharing one 128-row MMA tile:
-//  * middle pair (i, i+1): the key blocks streamed are the union of the two
-//    attended sets A(i) and A(i+1) (window, the two global blocks, random
-//    blocks); each key block carries a 2-bit mask saying which half of the
-//    tile attends it.  Blocks i and i+1, 0 and nb-1 are always shared.
-//  * global chunk: rows 0 and nb-1 (which attend every key block) over a
-//    chunk of kChunk consecutive key blocks; partial (O, m, l) go to the
-//    workspace and fwd_combine_kernel merges the chunks.
+// Work item = 128 query rows of one (b, h) in one 128-row MMA tile (see
+// tc_common.cuh): a middle window streams the union of its row groups'
+// attended key tiles, each with a mask of which 32-row group attends which
+// 32 columns; a global item streams a chunk of all key tiles for the rows of
+// blocks 0 and nb-1 and writes partial (O, m, l) that fwd_combine_kernel
+// merges.  Blocks of 32, 64 and 128 tokens all map onto 64-token tiles.
 //
 // Roles (192 threads): warp 0 lane 0 issues TMA loads (Q pair once per item,
 // K and V per key block through a kNST-stage ring); warp 1 lane 0 issues the
@@ -123,13 +121,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
         const int row0 = L.bh * p.L;
-        const uint32_t qbytes = (L.blk[1] >= 0 ? 2u : 1u) * kTileBytes;
+        const uint32_t qbytes = (L.t[1] >= 0 ? 2u : 1u) * kTileBytes;
         mbar_expect_tx(&bars.q_full[slot], qbytes);
         uint8_t* q = Qs + slot * 2 * kTileBytes;
-        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.blk[0] * kBS);
-        if (L.blk[1] >= 0)
+        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.t[0] * kTile);
+        if (L.t[1] >= 0)
           tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
-                      row0 + L.blk[1] * kBS);
+                      row0 + L.t[1] * kTile);
         qissued[slot] = 1;
         qpar[slot] = ph;
         bool ok = true;
@@ -142,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
           mbar_expect_tx(&bars.kv_full[st], 2 * kTileBytes);
           uint8_t* kv = KVs + st * 2 * kTileBytes;
-          const int y = row0 + L.tile[t] * kBS;
+          const int y = row0 + L.tile[t] * kTile;
           tma_load_2d(kv, &tmK, &bars.kv_full[st], 0, y);
           tma_load_2d(kv + kTileBytes, &tmV, &bars.kv_full[st], 0, y);
           ++g;
@@ -245,7 +243,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // TMEM lane = tile row
     const int half = row >> 6;
-    const int hbit = 1 << half;
+    const int gshift = 2 * quarter;  // this warp's row group = its quarter
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const uint32_t tO = tmem + kColO + lane_off;
     const float c = p.scale * kLog2e;
@@ -263,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t uu = u + t;
         const int b2 = uu & 1;
         const uint32_t par = (uu >> 1) & 1;
-        const bool att = (L.mask[t] & hbit) != 0;
+        const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
+        const bool att = m2 != 0;
         if (!mbar_wait(&bars.s_full[b2], par, &abort_flag, p.status)) {
           ok = false;
           break;
@@ -294,22 +293,27 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
         if (att) {
           const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          const uint64_t hb = half_bits(m2);
           float mx;
-          if (kb == ~0ull && c > 0.f) {
+          if (kb == ~0ull && hb == ~0ull && c > 0.f) {
             float mx8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
             mx = max8(mx8) * c;
           } else {
+            // Columns outside the attended blocks are absent (-inf, p = 0);
+            // masked keys inside them get the finite offset.
 #pragma unroll
             for (int e = 0; e < 64; ++e)
-              z[e] = fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl);
+              z[e] = ((hb >> e) & 1ull)
+                         ? fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl)
+                         : -INFINITY;
             float mx8[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
             mx = max8(mx8);
           }
-          const bool scaled = !(kb == ~0ull && c > 0.f);
+          const bool scaled = !(kb == ~0ull && hb == ~0ull && c > 0.f);
           // Lazy running max: move it only when the row max exceeds it by
           // more than the threshold (or on the row's first attended tile).
           const bool first = (m == -INFINITY);
@@ -379,13 +383,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                      p.status))
         break;
       tc_fence_after();
-      const int blk = L.blk[half];
       const int r64 = row & 63;
-      const bool write = blk >= 0;
+      const bool write = (L.gvalid >> quarter) & 1;
       const float inv = L.global ? 1.f : 1.f / l;
-      const size_t grow = (size_t)L.bh * p.L + (size_t)(write ? blk : 0) * kBS + r64;
+      const size_t grow = (size_t)L.bh * p.L + (size_t)(write ? L.t[half] : 0) * kTile + r64;
       float* part = p.part +
-                    (((size_t)L.bh * a.nchunks + L.chunk) * 128 + row) * kPartStride;
+                    ((((size_t)L.bh * a.geo.n_git + L.gi) * a.geo.nchunks + L.chunk) * 128 +
+                     row) * kPartStride;
 #pragma unroll
       for (int q16 = 0; q16 < 4; ++q16) {
         uint32_t o[16];
@@ -435,39 +439,39 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// Merge the global rows' split partials: one warp per row, lanes over d.
+// Merge the global rows' split partials: one warp per row of a global item,
+// lanes over d; rows outside the global blocks are skipped.
 __global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
   const Problem& p = a.p;
-  const int nhalves = p.nb > 1 ? 2 : 1;
+  const Geom& g = a.geo;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t grow_id = (size_t)blockIdx.x * 8 + warp;  // over bh x half x 64
-  const size_t total = (size_t)p.B * p.H * nhalves * kBS;
-  if (grow_id >= total) return;
-  const int r64 = grow_id % kBS;
-  const int half = (grow_id / kBS) % nhalves;
-  const size_t bh = grow_id / (kBS * nhalves);
-  const int row = half * 64 + r64;
+  const size_t id = (size_t)blockIdx.x * 8 + warp;  // over bh x gi x 128
+  const size_t total = (size_t)p.B * p.H * g.n_git * 128;
+  if (id >= total) return;
+  const int row = id % 128;
+  const int gi = (id / 128) % g.n_git;
+  const size_t bh = id / (128 * g.n_git);
+  int t[2], gvalid;
+  item_rows(g, true, gi, t, gvalid);
+  if (!((gvalid >> (row >> 5)) & 1)) return;
+  const float* base = p.part + ((bh * g.n_git + gi) * g.nchunks * 128 + row) * kPartStride;
   float M = -INFINITY;
-  for (int c = 0; c < a.nchunks; ++c) {
-    const float* src = p.part + ((bh * a.nchunks + c) * 128 + row) * kPartStride;
-    M = fmaxf(M, src[64]);
-  }
-  float L = 0.f, o0 = 0.f, o1 = 0.f;
-  for (int c = 0; c < a.nchunks; ++c) {
-    const float* src = p.part + ((bh * a.nchunks + c) * 128 + row) * kPartStride;
+  for (int c = 0; c < g.nchunks; ++c) M = fmaxf(M, base[(size_t)c * 128 * kPartStride + 64]);
+  float Lsum = 0.f, o0 = 0.f, o1 = 0.f;
+  for (int c = 0; c < g.nchunks; ++c) {
+    const float* src = base + (size_t)c * 128 * kPartStride;
     const float w = ex2(src[64] - M);
-    L = fmaf(w, src[65], L);
+    Lsum = fmaf(w, src[65], Lsum);
     const float2 o = reinterpret_cast<const float2*>(src)[lane];
     o0 = fmaf(w, o.x, o0);
     o1 = fmaf(w, o.y, o1);
   }
-  const float inv = 1.f / L;
-  const int blk = half == 0 ? 0 : p.nb - 1;
-  const size_t grow = bh * p.L + (size_t)blk * kBS + r64;
+  const float inv = 1.f / Lsum;
+  const size_t grow = bh * p.L + (size_t)t[row >> 6] * kTile + (row & 63);
   reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) +
                               grow * kHeadDim)[lane] =
       pack_bf16(o0 * inv, o1 * inv);
-  if (lane == 0) p.lse_out[grow] = (M + __log2f(L)) * (1.0f / kLog2e);
+  if (lane == 0) p.lse_out[grow] = (M + __log2f(Lsum)) * (1.0f / kLog2e);
 }
 
 }  // namespace
@@ -475,8 +479,8 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
 // ---- host side ----------------------------------------------------------
 
 size_t tc_fwd_part_bytes(const Problem& p) {
-  const int nchunks = (p.nb + kChunk - 1) / kChunk;
-  return (size_t)p.B * p.H * nchunks * 128 * kPartStride * sizeof(float);
+  const Geom g = make_geom(p.L, p.bs);
+  return (size_t)p.B * p.H * g.n_git * g.nchunks * 128 * kPartStride * sizeof(float);
 }
 
 bool tc_fwd_supported(const Problem& p) { return tc_shape_ok(p); }
@@ -497,7 +501,7 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
   if (e != cudaSuccess) return e;
   e = marks->mark(s);
   if (e != cudaSuccess) return e;
-  const size_t rows = (size_t)p.B * p.H * (p.nb > 1 ? 2 : 1) * kBS;
+  const size_t rows = (size_t)p.B * p.H * a.geo.n_git * 128;
   fwd_combine_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(a);
   return cudaGetLastError();
 }

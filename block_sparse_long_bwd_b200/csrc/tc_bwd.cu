@@ -533,14 +533,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         if (lane == 0) {
+          // P^T / dS^T columns: K step kk (16 query rows) at kk * 8, plus 16
+          // for the second query half; low parts 16 columns further.
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tDV, tS + kk * 8, sdesc_sw128(gaddr + kk * 2048, 8192), idAcc,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tDV, tS + kk * 8 + (kk >> 1) * 16, sdesc_sw128(gaddr + kk * 2048, 8192),
+                   idAcc, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tDK, tDP + kk * 8, sdesc_sw128(qaddr + kk * 2048, 8192), idAcc,
-                   (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16, sdesc_sw128(qaddr + kk * 2048, 8192),
+                   idAcc, (t > 0 || kk > 0) ? 1u : 0u);
+          if (it.global) {
+            // Global key blocks sum over every query row: their P^T and
+            // dS^T also carry a bf16 low part, so the products keep ~16
+            // bits instead of 8.
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tDV, tS + kk * 8 + (kk >> 1) * 16 + 16,
+                     sdesc_sw128(gaddr + kk * 2048, 8192), idAcc, 1u);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16 + 16,
+                     sdesc_sw128(qaddr + kk * 2048, 8192), idAcc, 1u);
+          }
           mma_commit(&bars.qt_empty[st]);
         }
         __syncwarp();
@@ -583,29 +598,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         const int m2 = (mask >> gshift) & 3;  // attending query-column halves
-        const bool att = m2 != 0;
-        uint32_t P[32], dS[32];
+        const bool split = it.global;          // also write bf16 low parts
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
-        if (att && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
-                              p.status)) {
+        if (m2 && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
+                             p.status)) {
           ok = false;
           break;
         }
-        if (att) {
-          const float* NLs = reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
-          const float* Ds = NLs + 64;
+        const float* NLs =
+            reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
+        const float* Ds = NLs + 64;
+        // Per query-column half hc (32 columns): read S^T and dP^T, then
+        // write P^T and dS^T (bf16 pairs, 16 columns) over the columns just
+        // read: high parts at 32 hc, low parts (global items) at 32 hc + 16.
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            if (!((m2 >> hc) & 1)) {  // query rows outside attending blocks
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                P[hc * 16 + e] = 0u;
-                dS[hc * 16 + e] = 0u;
-              }
-              continue;
-            }
-            uint32_t s[32], dp[32];
-            tmem_ld32(tS + hc * 32 + lane_off, s);
+        for (int hc = 0; hc < 2; ++hc) {
+          uint32_t ph[16], dh[16], pl[16], dl[16];
+          if ((m2 >> hc) & 1) {
+            uint32_t sv[32], dp[32];
+            tmem_ld32(tS + hc * 32 + lane_off, sv);
             tmem_ld32(tDP + hc * 32 + lane_off, dp);
             tmem_ld_wait();
 #pragma unroll
@@ -618,38 +629,32 @@ __global__ void __launch_bounds__(kThreads, 2)
               float pv[4], dv[4];
 #pragma unroll
               for (int x = 0; x < 4; ++x) {
-                pv[x] = ex2(fmaf(__uint_as_float(s[e + x]), c, nls[x] + off));
+                pv[x] = ex2(fmaf(__uint_as_float(sv[e + x]), c, nls[x] + off));
                 dv[x] = pv[x] * (__uint_as_float(dp[e + x]) - dds[x]);
               }
-              P[col >> 1] = pack_bf16(pv[0], pv[1]);
-              P[(col >> 1) + 1] = pack_bf16(pv[2], pv[3]);
-              dS[col >> 1] = pack_bf16(dv[0], dv[1]);
-              dS[(col >> 1) + 1] = pack_bf16(dv[2], dv[3]);
+#pragma unroll
+              for (int x = 0; x < 2; ++x) {
+                const int o = (e >> 1) + x;
+                ph[o] = pack_bf16(pv[2 * x], pv[2 * x + 1]);
+                dh[o] = pack_bf16(dv[2 * x], dv[2 * x + 1]);
+                if (split) {
+                  pl[o] = pack_bf16(pv[2 * x] - __uint_as_float(ph[o] << 16),
+                                    pv[2 * x + 1] - __uint_as_float(ph[o] & 0xFFFF0000u));
+                  dl[o] = pack_bf16(dv[2 * x] - __uint_as_float(dh[o] << 16),
+                                    dv[2 * x + 1] - __uint_as_float(dh[o] & 0xFFFF0000u));
+                }
+              }
             }
-          }
-        } else {
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            P[e] = 0u;
-            dS[e] = 0u;
+            for (int e = 0; e < 16; ++e) ph[e] = dh[e] = pl[e] = dl[e] = 0u;
           }
-        }
-        {
-          uint32_t a0[16], a1[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            a0[e] = P[e];
-            a1[e] = P[16 + e];
+          tmem_st16(tS + hc * 32 + lane_off, ph);
+          tmem_st16(tDP + hc * 32 + lane_off, dh);
+          if (split) {
+            tmem_st16(tS + hc * 32 + 16 + lane_off, pl);
+            tmem_st16(tDP + hc * 32 + 16 + lane_off, dl);
           }
-          tmem_st16(tS + lane_off, a0);
-          tmem_st16(tS + 16 + lane_off, a1);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            a0[e] = dS[e];
-            a1[e] = dS[16 + e];
-          }
-          tmem_st16(tDP + lane_off, a0);
-          tmem_st16(tDP + 16 + lane_off, a1);
         }
         tmem_st_wait();
         tc_fence_before();

@@ -1,6 +1,6 @@
 // Backward preprocessing: D = rowsum(dO * O) and the transposed block
 // adjacency (for each key block j, the sorted query blocks i with j in A(i)).
-#include "common.cuh"
+#include "tc_common.cuh"
 
 namespace bb {
 namespace {
@@ -135,6 +135,67 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
       L[c + 1] = x;
     }
   }
+  if (!p.qplan) return;  // CUDA-core path: the CSR is all it needs
+
+  // Tensor-core plans of this head.  Query side: the key tiles of every
+  // item.  Key side: each item's walk over the query tiles that attend its
+  // key rows (merging this head's CSR lists, complete after the barrier).
+  __syncthreads();
+  const Geom g = make_geom(p.L, p.bs);
+  TileList* qplan = static_cast<TileList*>(p.qplan) + (size_t)h * g.per_bh;
+  for (int loc = tid; loc < g.per_bh; loc += kCsrThreads)
+    if (!build_tile_list(p, g, h, loc, qplan[loc])) set_status(p.status, BB_ERR_BAD_TABLE);
+  int* kof = p.kof + (size_t)h * (g.per_bh + 1);
+  uint32_t* kplan = p.kplan + (size_t)h * p.kcap;
+  // pass 1: walk lengths, into tsum-chunked exclusive offsets
+  const int kchunk = (g.per_bh + kCsrThreads - 1) / kCsrThreads;
+  const int k0 = tid * kchunk, k1 = min(g.per_bh, k0 + kchunk);
+  int klocal = 0;
+  for (int loc = k0; loc < k1; ++loc) {
+    KeyWalk w;
+    w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, h * g.per_bh + loc);
+    int tile, mask, n = 0;
+    while (w.next(tile, mask)) ++n;
+    kof[loc] = n;
+    klocal += n;
+  }
+  __syncthreads();
+  tsum[tid] = klocal;
+  __syncthreads();
+  for (int step = 1; step < kCsrThreads; step <<= 1) {
+    int add = tid >= step ? tsum[tid - step] : 0;
+    __syncthreads();
+    tsum[tid] += add;
+    __syncthreads();
+  }
+  int krun = tsum[tid] - klocal;
+  for (int loc = k0; loc < k1; ++loc) {
+    const int n = kof[loc];
+    kof[loc] = krun;
+    krun += n;
+  }
+  if (tid == kCsrThreads - 1) kof[g.per_bh] = tsum[kCsrThreads - 1];
+  __syncthreads();
+  // pass 2: fill (the planner sized kcap for the worst case of this table)
+  for (int loc = k0; loc < k1; ++loc) {
+    KeyWalk w;
+    w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, h * g.per_bh + loc);
+    int tile, mask, e = kof[loc];
+    while (w.next(tile, mask)) {
+      if (e < p.kcap) kplan[e] = kentry(tile, mask);
+      ++e;
+    }
+  }
+}
+
+// Query-side plans for the forward: one thread per (head, item).
+__global__ void __launch_bounds__(128) plan_q_kernel(Problem p) {
+  const Geom g = make_geom(p.L, p.bs);
+  const int id = blockIdx.x * 128 + threadIdx.x;
+  if (id >= p.H * g.per_bh) return;
+  const int h = id / g.per_bh, loc = id % g.per_bh;
+  TileList* qplan = static_cast<TileList*>(p.qplan);
+  if (!build_tile_list(p, g, h, loc, qplan[id])) set_status(p.status, BB_ERR_BAD_TABLE);
 }
 
 }  // namespace
@@ -146,6 +207,26 @@ cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s) {
     bwd_pre_kernel<float><<<grid, 256, 0, s>>>(p);
   else
     bwd_pre_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+size_t tc_items_per_bh(const Problem& p) { return make_geom(p.L, p.bs).per_bh; }
+
+size_t tc_qplan_bytes(const Problem& p) {
+  return (size_t)p.H * tc_items_per_bh(p) * sizeof(TileList);
+}
+
+// Upper bound of key-side walk entries per head: every entry of a middle
+// window stands for at least one attended (query block, key block) pair
+// (two tiles per block at block size 128); global items visit all tiles.
+int tc_kplan_cap(const Problem& p) {
+  const Geom g = make_geom(p.L, p.bs);
+  return 2 * pair_cap(p.nb, p.r) + g.n_git * g.nt + 64;
+}
+
+cudaError_t launch_plan_q(const Problem& p, cudaStream_t s) {
+  const int n = p.H * (int)tc_items_per_bh(p);
+  plan_q_kernel<<<(n + 127) / 128, 128, 0, s>>>(p);
   return cudaGetLastError();
 }
 

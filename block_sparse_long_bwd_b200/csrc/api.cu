@@ -21,6 +21,8 @@ WsLayout ws_layout(const Problem& p, int pass) {
   if (pass == 0 && tc_fwd_supported(p)) {
     w.part_off = off;
     off = align_up(off + tc_fwd_part_bytes(p), 256);
+    w.qplan_off = off;
+    off = align_up(off + tc_qplan_bytes(p), 256);
     w.total = off;
     return w;
   }
@@ -34,6 +36,12 @@ WsLayout ws_layout(const Problem& p, int pass) {
     if (tc_bwd_supported(p)) {
       w.part_off = off;
       off = align_up(off + tc_bwd_extra_bytes(p), 256);
+      w.qplan_off = off;
+      off = align_up(off + tc_qplan_bytes(p), 256);
+      w.kof_off = off;
+      off = align_up(off + (size_t)p.H * (tc_items_per_bh(p) + 1) * sizeof(int), 256);
+      w.kplan_off = off;
+      off = align_up(off + (size_t)p.H * tc_kplan_cap(p) * sizeof(uint32_t), 256);
       w.total = off;
       return w;
     }
@@ -111,6 +119,12 @@ int carve(Problem* p, int pass, void* ws, size_t ws_bytes) {
   }
   p->part = (float*)(base + w.part_off);
   p->part_floats = (ws_bytes - w.part_off) / sizeof(float);
+  if (w.qplan_off) p->qplan = base + w.qplan_off;
+  if (w.kof_off) {
+    p->kof = (int*)(base + w.kof_off);
+    p->kplan = (uint32_t*)(base + w.kplan_off);
+    p->kcap = tc_kplan_cap(*p);
+  }
   return BB_OK;
 }
 
@@ -202,6 +216,8 @@ static int fwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   if (tc_fwd_supported(p)) {
     TensorMaps tm;
     if (!encode_tensor_maps(p, 0, &tm)) return BB_ERR_CUDA;
+    if (launch_plan_q(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
     if (launch_tc_fwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
   } else {
     if (launch_simt_fwd(p, s) != cudaSuccess) return BB_ERR_CUDA;
@@ -263,7 +279,7 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
 // Names of the launches each pass makes, in order (kept beside the
 // dispatch in fwd_impl / bwd_impl).
 static const char* const kFwdSimt[] = {"simt_fwd"};
-static const char* const kFwdTc[] = {"tc_fwd", "fwd_combine"};
+static const char* const kFwdTc[] = {"plan", "tc_fwd", "fwd_combine"};
 static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
 static const char* const kBwdTc[] = {"csr_build", "tc_dq", "tc_dkdv",
@@ -278,7 +294,7 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
   if (pass == 0) {
     const bool tc = tc_fwd_supported(p);
     *names = tc ? kFwdTc : kFwdSimt;
-    *n = tc ? 2 : 1;
+    *n = tc ? 3 : 1;
   } else {
     *names = tc_bwd_supported(p) ? kBwdTc : kBwdSimt;
     *n = 4;

@@ -45,6 +45,11 @@ struct Problem {
   int csr_cap;
   float* part;       // split partials (tensor-core path)
   size_t part_floats;
+  // tensor-core plans (see tc_common.cuh)
+  void* qplan;       // [H][items per (b, h)] tile lists, query side
+  int* kof;          // [H][items per (b, h) + 1] offsets of the key-side walks
+  uint32_t* kplan;   // [H][kcap] key-side walk entries
+  int kcap;
 };
 
 // Upper bound of attended (query block, key block) pairs per head.
@@ -52,7 +57,9 @@ inline int pair_cap(int nb, int r) { return nb * (7 + r) + 8; }
 
 // Workspace layout, identical for sizing and for carving.
 struct WsLayout {
-  size_t status_off, D_off, offs_off, list_off, part_off, total;
+  size_t status_off, D_off, offs_off, list_off, part_off;
+  size_t qplan_off, kof_off, kplan_off;  // tensor-core plans (0: none)
+  size_t total;
 };
 WsLayout ws_layout(const Problem& p, int pass);
 
@@ -88,6 +95,10 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);
 
 bool tc_bwd_supported(const Problem& p);
+size_t tc_qplan_bytes(const Problem& p);
+int tc_kplan_cap(const Problem& p);
+size_t tc_items_per_bh(const Problem& p);
+cudaError_t launch_plan_q(const Problem& p, cudaStream_t s);
 size_t tc_bwd_extra_bytes(const Problem& p);
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);

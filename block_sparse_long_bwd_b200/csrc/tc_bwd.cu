@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                  const __grid_constant__ CUtensorMap tmG) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ DqBars bars;
-  __shared__ ItemList lists[2];
+  __shared__ TileList lists[2];  // bulk-copy destinations (16-byte aligned)
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -126,15 +126,21 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(&bars.list_empty[slot], ((k >> 1) & 1) ^ 1, &abort_flag,
                        p.status))
           break;
-        ItemList& L = lists[slot];
-        build_pair_item(a, item, L);
-        mbar_arrive(&bars.list_full[slot]);
-        if (!mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
-        const int row0 = L.bh * p.L;
-        const int nh = L.t[1] >= 0 ? 2 : 1;
+        // Planned key-tile list: one bulk copy into the slot.
+        const ItemMeta m = item_meta(a.geo, p.H, item);
+        const TileList& L = lists[slot];
+        mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
+        bulk_load(&lists[slot],
+                  static_cast<const TileList*>(p.qplan) + (size_t)m.h * a.geo.per_bh + m.loc,
+                  sizeof(TileList), &bars.list_full[slot]);
+        if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status) ||
+            !mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status))
+          break;
+        const int row0 = m.bh * p.L;
+        const int nh = m.t[1] >= 0 ? 2 : 1;
         mbar_expect_tx(&bars.q_full, 2u * nh * kTileBytes);
         for (int hh = 0; hh < nh; ++hh) {
-          const int y = row0 + L.t[hh] * kTile;
+          const int y = row0 + m.t[hh] * kTile;
           tma_load_2d(Qs + hh * kTileBytes, &tmQ, &bars.q_full, 0, y);
           tma_load_2d(Gs + hh * kTileBytes, &tmG, &bars.q_full, 0, y);
         }
@@ -249,10 +255,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int slot = k & 1;
       if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
-      const ItemList& L = lists[slot];
+      const TileList& L = lists[slot];
+      const ItemMeta im = item_meta(a.geo, p.H, item);
       const int n = L.n;
-      const bool rvalid = (L.gvalid >> quarter) & 1;
-      const size_t grow = (size_t)L.bh * p.L + (size_t)(rvalid ? L.t[half] : 0) * kTile + r64;
+      const bool rvalid = (im.gvalid >> quarter) & 1;
+      const size_t grow = (size_t)im.bh * p.L + (size_t)(rvalid ? im.t[half] : 0) * kTile + r64;
       float nl2 = 0.f, Dr = 0.f;
       if (rvalid) {
         nl2 = -p.lse[grow] * kLog2e;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int e = 0; e < 8; ++e) Dr = fmaf(fo[e], fg[e], Dr);
         }
-        if (!L.global || L.chunk == 0) {
+        if (!im.global || im.chunk == 0) {
           ba.D[grow] = Dr;
           ba.NL[grow] = nl2;
         }
@@ -281,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
         uint32_t dS[32];
         if (m2) {
-          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          const uint64_t kb = p.key_mask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
 #pragma unroll
           for (int hc = 0; hc < 2; ++hc) {
             if (!((m2 >> hc) & 1)) {  // keys outside the attended blocks
@@ -333,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.dq_empty);
       if (rvalid) {
-        if (!L.global) {
+        if (!im.global) {
           uint4* dst = reinterpret_cast<uint4*>(
               static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim);
 #pragma unroll
@@ -348,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         } else {
           float4* dst = reinterpret_cast<float4*>(
-              ba.dqpart + ((((size_t)L.bh * a.geo.n_git + L.gi) * a.geo.nchunks + L.chunk) *
+              ba.dqpart + ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) *
                                128 + row) * 64);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -437,8 +444,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t kp_par = 0;
       for (int k = 0, item = blockIdx.x; item < ba.qa.items;
            ++k, item += gridDim.x) {
-        KeyWalk it;
-        it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
+        const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+        const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
+        const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
+        const int e0 = wof[it.loc], e1 = wof[it.loc + 1];
         if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
@@ -450,9 +459,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         kp_issued = 1;
         kp_par = k & 1;
-        int i, mask;
         bool ok = true;
-        while (it.next(i, mask)) {
+        for (int e = e0; e < e1; ++e) {
+          const int i = (int)(__ldg(walk + e) & 0xFFFFu);  // query tile
           const int st = g % kQStages;
           if (!mbar_wait(&bars.qt_empty[st], ((g / kQStages) & 1) ^ 1,
                          &abort_flag, p.status)) {
@@ -495,12 +504,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     bool ok = true;
     for (int k = 0, item = blockIdx.x; item < ba.qa.items && ok;
          ++k, item += gridDim.x) {
-      KeyWalk it;
-      it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
+      const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+      const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
+      const int nwalk = wof[it.loc + 1] - wof[it.loc];
       if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
-      int i, mask, t = 0;
-      while (it.next(i, mask)) {
+      for (int t = 0; t < nwalk;) {
         const int st = g % kQStages;
         // S^T and dP^T overwrite the buffers that hold the previous tile's
         // P^T and dS^T; the dV / dK MMAs reading those were issued earlier by
@@ -580,17 +589,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float mvl = p.mask_value * kLog2e;
     uint32_t g = 0, u = 0;
     for (int k = 0, item = blockIdx.x; item < ba.qa.items; ++k, item += gridDim.x) {
-      KeyWalk it;
-      it.init(ba.qa, p.csr_offs, p.csr_list, p.csr_cap, item);
+      const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+      const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
+      const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
+      const int e0 = wof[it.loc], e1 = wof[it.loc + 1];
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;
       float off = 0.f;
       if (rvalid && p.key_mask)
         off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
-      int i, mask;
       bool ok = true;
-      while (it.next(i, mask)) {
+      for (int e = e0; e < e1; ++e) {
+        const int mask = (int)(__ldg(walk + e) >> 16);
         const int st = g % kQStages;
         if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
           ok = false;

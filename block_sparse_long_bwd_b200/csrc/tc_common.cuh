@@ -93,15 +93,24 @@ __host__ __device__ __forceinline__ void for_block_tiles(const Geom& g, int j, F
   }
 }
 
-struct ItemList {
+// The tiles an item visits, planned once per call (one per (head, item):
+// lists do not depend on the batch index) and copied into shared memory by
+// the producer with one bulk copy.  208 bytes, a multiple of 16.
+struct __align__(16) TileList {
   int n;
+  int pad[3];
+  int16_t tile[kMaxT];
+  uint8_t mask[kMaxT];
+};
+static_assert(sizeof(TileList) % 16 == 0, "bulk-copy size");
+
+// What an item covers, computable from its index alone.
+struct ItemMeta {
+  int bh, b, h, loc;
   int global;   // 1 = global item
-  int bh, b;
   int t[2];     // row tile of half 0 / 1 (-1: absent)
   int gvalid;   // 4-bit: groups whose rows this item produces
   int gi, chunk;
-  int16_t tile[kMaxT];
-  uint8_t mask[kMaxT];
 };
 
 struct PairArgs {
@@ -118,7 +127,7 @@ inline PairArgs make_pair_args(const Problem& p) {
   return a;
 }
 
-__host__ __device__ __forceinline__ void list_add(ItemList& L, int tile, int bits) {
+__host__ __device__ __forceinline__ void list_add(TileList& L, int tile, int bits) {
   for (int c = 0; c < L.n; ++c)
     if (L.tile[c] == tile) {
       L.mask[c] |= (uint8_t)bits;
@@ -158,42 +167,50 @@ __host__ __device__ __forceinline__ int expand_groups(int groups, int halves) {
   return m;
 }
 
-// Fills L for query-side item `item` ((b, h)-major; within one (b, h) the
-// global items' chunks come first, then the middle windows).
-__host__ __device__ inline void build_pair_item(const PairArgs& a, int item,
-                                                ItemList& L) {
-  const Problem& p = a.p;
-  const Geom& g = a.geo;
-  const int bh = item / g.per_bh, loc = item % g.per_bh;
-  L.n = 0;
-  L.bh = bh;
-  L.b = bh / p.H;
-  const int h = bh % p.H;
+// Metadata of item `item` ((b, h)-major; within one (b, h) the global items'
+// chunks come first, then the middle windows).  Same decoding on both sides.
+__host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int item) {
+  ItemMeta m;
+  m.bh = item / g.per_bh;
+  m.loc = item % g.per_bh;
+  m.b = m.bh / H;
+  m.h = m.bh % H;
   const int nglob = g.n_git * g.nchunks;
-  if (loc < nglob) {
-    L.global = 1;
-    L.gi = loc / g.nchunks;
-    L.chunk = loc % g.nchunks;
-    item_rows(g, true, L.gi, L.t, L.gvalid);
-    const int m = expand_groups(L.gvalid, 3);
-    const int j1 = g.nt < (L.chunk + 1) * kChunk ? g.nt : (L.chunk + 1) * kChunk;
-    for (int j = L.chunk * kChunk; j < j1; ++j) {
+  if (m.loc < nglob) {
+    m.global = 1;
+    m.gi = m.loc / g.nchunks;
+    m.chunk = m.loc % g.nchunks;
+    item_rows(g, true, m.gi, m.t, m.gvalid);
+  } else {
+    m.global = 0;
+    m.gi = 0;
+    m.chunk = 0;
+    item_rows(g, false, g.w_first + (m.loc - nglob), m.t, m.gvalid);
+  }
+  return m;
+}
+
+// Plans the key tiles of query-side item (h, loc) into L.  Returns false if
+// the random table held an entry outside [-1, nb) (ignored).
+__host__ __device__ inline bool build_tile_list(const Problem& p, const Geom& g,
+                                                int h, int loc, TileList& L) {
+  ItemMeta m = item_meta(g, p.H, h * g.per_bh + loc);  // b = 0: lists ignore b
+  L.n = 0;
+  bool table_ok = true;
+  if (m.global) {
+    const int bits = expand_groups(m.gvalid, 3);
+    const int j1 = g.nt < (m.chunk + 1) * kChunk ? g.nt : (m.chunk + 1) * kChunk;
+    for (int j = m.chunk * kChunk; j < j1; ++j) {
       L.tile[L.n] = (int16_t)j;
-      L.mask[L.n] = (uint8_t)m;
+      L.mask[L.n] = (uint8_t)bits;
       ++L.n;
     }
-    return;
+    return true;
   }
-  L.global = 0;
-  L.gi = 0;
-  L.chunk = 0;
-  const int w = g.w_first + (loc - nglob);
-  item_rows(g, false, w, L.t, L.gvalid);
   const int nb = g.nb;
-  int last_blk = -1;
   for (int gr = 0; gr < 4; ++gr) {
-    if (!(L.gvalid & (1 << gr))) continue;
-    const int i = block_of(g, L.t[gr >> 1] * kTile + 32 * (gr & 1));
+    if (!(m.gvalid & (1 << gr))) continue;
+    const int i = block_of(g, m.t[gr >> 1] * kTile + 32 * (gr & 1));
     const int gbits = 1 << (2 * gr);
     auto add_block = [&](int j) {
       for_block_tiles(g, j, [&](int tile, int halves) {
@@ -210,15 +227,18 @@ __host__ __device__ inline void build_pair_item(const PairArgs& a, int item,
       const int j = row[c];
       if (j == -1) continue;
       if (j < 0 || j >= nb) {
-#ifdef __CUDA_ARCH__
-        if (i != last_blk) set_status(p.status, BB_ERR_BAD_TABLE);
-#endif
+        table_ok = false;
         continue;
       }
       add_block(j);
     }
-    last_blk = i;
   }
+  return table_ok;
+}
+
+// Key-side walk entries: query tile in the low 16 bits, mask in bits 16-23.
+__host__ __device__ __forceinline__ uint32_t kentry(int tile, int mask) {
+  return (uint32_t)tile | ((uint32_t)mask << 16);
 }
 
 // Walk of one key-side item over the query tiles that attend it, with the
@@ -239,33 +259,28 @@ struct KeyWalk {
   int bs;
   int pend_tile, pend_mask;  // block 128: second tile of a query block
 
-  __host__ __device__ void init(const PairArgs& a, const int* csr_offs,
-                       const int* csr_list, int csr_cap, int item) {
-    const Problem& p = a.p;
-    const Geom& g = a.geo;
-    bh = item / g.per_bh;
-    b = bh / p.H;
-    const int h = bh % p.H;
-    const int loc = item % g.per_bh;
-    const int nglob = g.n_git * g.nchunks;
+  __host__ __device__ void init(const Geom& g, int H, const int* csr_offs,
+                                const int* csr_list, int csr_cap, int item) {
+    const ItemMeta m = item_meta(g, H, item);
+    bh = m.bh;
+    b = m.b;
+    const int h = m.h;
     bs = g.bs;
     pend_tile = -1;
     pend_mask = 0;
     nl = 0;
-    if (loc < nglob) {
-      global = 1;
-      gi = loc / g.nchunks;
-      chunk = loc % g.nchunks;
-      item_rows(g, true, gi, t, gvalid);
+    global = m.global;
+    gi = m.gi;
+    chunk = m.chunk;
+    t[0] = m.t[0];
+    t[1] = m.t[1];
+    gvalid = m.gvalid;
+    if (global) {
       gmask = expand_groups(gvalid, 3);
       cur = chunk * kChunk;
       end = g.nt < cur + kChunk ? g.nt : cur + kChunk;
       return;
     }
-    global = 0;
-    gi = 0;
-    chunk = 0;
-    item_rows(g, false, g.w_first + (loc - nglob), t, gvalid);
     const int* offs = csr_offs + (size_t)h * (g.nb + 1);
     const int* list = csr_list + (size_t)h * csr_cap;
     for (int gr = 0; gr < 4; ++gr) {

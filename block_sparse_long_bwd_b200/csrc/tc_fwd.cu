@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                   const __grid_constant__ CUtensorMap tmV) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
-  __shared__ ItemList lists[2];
+  __shared__ TileList lists[2];  // bulk-copy destinations (16-byte aligned)
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -115,19 +115,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t ph = (k >> 1) & 1;
         if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
-        ItemList& L = lists[slot];
-        build_pair_item(a, item, L);
-        mbar_arrive(&bars.list_full[slot]);
-        if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
+        // The item's key-tile list was planned before this kernel: one bulk
+        // copy into the slot (the producer waits for it like the others).
+        const ItemMeta m = item_meta(a.geo, p.H, item);
+        const TileList& L = lists[slot];
+        mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
+        bulk_load(&lists[slot],
+                  static_cast<const TileList*>(p.qplan) + (size_t)m.h * a.geo.per_bh + m.loc,
+                  sizeof(TileList), &bars.list_full[slot]);
+        if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status) ||
+            !mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
-        const int row0 = L.bh * p.L;
-        const uint32_t qbytes = (L.t[1] >= 0 ? 2u : 1u) * kTileBytes;
+        const int row0 = m.bh * p.L;
+        const uint32_t qbytes = (m.t[1] >= 0 ? 2u : 1u) * kTileBytes;
         mbar_expect_tx(&bars.q_full[slot], qbytes);
         uint8_t* q = Qs + slot * 2 * kTileBytes;
-        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + L.t[0] * kTile);
-        if (L.t[1] >= 0)
+        tma_load_2d(q, &tmQ, &bars.q_full[slot], 0, row0 + m.t[0] * kTile);
+        if (m.t[1] >= 0)
           tma_load_2d(q + kTileBytes, &tmQ, &bars.q_full[slot], 0,
-                      row0 + L.t[1] * kTile);
+                      row0 + m.t[1] * kTile);
         qissued[slot] = 1;
         qpar[slot] = ph;
         bool ok = true;
@@ -253,7 +259,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
       if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
-      const ItemList& L = lists[slot];
+      const TileList& L = lists[slot];
+      const ItemMeta im = item_meta(a.geo, p.H, item);
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
         if (att) {
-          const uint64_t kb = p.key_mask ? key_bits(p, L.b, L.tile[t]) : ~0ull;
+          const uint64_t kb = p.key_mask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
           const uint64_t hb = half_bits(m2);
           float mx;
           if (kb == ~0ull && hb == ~0ull && c > 0.f) {
@@ -384,11 +391,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         break;
       tc_fence_after();
       const int r64 = row & 63;
-      const bool write = (L.gvalid >> quarter) & 1;
-      const float inv = L.global ? 1.f : 1.f / l;
-      const size_t grow = (size_t)L.bh * p.L + (size_t)(write ? L.t[half] : 0) * kTile + r64;
+      const bool write = (im.gvalid >> quarter) & 1;
+      const float inv = im.global ? 1.f : 1.f / l;
+      const size_t grow = (size_t)im.bh * p.L + (size_t)(write ? im.t[half] : 0) * kTile + r64;
       float* part = p.part +
-                    ((((size_t)L.bh * a.geo.n_git + L.gi) * a.geo.nchunks + L.chunk) * 128 +
+                    ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) * 128 +
                      row) * kPartStride;
 #pragma unroll
       for (int q16 = 0; q16 < 4; ++q16) {
@@ -399,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           float v[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(o[e]) * inv;
-          if (!L.global) {
+          if (!im.global) {
             uint4* dst = reinterpret_cast<uint4*>(
                 static_cast<__nv_bfloat16*>(p.out) + grow * kHeadDim + q16 * 16);
             dst[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
@@ -421,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_arrive(&bars.list_empty[slot]);
       }
       if (write) {
-        if (!L.global) {
+        if (!im.global) {
           p.lse_out[grow] = (m + __log2f(l)) * (1.0f / kLog2e);
         } else {
           part[64] = m;

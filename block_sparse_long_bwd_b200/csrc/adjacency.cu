@@ -135,67 +135,164 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
       L[c + 1] = x;
     }
   }
-  if (!p.qplan) return;  // CUDA-core path: the CSR is all it needs
+}
 
-  // Tensor-core plans of this head.  Query side: the key tiles of every
-  // item.  Key side: each item's walk over the query tiles that attend its
-  // key rows (merging this head's CSR lists, complete after the barrier).
-  __syncthreads();
-  const Geom g = make_geom(p.L, p.bs);
-  TileList* qplan = static_cast<TileList*>(p.qplan) + (size_t)h * g.per_bh;
-  for (int loc = tid; loc < g.per_bh; loc += kCsrThreads)
-    if (!build_tile_list(p, g, h, loc, qplan[loc])) set_status(p.status, BB_ERR_BAD_TABLE);
-  int* kof = p.kof + (size_t)h * (g.per_bh + 1);
-  uint32_t* kplan = p.kplan + (size_t)h * p.kcap;
-  // pass 1: walk lengths, into tsum-chunked exclusive offsets
-  const int kchunk = (g.per_bh + kCsrThreads - 1) / kCsrThreads;
-  const int k0 = tid * kchunk, k1 = min(g.per_bh, k0 + kchunk);
-  int klocal = 0;
-  for (int loc = k0; loc < k1; ++loc) {
-    KeyWalk w;
-    w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, h * g.per_bh + loc);
-    int tile, mask, n = 0;
-    while (w.next(tile, mask)) ++n;
-    kof[loc] = n;
-    klocal += n;
-  }
-  __syncthreads();
-  tsum[tid] = klocal;
-  __syncthreads();
-  for (int step = 1; step < kCsrThreads; step <<= 1) {
-    int add = tid >= step ? tsum[tid - step] : 0;
-    __syncthreads();
-    tsum[tid] += add;
-    __syncthreads();
-  }
-  int krun = tsum[tid] - klocal;
-  for (int loc = k0; loc < k1; ++loc) {
-    const int n = kof[loc];
-    kof[loc] = krun;
-    krun += n;
-  }
-  if (tid == kCsrThreads - 1) kof[g.per_bh] = tsum[kCsrThreads - 1];
-  __syncthreads();
-  // pass 2: fill (the planner sized kcap for the worst case of this table)
-  for (int loc = k0; loc < k1; ++loc) {
-    KeyWalk w;
-    w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, h * g.per_bh + loc);
-    int tile, mask, e = kof[loc];
-    while (w.next(tile, mask)) {
-      if (e < p.kcap) kplan[e] = kentry(tile, mask);
-      ++e;
+constexpr int kPlanWarps = 4;
+constexpr int kStageCap = 512;  // CSR entries staged per warp (key side)
+
+// Bitonic sort of 128 ints in shared memory by one warp.
+__device__ __forceinline__ void warp_sort128(int* v, int lane) {
+  for (int k = 2; k <= 128; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = lane + 32 * r;
+        const int x = i ^ j;
+        if (x > i) {
+          const int a = v[i], b = v[x];
+          const bool up = (i & k) == 0;
+          if ((a > b) == up) {
+            v[i] = b;
+            v[x] = a;
+          }
+        }
+      }
+      __syncwarp();
     }
   }
 }
 
-// Query-side plans for the forward: one thread per (head, item).
-__global__ void __launch_bounds__(128) plan_q_kernel(Problem p) {
+// Query-side plan of item (h, loc), one warp: every (group, attended block,
+// tile) candidate as (tile << 8 | mask bits), sorted, equal tiles merged.
+__device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
+                            int* cand, int lane) {
+  const ItemMeta m = item_meta(g, p.H, h * g.per_bh + loc);
+  TileList& L = static_cast<TileList*>(p.qplan)[(size_t)h * g.per_bh + loc];
+  if (m.global) {
+    const int bits = expand_groups(m.gvalid, 3);
+    const int j0 = m.chunk * kChunk, j1 = min(g.nt, j0 + kChunk);
+    if (lane < j1 - j0) {
+      L.tile[lane] = (int16_t)(j0 + lane);
+      L.mask[lane] = (uint8_t)bits;
+    }
+    if (lane == 0) L.n = j1 - j0;
+    return;
+  }
+  const int S = 5 + p.r, T = g.bs == 128 ? 2 : 1;
+  bool bad = false;
+  for (int idx = lane; idx < 128; idx += 32) {
+    int v = 0x7FFFFFFF;
+    const int gr = idx / (S * T), s = (idx / T) % S, tt = idx % T;
+    if (gr < 4 && (m.gvalid >> gr) & 1) {
+      const int i = block_of(g, m.t[gr >> 1] * kTile + 32 * (gr & 1));
+      int j;
+      if (s < 5) {
+        const int base[5] = {0, i - 1, i, i + 1, g.nb - 1};
+        j = base[s];
+      } else {
+        j = p.rand_idx[((size_t)h * g.nb + i) * p.r + (s - 5)];
+        if (j != -1 && (j < 0 || j >= g.nb)) bad = true;
+        if (j < 0 || j >= g.nb) j = -1;
+      }
+      if (j >= 0) {
+        int tile, halves;
+        if (g.bs == 32) {
+          tile = j >> 1;
+          halves = 1 << (j & 1);
+        } else if (g.bs == 64) {
+          tile = j;
+          halves = 3;
+        } else {
+          tile = 2 * j + tt;
+          halves = 3;
+        }
+        v = (tile << 8) | (halves << (2 * gr));
+      }
+    }
+    cand[idx] = v;
+  }
+  if (bad) set_status(p.status, BB_ERR_BAD_TABLE);
+  __syncwarp();
+  warp_sort128(cand, lane);
+  int base_pos = 0;
+  for (int r = 0; r < 4; ++r) {
+    const int e = lane + 32 * r;
+    const int v = cand[e];
+    const bool head = v != 0x7FFFFFFF && (e == 0 || (cand[e - 1] >> 8) != (v >> 8));
+    int bits = 0;
+    if (head) {
+      for (int x = e; x < 128 && (cand[x] >> 8) == (v >> 8) && cand[x] != 0x7FFFFFFF; ++x)
+        bits |= cand[x] & 0xFF;
+    }
+    const unsigned hb = __ballot_sync(0xFFFFFFFFu, head);
+    if (head) {
+      const int pos = base_pos + __popc(hb & ((1u << lane) - 1));
+      if (pos < kMaxT) {
+        L.tile[pos] = (int16_t)(v >> 8);
+        L.mask[pos] = (uint8_t)bits;
+      }
+    }
+    base_pos += __popc(hb);
+  }
+  if (lane == 0) L.n = min(base_pos, kMaxT);
+}
+
+// Key-side walk of item (h, loc), one warp: the attending query tiles of
+// its key rows, ascending, placed in the head's walk area by an atomic
+// allocator (placement order does not affect results).
+__device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
+                            int* stage, int lane) {
+  const int item = h * g.per_bh + loc;
+  KeyWalk w;
+  w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, item);
+  uint32_t* walk = p.kplan + (size_t)h * p.kcap;
+  int* kofs = p.kof + 2 * (size_t)item;
+  // Stage the (at most four) CSR lists in shared memory when they fit.
+  int total = 0;
+  for (int x = 0; x < w.nl; ++x) total += w.ln[x];
+  if (!w.global && total <= kStageCap) {
+    int off = 0;
+    for (int x = 0; x < w.nl; ++x) {
+      for (int e = lane; e < w.ln[x]; e += 32) stage[off + e] = w.lp[x][e];
+      w.lp[x] = stage + off;
+      off += w.ln[x];
+    }
+  }
+  __syncwarp();
+  int n = 0, base = 0;
+  if (lane == 0) {
+    KeyWalk c = w;
+    int tile, mask;
+    while (c.next(tile, mask)) ++n;
+    base = atomicAdd(p.kof + 2 * (size_t)p.H * g.per_bh + h, n);
+    if (base + n > p.kcap) {  // cannot happen within the planner's bound
+      set_status(p.status, BB_ERR_BAD_TABLE);
+      n = max(0, p.kcap - base);
+    }
+    int e = 0;
+    while (e < n && w.next(tile, mask)) walk[base + e++] = kentry(tile, mask);
+    kofs[0] = base;
+    kofs[1] = n;
+  }
+}
+
+// Plans, one warp per item: query-side lists (do_q) and key-side walks
+// (do_k, after the CSR exists).
+__global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do_q,
+                                                               int do_k) {
+  __shared__ int cand[kPlanWarps][128];
+  __shared__ int stage[kPlanWarps][kStageCap];
   const Geom g = make_geom(p.L, p.bs);
-  const int id = blockIdx.x * 128 + threadIdx.x;
-  if (id >= p.H * g.per_bh) return;
-  const int h = id / g.per_bh, loc = id % g.per_bh;
-  TileList* qplan = static_cast<TileList*>(p.qplan);
-  if (!build_tile_list(p, g, h, loc, qplan[id])) set_status(p.status, BB_ERR_BAD_TABLE);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nitems = p.H * g.per_bh;
+  const int id = blockIdx.x * kPlanWarps + warp;
+  const int nq = do_q ? nitems : 0;
+  if (id < nq) {
+    plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], lane);
+  } else if (do_k && id - nq < nitems) {
+    const int k = id - nq;
+    plan_k_item(p, g, k / g.per_bh, k % g.per_bh, stage[warp], lane);
+  }
 }
 
 }  // namespace
@@ -224,9 +321,17 @@ int tc_kplan_cap(const Problem& p) {
   return 2 * pair_cap(p.nb, p.r) + g.n_git * g.nt + 64;
 }
 
-cudaError_t launch_plan_q(const Problem& p, cudaStream_t s) {
-  const int n = p.H * (int)tc_items_per_bh(p);
-  plan_q_kernel<<<(n + 127) / 128, 128, 0, s>>>(p);
+cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
+  const int items = p.H * (int)tc_items_per_bh(p);
+  const int n = items * (key_side ? 2 : 1);
+  if (key_side) {
+    // per-head allocation counters live after the [items][2] offsets
+    cudaError_t e = cudaMemsetAsync(p.kof + 2 * (size_t)items, 0,
+                                    sizeof(int) * p.H, s);
+    if (e != cudaSuccess) return e;
+  }
+  plan_kernel<<<(n + kPlanWarps - 1) / kPlanWarps, 32 * kPlanWarps, 0, s>>>(
+      p, 1, key_side ? 1 : 0);
   return cudaGetLastError();
 }
 

@@ -39,7 +39,7 @@ WsLayout ws_layout(const Problem& p, int pass) {
       w.qplan_off = off;
       off = align_up(off + tc_qplan_bytes(p), 256);
       w.kof_off = off;
-      off = align_up(off + (size_t)p.H * (tc_items_per_bh(p) + 1) * sizeof(int), 256);
+      off = align_up(off + ((size_t)p.H * tc_items_per_bh(p) * 2 + p.H) * sizeof(int), 256);
       w.kplan_off = off;
       off = align_up(off + (size_t)p.H * tc_kplan_cap(p) * sizeof(uint32_t), 256);
       w.total = off;
@@ -216,7 +216,7 @@ static int fwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   if (tc_fwd_supported(p)) {
     TensorMaps tm;
     if (!encode_tensor_maps(p, 0, &tm)) return BB_ERR_CUDA;
-    if (launch_plan_q(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (launch_plan(p, false, s) != cudaSuccess) return BB_ERR_CUDA;
     if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
     if (launch_tc_fwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
   } else {
@@ -264,6 +264,8 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
     if (!encode_tensor_maps(p, 1, &tm)) return BB_ERR_CUDA;
     if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
     if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
+    if (launch_plan(p, true, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
     if (launch_tc_bwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
   } else {
     if (launch_bwd_pre(p, s) != cudaSuccess) return BB_ERR_CUDA;
@@ -282,7 +284,7 @@ static const char* const kFwdSimt[] = {"simt_fwd"};
 static const char* const kFwdTc[] = {"plan", "tc_fwd", "fwd_combine"};
 static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
-static const char* const kBwdTc[] = {"csr_build", "tc_dq", "tc_dkdv",
+static const char* const kBwdTc[] = {"csr_build", "plan", "tc_dq", "tc_dkdv",
                                      "bwd_finish"};
 
 static int launch_plan(const bb_attn_desc* desc, int pass,
@@ -296,8 +298,9 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     *names = tc ? kFwdTc : kFwdSimt;
     *n = tc ? 3 : 1;
   } else {
-    *names = tc_bwd_supported(p) ? kBwdTc : kBwdSimt;
-    *n = 4;
+    const bool tc = tc_bwd_supported(p);
+    *names = tc ? kBwdTc : kBwdSimt;
+    *n = tc ? 5 : 4;
   }
   return BB_OK;
 }

@@ -47,7 +47,8 @@ struct Problem {
   size_t part_floats;
   // tensor-core plans (see tc_common.cuh)
   void* qplan;       // [H][items per (b, h)] tile lists, query side
-  int* kof;          // [H][items per (b, h) + 1] offsets of the key-side walks
+  int* kof;          // [H * items][2] (start, length) of the key-side walks,
+                     // then [H] allocation counters
   uint32_t* kplan;   // [H][kcap] key-side walk entries
   int kcap;
 };
@@ -98,7 +99,7 @@ bool tc_bwd_supported(const Problem& p);
 size_t tc_qplan_bytes(const Problem& p);
 int tc_kplan_cap(const Problem& p);
 size_t tc_items_per_bh(const Problem& p);
-cudaError_t launch_plan_q(const Problem& p, cudaStream_t s);
+cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s);
 size_t tc_bwd_extra_bytes(const Problem& p);
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);

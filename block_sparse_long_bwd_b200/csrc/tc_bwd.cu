@@ -400,6 +400,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ volatile int abort_flag;
 
   const Problem& p = ba.qa.p;
+  // bf16 hi/lo split of the global key blocks' P^T and dS^T once they sum
+  // over enough query rows for bf16 products to cost accuracy (>= 16K).
+  const bool split_global = p.L >= 16384;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -446,8 +449,7 @@ __global__ void __launch_bounds__(kThreads, 2)
            ++k, item += gridDim.x) {
         const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-        const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
-        const int e0 = wof[it.loc], e1 = wof[it.loc + 1];
+        const int e0 = p.kof[2 * (size_t)item], e1 = e0 + p.kof[2 * (size_t)item + 1];
         if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
@@ -505,8 +507,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int k = 0, item = blockIdx.x; item < ba.qa.items && ok;
          ++k, item += gridDim.x) {
       const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
-      const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
-      const int nwalk = wof[it.loc + 1] - wof[it.loc];
+      const int nwalk = p.kof[2 * (size_t)item + 1];
       if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       for (int t = 0; t < nwalk;) {
@@ -552,10 +553,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16, sdesc_sw128(qaddr + kk * 2048, 8192),
                    idAcc, (t > 0 || kk > 0) ? 1u : 0u);
-          if (it.global) {
-            // Global key blocks sum over every query row: their P^T and
-            // dS^T also carry a bf16 low part, so the products keep ~16
-            // bits instead of 8.
+          if (it.global && split_global) {
+            // Global key blocks sum over every query row: at long lengths
+            // their P^T and dS^T also carry a bf16 low part, so the products
+            // keep ~16 bits instead of 8.
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_ts(tDV, tS + kk * 8 + (kk >> 1) * 16 + 16,
@@ -591,8 +592,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int k = 0, item = blockIdx.x; item < ba.qa.items; ++k, item += gridDim.x) {
       const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-      const int* wof = p.kof + (size_t)it.h * (ba.qa.geo.per_bh + 1);
-      const int e0 = wof[it.loc], e1 = wof[it.loc + 1];
+      const int e0 = p.kof[2 * (size_t)item], e1 = e0 + p.kof[2 * (size_t)item + 1];
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;
@@ -609,7 +609,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         const int m2 = (mask >> gshift) & 3;  // attending query-column halves
-        const bool split = it.global;          // also write bf16 low parts
+        const bool split = it.global && split_global;  // bf16 low parts too
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
         if (m2 && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
                              p.status)) {

@@ -393,9 +393,10 @@ inline bool tc_shape_ok(const Problem& p) {
   if (p.bs != 32 && p.bs != 64 && p.bs != 128) return false;
   if (p.L % kTile != 0) return false;
   if ((size_t)p.B * p.H * p.L >= (1ull << 31)) return false;
-  // tiles per middle item: 4 groups x (5 + r) blocks, each one tile (32),
-  // or 2 blocks per item x (5 + r) tiles (64), or (5 + r) x 2 tiles (128)
-  const int per = p.bs == 32 ? 4 * (5 + p.r) : 2 * (5 + p.r);
+  // Planner bounds: a middle item's (group, block, tile) candidates fit the
+  // 128-entry sort (4 groups x (5 + r) blocks x tiles per block) and its
+  // distinct tiles fit kMaxT.
+  const int per = p.bs == 64 ? 2 * (5 + p.r) : 4 * (5 + p.r);
   return per <= kMaxT;
 }
 

@@ -382,6 +382,17 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // ======================= dK / dV =======================
 
+// Entries [e0, e1) of this head's walk area that hold the item's query
+// tiles.  Walks are planned per (head, item) - they do not depend on the
+// batch index - so they are looked up by (h, loc), and the range is clamped
+// to the area the plan allocated.
+__device__ __forceinline__ void walk_range(const Problem& p, const Geom& g,
+                                           const ItemMeta& it, int& e0, int& e1) {
+  const size_t k = (size_t)it.h * g.per_bh + it.loc;
+  e0 = max(0, min(p.kof[2 * k], p.kcap));
+  e1 = max(e0, min(e0 + p.kof[2 * k + 1], p.kcap));
+}
+
 struct KvBars {
   uint64_t kp_full, kp_empty;
   uint64_t qt_full[kQStages], qt_empty[kQStages];
@@ -449,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 2)
            ++k, item += gridDim.x) {
         const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-        const int e0 = p.kof[2 * (size_t)item], e1 = e0 + p.kof[2 * (size_t)item + 1];
+        int e0, e1;
+        walk_range(p, ba.qa.geo, it, e0, e1);
         if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
@@ -507,7 +519,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int k = 0, item = blockIdx.x; item < ba.qa.items && ok;
          ++k, item += gridDim.x) {
       const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
-      const int nwalk = p.kof[2 * (size_t)item + 1];
+      int w0, w1;
+      walk_range(p, ba.qa.geo, it, w0, w1);
+      const int nwalk = w1 - w0;
       if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       for (int t = 0; t < nwalk;) {
@@ -592,7 +606,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int k = 0, item = blockIdx.x; item < ba.qa.items; ++k, item += gridDim.x) {
       const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-      const int e0 = p.kof[2 * (size_t)item], e1 = e0 + p.kof[2 * (size_t)item + 1];
+      int e0, e1;
+      walk_range(p, ba.qa.geo, it, e0, e1);
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;

@@ -474,8 +474,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         kp_issued = 1;
         kp_par = k & 1;
         bool ok = true;
+        uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
         for (int e = e0; e < e1; ++e) {
-          const int i = (int)(__ldg(walk + e) & 0xFFFFu);  // query tile
+          const int i = (int)(nxt & 0xFFFFu);  // query tile
+          if (e + 1 < e1) nxt = __ldg(walk + e + 1);
           const int st = g % kQStages;
           if (!mbar_wait(&bars.qt_empty[st], ((g / kQStages) & 1) ^ 1,
                          &abort_flag, p.status)) {
@@ -615,8 +617,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (rvalid && p.key_mask)
         off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
       bool ok = true;
+      uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
       for (int e = e0; e < e1; ++e) {
-        const int mask = (int)(__ldg(walk + e) >> 16);
+        const int mask = (int)(nxt >> 16);
+        if (e + 1 < e1) nxt = __ldg(walk + e + 1);
         const int st = g % kQStages;
         if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
           ok = false;

@@ -399,6 +399,11 @@ struct KvBars {
   uint64_t s_full, p_full, acc_full, acc_empty;
 };
 
+// kSplit: bf16 hi/lo split of the global key blocks' P^T and dS^T, for
+// lengths where they sum over enough query rows (>= 16K) for bf16 products
+// to cost accuracy.  A template flag keeps the low parts out of the shorter
+// lengths' register budget.
+template <bool kSplit>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_dkdv_kernel(const __grid_constant__ BwdArgs ba,
                    const __grid_constant__ CUtensorMap tmQ,
@@ -411,9 +416,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   __shared__ volatile int abort_flag;
 
   const Problem& p = ba.qa.p;
-  // bf16 hi/lo split of the global key blocks' P^T and dS^T once they sum
-  // over enough query rows for bf16 products to cost accuracy (>= 16K).
-  const bool split_global = p.L >= 16384;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -569,7 +571,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16, sdesc_sw128(qaddr + kk * 2048, 8192),
                    idAcc, (t > 0 || kk > 0) ? 1u : 0u);
-          if (it.global && split_global) {
+          if (kSplit && it.global) {
             // Global key blocks sum over every query row: at long lengths
             // their P^T and dS^T also carry a bf16 low part, so the products
             // keep ~16 bits instead of 8.
@@ -628,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         const int m2 = (mask >> gshift) & 3;  // attending query-column halves
-        const bool split = it.global && split_global;  // bf16 low parts too
+        const bool split = kSplit && it.global;  // bf16 low parts too
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
         if (m2 && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
                              p.status)) {
@@ -841,10 +843,11 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   if (e != cudaSuccess) return e;
 
   const size_t smem_kv = 1024 + 4 * kTileBytes + kQStages * kQStageBytes;
-  e = cudaFuncSetAttribute(tc_dkdv_kernel,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_kv);
+  auto* kv_kernel = p.L >= 16384 ? tc_dkdv_kernel<true> : tc_dkdv_kernel<false>;
+  e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_kv);
   if (e != cudaSuccess) return e;
-  tc_dkdv_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_kv, s>>>(
+  kv_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_kv, s>>>(
       ba, tm.q, tm.k, tm.v, tm.dout);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

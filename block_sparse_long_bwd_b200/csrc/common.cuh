@@ -84,6 +84,7 @@ struct EventMarks {
 // for the backward), 64 x 64 boxes, 128-byte swizzle.
 struct TensorMaps {
   CUtensorMap q, k, v, o, dout;
+  CUtensorMap out32;  // forward output, 32-row boxes (one softmax warp's rows)
 };
 // Encodes the maps a pass needs; false if the driver entry point or the
 // encode call fails.

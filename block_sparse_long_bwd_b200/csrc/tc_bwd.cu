@@ -120,14 +120,14 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int q_issued = 0;
       uint32_t q_par = 0;
-      for (int k = 0, item = blockIdx.x; item < a.items;
-           ++k, item += gridDim.x) {
+      ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
+      for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
         const int slot = k & 1;
         if (!mbar_wait(&bars.list_empty[slot], ((k >> 1) & 1) ^ 1, &abort_flag,
                        p.status))
           break;
         // Planned key-tile list: one bulk copy into the slot.
-        const ItemMeta m = item_meta(a.geo, p.H, item);
+        const ItemMeta m = cur.meta(a.geo, p.H);
         const TileList& L = lists[slot];
         mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
         bulk_load(&lists[slot],
@@ -251,12 +251,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;
-    for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
+    ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
       const int slot = k & 1;
       if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
       const TileList& L = lists[slot];
-      const ItemMeta im = item_meta(a.geo, p.H, item);
+      const ItemMeta im = cur.meta(a.geo, p.H);
       const int n = L.n;
       const bool rvalid = (im.gvalid >> quarter) & 1;
       const size_t grow = (size_t)im.bh * p.L + (size_t)(rvalid ? im.t[half] : 0) * kTile + r64;
@@ -458,9 +459,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int kp_issued = 0;
       uint32_t kp_par = 0;
-      for (int k = 0, item = blockIdx.x; item < ba.qa.items;
-           ++k, item += gridDim.x) {
-        const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+      ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
+      for (int k = 0; cur.item < ba.qa.items;
+           ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
+        const ItemMeta it = cur.meta(ba.qa.geo, p.H);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.qa.geo, it, e0, e1);
@@ -520,9 +522,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
     uint32_t g = 0, u = 0;
     bool ok = true;
-    for (int k = 0, item = blockIdx.x; item < ba.qa.items && ok;
-         ++k, item += gridDim.x) {
-      const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+    ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < ba.qa.items && ok;
+         ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
+      const ItemMeta it = cur.meta(ba.qa.geo, p.H);
       int w0, w1;
       walk_range(p, ba.qa.geo, it, w0, w1);
       const int nwalk = w1 - w0;
@@ -607,8 +610,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t g = 0, u = 0;
-    for (int k = 0, item = blockIdx.x; item < ba.qa.items; ++k, item += gridDim.x) {
-      const ItemMeta it = item_meta(ba.qa.geo, p.H, item);
+    ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < ba.qa.items;
+         ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
+      const ItemMeta it = cur.meta(ba.qa.geo, p.H);
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
       int e0, e1;
       walk_range(p, ba.qa.geo, it, e0, e1);

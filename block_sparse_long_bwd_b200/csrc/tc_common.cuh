@@ -37,6 +37,7 @@ constexpr int kPartStride = 68;                       // floats per fwd partial 
 // Geometry of the tiled problem (host and device).
 struct Geom {
   int bs, nb, nt;       // block size, blocks, 64-token tiles
+  int bs_shift;         // log2(bs): bs is 32, 64 or 128 on this path
   int w_first, n_mid;   // middle windows
   int ngt;              // tiles holding global blocks (ascending in gt)
   int gt[4];
@@ -48,6 +49,7 @@ struct Geom {
 __host__ __device__ inline Geom make_geom(int L, int bs) {
   Geom g;
   g.bs = bs;
+  g.bs_shift = bs == 32 ? 5 : bs == 64 ? 6 : 7;
   g.nb = L / bs;
   g.nt = L / kTile;
   // Windows intersecting the middle tokens [bs, L - bs).
@@ -76,7 +78,7 @@ __host__ __device__ inline Geom make_geom(int L, int bs) {
 
 // Block of token row `tok`.
 __host__ __device__ inline int block_of(const Geom& g, int tok) {
-  return tok / g.bs;
+  return tok >> g.bs_shift;
 }
 
 // Tiles covering block j and the column halves of each it spans:
@@ -169,26 +171,66 @@ __host__ __device__ __forceinline__ int expand_groups(int groups, int halves) {
 
 // Metadata of item `item` ((b, h)-major; within one (b, h) the global items'
 // chunks come first, then the middle windows).  Same decoding on both sides.
-__host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int item) {
+// Item at (b, h, loc): no divisions (at most two global items per (b, h)).
+__host__ __device__ __forceinline__ ItemMeta item_meta_at(const Geom& g, int b, int h,
+                                                          int H, int loc) {
   ItemMeta m;
-  m.bh = item / g.per_bh;
-  m.loc = item % g.per_bh;
-  m.b = m.bh / H;
-  m.h = m.bh % H;
+  m.b = b;
+  m.h = h;
+  m.bh = b * H + h;
+  m.loc = loc;
   const int nglob = g.n_git * g.nchunks;
-  if (m.loc < nglob) {
+  if (loc < nglob) {
     m.global = 1;
-    m.gi = m.loc / g.nchunks;
-    m.chunk = m.loc % g.nchunks;
+    m.gi = loc >= g.nchunks ? 1 : 0;
+    m.chunk = loc - m.gi * g.nchunks;
     item_rows(g, true, m.gi, m.t, m.gvalid);
   } else {
     m.global = 0;
     m.gi = 0;
     m.chunk = 0;
-    item_rows(g, false, g.w_first + (m.loc - nglob), m.t, m.gvalid);
+    item_rows(g, false, g.w_first + (loc - nglob), m.t, m.gvalid);
   }
   return m;
 }
+
+__host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int item) {
+  const int bh = item / g.per_bh;
+  return item_meta_at(g, bh / H, bh % H, H, item % g.per_bh);
+}
+
+// A CTA's items start, stride: the (b, h, loc) decomposition is stepped
+// forward instead of divided out at every item.
+struct ItemCursor {
+  int item, b, h, loc;
+  int step_bh, step_loc;
+  __device__ __forceinline__ ItemCursor(const Geom& g, int H, int start, int stride) {
+    item = start;
+    const int bh = start / g.per_bh;
+    loc = start % g.per_bh;
+    b = bh / H;
+    h = bh % H;
+    step_bh = stride / g.per_bh;
+    step_loc = stride % g.per_bh;
+  }
+  __device__ __forceinline__ void next(const Geom& g, int H, int stride) {
+    item += stride;
+    loc += step_loc;
+    int dbh = step_bh;
+    if (loc >= g.per_bh) {
+      loc -= g.per_bh;
+      ++dbh;
+    }
+    h += dbh;
+    while (h >= H) {
+      h -= H;
+      ++b;
+    }
+  }
+  __device__ __forceinline__ ItemMeta meta(const Geom& g, int H) const {
+    return item_meta_at(g, b, h, H, loc);
+  }
+};
 
 // Plans the key tiles of query-side item (h, loc) into L.  Returns false if
 // the random table held an entry outside [-1, nb) (ignored).

@@ -55,7 +55,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV) {
+                  const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmO) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ TileList lists[2];  // bulk-copy destinations (16-byte aligned)
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -109,15 +111,15 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int qissued[2] = {0, 0};
       uint32_t qpar[2] = {0, 0};
-      for (int k = 0, item = blockIdx.x; item < a.items;
-           ++k, item += gridDim.x) {
+      ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
+      for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
         const int slot = k & 1;
         const uint32_t ph = (k >> 1) & 1;
         if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
         // The item's key-tile list was planned before this kernel: one bulk
         // copy into the slot (the producer waits for it like the others).
-        const ItemMeta m = item_meta(a.geo, p.H, item);
+        const ItemMeta m = cur.meta(a.geo, p.H);
         const TileList& L = lists[slot];
         mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
         bulk_load(&lists[slot],
@@ -255,12 +257,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;  // tile counter (same sequence as the MMA warp)
-    for (int k = 0, item = blockIdx.x; item < a.items; ++k, item += gridDim.x) {
+    ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
       if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
       const TileList& L = lists[slot];
-      const ItemMeta im = item_meta(a.geo, p.H, item);
+      const ItemMeta im = cur.meta(a.geo, p.H);
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -397,7 +400,16 @@ __global__ void __launch_bounds__(kThreads, 2)
       float* part = p.part +
                     ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) * 128 +
                      row) * kPartStride;
-#pragma unroll
+      // Middle rows leave through shared memory and one TMA store per warp
+      // (a row per lane would make every store instruction touch 32 lines).
+      // The staging area is this warp's quarter of the item's Q slot: every
+      // S MMA that read it has completed (they precede the last P V), and the
+      // producer refills the slot only after this item's list_empty.
+      uint8_t* stage = Qs + slot * 2 * kTileBytes + quarter * 4096;
+      const bool tma_out = write && !im.global;
+      // Not unrolled: runs once per item, so a small loop body costs less
+      // instruction fetch than four copies.
+#pragma unroll 1
       for (int q16 = 0; q16 < 4; ++q16) {
         uint32_t o[16];
         tmem_ld16(tO + q16 * 16, o);
@@ -407,12 +419,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(o[e]) * inv;
           if (!im.global) {
-            uint4* dst = reinterpret_cast<uint4*>(
-                static_cast<__nv_bfloat16*>(p.out) + grow * kHeadDim + q16 * 16);
-            dst[0] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-            dst[1] = make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
-                                pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
+            // 16-byte chunks 2 q16 and 2 q16 + 1 of this row, 128-byte swizzle
+            // (chunk index XOR row mod 8), as the store's tensor map expects.
+            uint8_t* rowp = stage + lane * 128;
+            const int c0 = 2 * q16;
+            *reinterpret_cast<uint4*>(rowp + ((c0 ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                           pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+            *reinterpret_cast<uint4*>(rowp + (((c0 + 1) ^ (lane & 7)) << 4)) =
+                make_uint4(pack_bf16(v[8], v[9]), pack_bf16(v[10], v[11]),
+                           pack_bf16(v[12], v[13]), pack_bf16(v[14], v[15]));
           } else {
             float4* dst = reinterpret_cast<float4*>(part + q16 * 16);
 #pragma unroll
@@ -422,9 +438,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       tc_fence_before();
+      if (tma_out) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&bars.o_empty);
+        if (tma_out) {
+          tma_store_2d(&tmO, stage, 0,
+                       (int)((size_t)im.bh * p.L + (size_t)im.t[half] * kTile +
+                             (quarter & 1) * 32));
+          bulk_commit_group();
+          bulk_wait_read_all();  // the slot may be refilled after list_empty
+        }
         mbar_arrive(&bars.list_empty[slot]);
       }
       if (write) {
@@ -438,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
+  if (warp >= 2 && lane == 0) bulk_wait_all();  // output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -503,7 +528,7 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = min(a.items, 2 * sms);
-  tc_fwd_kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v);
+  tc_fwd_kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v, tm.out32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = marks->mark(s);

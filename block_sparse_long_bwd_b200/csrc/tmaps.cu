@@ -28,13 +28,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows][64] bf16 row view, box 64 x 64, 128-byte swizzle.
-bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows) {
+// [rows][64] bf16 row view, box 64 x box_rows, 128-byte swizzle.
+bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows,
+                 cuuint32_t box_rows = 64) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)kHeadDim * 2};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -48,6 +49,7 @@ bool encode_tensor_maps(const Problem& p, int pass, TensorMaps* tm) {
   const uint64_t rows = (uint64_t)p.B * p.H * p.L;
   bool ok = encode_rows(&tm->q, p.q, rows) && encode_rows(&tm->k, p.k, rows) &&
             encode_rows(&tm->v, p.v, rows);
+  if (ok && pass == 0) ok = encode_rows(&tm->out32, p.out, rows, 32);
   if (ok && pass == 1)
     ok = encode_rows(&tm->o, p.o, rows) && encode_rows(&tm->dout, p.dout, rows);
   return ok;

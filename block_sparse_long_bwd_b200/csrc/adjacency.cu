@@ -47,8 +47,13 @@ __device__ __forceinline__ int random_target(const int32_t* row, int a, int i,
 
 constexpr int kCsrThreads = 1024;
 
-// One CTA per head.  Shared memory: count[nb], cursor[nb], tsum[1024].
-__global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
+// Total list length: the inclusive scan's last element.
+__device__ __forceinline__ int total_sh(const int* tsum) { return tsum[kCsrThreads - 1]; }
+
+// One CTA per head.  Shared memory: count[nb], cursor[nb], tsum[1024] and,
+// when it fits (in_smem), the head's whole list, built there and copied out
+// once; otherwise the list is built in place in global memory.
+__global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p, int in_smem) {
   extern __shared__ int smi[];
   const int nb = p.nb, r = p.r, h = blockIdx.x, tid = threadIdx.x;
   int* cnt = smi;
@@ -56,7 +61,8 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
   int* tsum = cur + nb;
   const int32_t* table = p.rand_idx + (size_t)h * nb * r;
   int* offs = p.csr_offs + (size_t)h * (nb + 1);
-  int* list = p.csr_list + (size_t)h * p.csr_cap;
+  int* glist = p.csr_list + (size_t)h * p.csr_cap;
+  int* list = in_smem ? tsum + kCsrThreads : glist;
 
   for (int j = tid; j < nb; j += kCsrThreads) {
     int c;
@@ -91,9 +97,11 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
   }
   int run = tsum[tid] - local;  // exclusive prefix of this chunk
   for (int j = c0; j < c1; ++j) {
+    const int c = cnt[j];
     cur[j] = run;
     offs[j] = run;
-    run += cnt[j];
+    cnt[j] = run;  // from here on: start offset of list j
+    run += c;
   }
   if (tid == kCsrThreads - 1) offs[nb] = tsum[kCsrThreads - 1];
   __syncthreads();
@@ -124,8 +132,9 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
   // Sort each non-global list (short: 2 + 3 + random in-degree).
   for (int j = tid; j < nb; j += kCsrThreads) {
     if (j == 0 || j == nb - 1) continue;
-    int* L = list + offs[j];
-    const int n = offs[j + 1] - offs[j];
+    const int o0 = in_smem ? cnt[j] : offs[j];
+    int* L = list + o0;
+    const int n = (in_smem ? (j + 1 < nb ? cnt[j + 1] : total_sh(tsum)) : offs[j + 1]) - o0;
     for (int a = 1; a < n; ++a) {
       int x = L[a], c = a - 1;
       while (c >= 0 && L[c] > x) {
@@ -134,6 +143,11 @@ __global__ void __launch_bounds__(kCsrThreads) csr_build_kernel(Problem p) {
       }
       L[c + 1] = x;
     }
+  }
+  if (in_smem) {
+    __syncthreads();
+    const int total = total_sh(tsum);
+    for (int x = tid; x < total; x += kCsrThreads) glist[x] = list[x];
   }
 }
 
@@ -238,8 +252,12 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
 }
 
 // Key-side walk of item (h, loc), one warp: the attending query tiles of
-// its key rows, ascending, placed in the head's walk area by an atomic
-// allocator (placement order does not affect results).
+// its key rows, ascending.  Each item owns a fixed region of the head's walk
+// area, so no allocator is needed: a middle window's walk has at most T x
+// (the CSR list lengths of its key blocks) entries (T = 2 query tiles per
+// query block at block size 128, else 1), so its region starts at T times
+// the CSR offset of its first key block; global chunks (kChunk query tiles
+// each) follow T x (all CSR entries).
 __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
                             int* stage, int lane) {
   const int item = h * g.per_bh + loc;
@@ -247,6 +265,19 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
   w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, item);
   uint32_t* walk = p.kplan + (size_t)h * p.kcap;
   int* kofs = p.kof + 2 * (size_t)item;
+  const int* offs = p.csr_offs + (size_t)h * (g.nb + 1);
+  const int T = g.bs == 128 ? 2 : 1;
+  int base, cap;
+  if (w.global) {
+    base = T * offs[g.nb] + (w.gi * g.nchunks + w.chunk) * kChunk;
+    cap = kChunk;
+  } else {
+    const int row0 = w.t[0] * kTile;  // window rows [row0, row0 + 128)
+    const int jf = block_of(g, row0);
+    const int jl = min(g.nb - 1, block_of(g, min(row0 + 127, g.nb * g.bs - 1)));
+    base = T * offs[jf];
+    cap = T * (offs[jl + 1] - offs[jf]);
+  }
   // Stage the (at most four) CSR lists in shared memory when they fit.
   int total = 0;
   for (int x = 0; x < w.nl; ++x) total += w.ln[x];
@@ -259,18 +290,14 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
     }
   }
   __syncwarp();
-  int n = 0, base = 0;
   if (lane == 0) {
-    KeyWalk c = w;
-    int tile, mask;
-    while (c.next(tile, mask)) ++n;
-    base = atomicAdd(p.kof + 2 * (size_t)p.H * g.per_bh + h, n);
-    if (base + n > p.kcap) {  // cannot happen within the planner's bound
+    int n = 0, tile, mask;
+    if (base < 0 || base + cap > p.kcap) {  // cannot happen within the bound
       set_status(p.status, BB_ERR_BAD_TABLE);
-      n = max(0, p.kcap - base);
+      cap = 0;
+      base = 0;
     }
-    int e = 0;
-    while (e < n && w.next(tile, mask)) walk[base + e++] = kentry(tile, mask);
+    while (n < cap && w.next(tile, mask)) walk[base + n++] = kentry(tile, mask);
     kofs[0] = base;
     kofs[1] = n;
   }
@@ -324,23 +351,20 @@ int tc_kplan_cap(const Problem& p) {
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
   const int items = p.H * (int)tc_items_per_bh(p);
   const int n = items * (key_side ? 2 : 1);
-  if (key_side) {
-    // per-head allocation counters live after the [items][2] offsets
-    cudaError_t e = cudaMemsetAsync(p.kof + 2 * (size_t)items, 0,
-                                    sizeof(int) * p.H, s);
-    if (e != cudaSuccess) return e;
-  }
   plan_kernel<<<(n + kPlanWarps - 1) / kPlanWarps, 32 * kPlanWarps, 0, s>>>(
       p, 1, key_side ? 1 : 0);
   return cudaGetLastError();
 }
 
 cudaError_t launch_csr_build(const Problem& p, cudaStream_t s) {
-  const size_t smem = (size_t)(2 * p.nb + kCsrThreads) * sizeof(int);
+  const size_t base = (size_t)(2 * p.nb + kCsrThreads) * sizeof(int);
+  const size_t with_list = base + (size_t)p.csr_cap * sizeof(int);
+  const int in_smem = with_list <= 200u * 1024u ? 1 : 0;
+  const size_t smem = in_smem ? with_list : base;
   cudaError_t e = cudaFuncSetAttribute(
       csr_build_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  csr_build_kernel<<<p.H, kCsrThreads, smem, s>>>(p);
+  csr_build_kernel<<<p.H, kCsrThreads, smem, s>>>(p, in_smem);
   return cudaGetLastError();
 }
 

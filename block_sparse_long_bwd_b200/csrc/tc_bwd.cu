@@ -301,6 +301,21 @@ __global__ void __launch_bounds__(kThreads, 2)
             tmem_ld32(tS + hc * 32 + lane_off, s);
             tmem_ld32(tDP + hc * 32 + lane_off, dp);
             tmem_ld_wait();
+            if (kb == ~0ull) {
+              // No masked key in the tile: paired (f32x2) arithmetic.
+              const float2 c2 = make_float2(c, c), nl22 = make_float2(nl2, nl2);
+              const float2 D2 = make_float2(Dr, Dr);
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float2 a = fma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])),
+                                      c2, nl22);
+                const float2 pp = make_float2(ex2(a.x), ex2(a.y));
+                const float2 d = mul2(
+                    pp, sub2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), D2));
+                dS[(hc * 32 + e) >> 1] = pack_bf16(d.x, d.y);
+              }
+              continue;
+            }
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
               const int col = hc * 32 + e;
@@ -664,10 +679,21 @@ __global__ void __launch_bounds__(kThreads, 2)
               const float nls[4] = {nl.x, nl.y, nl.z, nl.w};
               const float dds[4] = {dd.x, dd.y, dd.z, dd.w};
               float pv[4], dv[4];
+              const float2 c2 = make_float2(c, c), off2 = make_float2(off, off);
 #pragma unroll
-              for (int x = 0; x < 4; ++x) {
-                pv[x] = ex2(fmaf(__uint_as_float(sv[e + x]), c, nls[x] + off));
-                dv[x] = pv[x] * (__uint_as_float(dp[e + x]) - dds[x]);
+              for (int x = 0; x < 4; x += 2) {
+                // Paired (f32x2) arithmetic, each element rounded as before.
+                const float2 a = fma2(
+                    make_float2(__uint_as_float(sv[e + x]), __uint_as_float(sv[e + x + 1])), c2,
+                    add2(make_float2(nls[x], nls[x + 1]), off2));
+                pv[x] = ex2(a.x);
+                pv[x + 1] = ex2(a.y);
+                const float2 d = mul2(
+                    make_float2(pv[x], pv[x + 1]),
+                    sub2(make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
+                         make_float2(dds[x], dds[x + 1])));
+                dv[x] = d.x;
+                dv[x + 1] = d.y;
               }
 #pragma unroll
               for (int x = 0; x < 2; ++x) {

@@ -45,10 +45,18 @@ struct Bars {
   uint64_t pv_done[2], o_empty;
 };
 
-__device__ __forceinline__ float max8(const float* z) {
-  const float a = fmaxf(z[0], z[1]), b = fmaxf(z[2], z[3]);
-  const float c = fmaxf(z[4], z[5]), d = fmaxf(z[6], z[7]);
-  return fmaxf(fmaxf(a, b), fmaxf(c, d));
+// Maximum of 64 values with three-input max: 32 instructions, depth 4.
+__device__ __forceinline__ float max64(const float* z) {
+  float m[22];
+#pragma unroll
+  for (int i = 0; i < 21; ++i) m[i] = fmax3(z[3 * i], z[3 * i + 1], z[3 * i + 2]);
+  m[21] = z[63];
+  float n[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) n[i] = fmax3(m[3 * i], m[3 * i + 1], m[3 * i + 2]);
+  n[7] = m[21];
+  const float a = fmax3(n[0], n[1], n[2]), b = fmax3(n[3], n[4], n[5]);
+  return fmax3(a, b, fmaxf(n[6], n[7]));
 }
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -306,10 +314,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint64_t hb = half_bits(m2);
           float mx;
           if (kb == ~0ull && hb == ~0ull && c > 0.f) {
-            float mx8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
-            mx = max8(mx8) * c;
+            mx = max64(z) * c;
           } else {
             // Columns outside the attended blocks are absent (-inf, p = 0);
             // masked keys inside them get the finite offset.
@@ -318,10 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               z[e] = ((hb >> e) & 1ull)
                          ? fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl)
                          : -INFINITY;
-            float mx8[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) mx8[e] = max8(z + 8 * e);
-            mx = max8(mx8);
+            mx = max64(z);
           }
           const bool scaled = !(kb == ~0ull && hb == ~0ull && c > 0.f);
           // Lazy running max: move it only when the row max exceeds it by
@@ -355,25 +357,27 @@ __global__ void __launch_bounds__(kThreads, 2)
             }
           }
           if (first) m = mx;
-          float sum8[8];
+          // Paired (f32x2) arithmetic: exponent arguments and row sums.
+          float2 sum2[4];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+          for (int e = 0; e < 4; ++e) sum2[e] = make_float2(0.f, 0.f);
           const float cc = scaled ? 1.f : c;
-          const float nm = -m;
+          const float2 cc2 = make_float2(cc, cc), nm2 = make_float2(-m, -m);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t Ph[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
-              const float p0 = ex2(fmaf(z[32 * hh + e], cc, nm));
-              const float p1 = ex2(fmaf(z[32 * hh + e + 1], cc, nm));
-              sum8[(e >> 1) & 7] += p0 + p1;
-              Ph[e >> 1] = pack_bf16(p0, p1);
+              const float2 a = fma2(make_float2(z[32 * hh + e], z[32 * hh + e + 1]), cc2, nm2);
+              const float2 pp = make_float2(ex2(a.x), ex2(a.y));
+              sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pp);
+              Ph[e >> 1] = pack_bf16(pp.x, pp.y);
             }
             tmem_st16(tP + 16 * hh, Ph);
           }
-          l += ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
-               ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+          const float2 s01 = add2(sum2[0], sum2[1]), s23 = add2(sum2[2], sum2[3]);
+          const float2 s4 = add2(s01, s23);
+          l += s4.x + s4.y;
         } else {
           uint32_t Z[16];
 #pragma unroll

@@ -53,11 +53,46 @@ __device__ __forceinline__ void ld_bf16x8_as_f(const __nv_bfloat16* p,
 
 // ======================= dQ =======================
 
+// P = 2^(S c + NL) of 32 key columns (col0: 0 or 32 within the tile) of
+// one row, in place over S; masked keys are offset by mvl.
+__device__ __forceinline__ void dq_p_half(uint32_t (&s)[32], uint64_t kb, int col0, float c,
+                                          float nl2, float mvl) {
+  if (((kb >> col0) & 0xFFFFFFFFull) == 0xFFFFFFFFull) {
+    // No masked key in these columns: paired (f32x2) arithmetic.
+    const float2 c2 = make_float2(c, c), nl22 = make_float2(nl2, nl2);
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const float2 a =
+          fma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, nl22);
+      s[e] = __float_as_uint(ex2(a.x));
+      s[e + 1] = __float_as_uint(ex2(a.y));
+    }
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float off = ((kb >> (col0 + e)) & 1ull) ? 0.f : mvl;
+    s[e] = __float_as_uint(ex2(fmaf(__uint_as_float(s[e]), c, nl2 + off)));
+  }
+}
+
+// dS = P (dP - D) of 32 key columns of one row, as 16 bf16 pairs.
+__device__ __forceinline__ void dq_ds_half(const uint32_t (&pv)[32], const uint32_t (&dp)[32],
+                                           float Dr, uint32_t* out) {
+  const float2 D2 = make_float2(Dr, Dr);
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float2 d = mul2(make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])),
+                          sub2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), D2));
+    out[e >> 1] = pack_bf16(d.x, d.y);
+  }
+}
+
 struct DqBars {
   uint64_t list_full[2], list_empty[2];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kKvStages], kv_empty[kKvStages];
-  uint64_t s_full, p_full, dq_full, dq_empty;
+  uint64_t s_full, s_free, dp_free, p_full, dq_done, dq_full, dq_empty;
 };
 
 __global__ void __launch_bounds__(kThreads, 2)
@@ -94,7 +129,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.kv_empty[s], 1);
     }
     mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_free, 4);
+    mbar_init(&bars.dp_free, 4);
     mbar_init(&bars.p_full, 4);
+    mbar_init(&bars.dq_done, 1);
     mbar_init(&bars.dq_full, 1);
     mbar_init(&bars.dq_empty, 4);
     fence_mbar_init();
@@ -113,7 +151,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tDQ = tmem, tS = tmem + 64, tDP = tmem + 128;
+  // dQ | S | dP | dS (bf16 pairs): dS has its own columns, so S and dP of
+  // the next tile can be computed while this tile's dS is still formed.
+  const uint32_t tDQ = tmem, tS = tmem + 64, tDP = tmem + 128, tDS = tmem + 192;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -194,14 +234,33 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int n = lists[slot].n;
       if (!mbar_wait(&bars.q_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
-      for (int t = 0; t < n; ++t, ++g, ++u) {
-        const int st = g % kKvStages;
-        // S and dP of this tile overwrite the previous tile's buffers (dS
-        // lives over S).  The previous dQ MMA, which reads that dS, was
-        // issued earlier by this thread, and MMAs from one thread execute in
-        // order, so there is no need to wait for it to complete.
-        if (!mbar_wait(&bars.kv_full[st], (g / kKvStages) & 1, &abort_flag,
-                       p.status)) {
+      // dQ += dS K of item tile t (global tile uu, K/V stage st).
+      auto issue_dq = [&](int t, uint32_t uu, int st) -> bool {
+        if (!mbar_wait(&bars.p_full, uu & 1, &abort_flag, p.status) ||
+            (t == 0 && !mbar_wait(&bars.dq_empty, (k & 1) ^ 1, &abort_flag, p.status)))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t kaddr = smem_u32(KVs + st * 2 * kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(tDQ, tDS + kk * 8, sdesc_sw128(kaddr + kk * 2048, 8192), idDQ,
+                   (t > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bars.dq_done);
+          mma_commit(&bars.kv_empty[st]);
+          if (t == n - 1) mma_commit(&bars.dq_full);
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int t = 0; t < n; ++t) {
+        const uint32_t uu = u + t;
+        const int st = (g + t) % kKvStages;
+        // S and dP of this tile overwrite the previous tile's once the
+        // softmax has read them (s_free, dp_free); dS has its own columns.
+        if (!mbar_wait(&bars.kv_full[st], ((g + t) / kKvStages) & 1, &abort_flag,
+                       p.status) ||
+            (uu > 0 && !mbar_wait(&bars.s_free, (uu - 1) & 1, &abort_flag, p.status))) {
           ok = false;
           break;
         }
@@ -213,16 +272,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tS, sdesc_sw128(qaddr + kk * 32, 16),
                    sdesc_sw128(kaddr + kk * 32, 16), idS, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tDP, sdesc_sw128(gaddr + kk * 32, 16),
-                   sdesc_sw128(vaddr + kk * 32, 16), idS, kk > 0);
-          mma_commit(&bars.s_full);
         }
         __syncwarp();
-        if (!mbar_wait(&bars.p_full, u & 1, &abort_flag, p.status) ||
-            (t == 0 &&
-             !mbar_wait(&bars.dq_empty, (k & 1) ^ 1, &abort_flag, p.status))) {
+        if (uu > 0 && !mbar_wait(&bars.dp_free, (uu - 1) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -230,16 +282,32 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (lane == 0) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tDQ, tS + kk * 8, sdesc_sw128(kaddr + kk * 2048, 8192), idDQ,
-                   (t > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&bars.kv_empty[st]);
-          if (t == n - 1) {
-            mma_commit(&bars.dq_full);
-            mma_commit(&bars.q_empty);
-          }
+            mma_ss(tDP, sdesc_sw128(gaddr + kk * 32, 16),
+                   sdesc_sw128(vaddr + kk * 32, 16), idS, kk > 0);
+          mma_commit(&bars.s_full);
+          if (t == n - 1) mma_commit(&bars.q_empty);  // Q, dO read only here
+        }
+        __syncwarp();
+        // The previous tile's dQ goes to the tensor pipe after this tile's
+        // S and dP, while the softmax works on the previous tile's dS.
+        if (t > 0 && !issue_dq(t - 1, uu - 1, (g + t - 1) % kKvStages)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok) break;
+      if (n > 0) {
+        if (!issue_dq(n - 1, u + n - 1, (g + n - 1) % kKvStages)) break;
+      } else {
+        if (!mbar_wait(&bars.dq_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        if (lane == 0) {
+          mma_commit(&bars.dq_full);
+          mma_commit(&bars.q_empty);
         }
         __syncwarp();
       }
+      g += n;
+      u += n;
       if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
     }
   } else {
@@ -287,59 +355,56 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tc_fence_after();
         const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
+        // S of the attended halves into registers: once every warp has it
+        // (s_free) the MMA warp computes the next tile's S; P is formed in
+        // place.  dP follows half by half; after the second half (dp_free)
+        // the next tile's dP may be computed.
+        uint32_t s0[32], s1[32], dp[32];
+        if (m2 & 1) tmem_ld32(tS + lane_off, s0);
+        if (m2 & 2) tmem_ld32(tS + 32 + lane_off, s1);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free);
+        const uint64_t kb = (m2 && p.key_mask) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
+        if (m2 & 1) dq_p_half(s0, kb, 0, c, nl2, mvl);
+        if (m2 & 2) dq_p_half(s1, kb, 32, c, nl2, mvl);
         uint32_t dS[32];
-        if (m2) {
-          const uint64_t kb = p.key_mask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
-#pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
-            if (!((m2 >> hc) & 1)) {  // keys outside the attended blocks
-#pragma unroll
-              for (int e = 0; e < 16; ++e) dS[hc * 16 + e] = 0u;
-              continue;
-            }
-            uint32_t s[32], dp[32];
-            tmem_ld32(tS + hc * 32 + lane_off, s);
-            tmem_ld32(tDP + hc * 32 + lane_off, dp);
-            tmem_ld_wait();
-            if (kb == ~0ull) {
-              // No masked key in the tile: paired (f32x2) arithmetic.
-              const float2 c2 = make_float2(c, c), nl22 = make_float2(nl2, nl2);
-              const float2 D2 = make_float2(Dr, Dr);
-#pragma unroll
-              for (int e = 0; e < 32; e += 2) {
-                const float2 a = fma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])),
-                                      c2, nl22);
-                const float2 pp = make_float2(ex2(a.x), ex2(a.y));
-                const float2 d = mul2(
-                    pp, sub2(make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), D2));
-                dS[(hc * 32 + e) >> 1] = pack_bf16(d.x, d.y);
-              }
-              continue;
-            }
-#pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              const int col = hc * 32 + e;
-              const float off0 = ((kb >> col) & 1ull) ? 0.f : mvl;
-              const float off1 = ((kb >> (col + 1)) & 1ull) ? 0.f : mvl;
-              const float p0 = ex2(fmaf(__uint_as_float(s[e]), c, nl2 + off0));
-              const float p1 = ex2(fmaf(__uint_as_float(s[e + 1]), c, nl2 + off1));
-              const float d0 = p0 * (__uint_as_float(dp[e]) - Dr);
-              const float d1 = p1 * (__uint_as_float(dp[e + 1]) - Dr);
-              dS[(col >> 1)] = pack_bf16(d0, d1);
-            }
-          }
+        if (m2 & 1) {
+          tmem_ld32(tDP + lane_off, dp);
+          tmem_ld_wait();
+          dq_ds_half(s0, dp, Dr, dS);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dS[e] = 0u;
+          for (int e = 0; e < 16; ++e) dS[e] = 0u;
         }
+        if (m2 & 2) {
+          tmem_ld32(tDP + 32 + lane_off, dp);
+          tmem_ld_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.dp_free);
+        if (m2 & 2) {
+          dq_ds_half(s1, dp, Dr, dS + 16);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dS[16 + e] = 0u;
+        }
+        // The dS columns are free once the previous tile's dQ MMA completed.
+        if (u > 0 && !mbar_wait(&bars.dq_done, (u - 1) & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         uint32_t d0[16], d1[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           d0[e] = dS[e];
           d1[e] = dS[16 + e];
         }
-        tmem_st16(tS + lane_off, d0);
-        tmem_st16(tS + 16 + lane_off, d1);
+        tmem_st16(tDS + lane_off, d0);
+        tmem_st16(tDS + 16 + lane_off, d1);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

@@ -179,7 +179,7 @@ __device__ __forceinline__ void warp_sort128(int* v, int lane) {
 // Query-side plan of item (h, loc), one warp: every (group, attended block,
 // tile) candidate as (tile << 8 | mask bits), sorted, equal tiles merged.
 __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
-                            int* cand, int lane) {
+                            int* cand, int* merged, int lane) {
   const ItemMeta m = item_meta(g, p.H, h * g.per_bh + loc);
   TileList& L = static_cast<TileList*>(p.qplan)[(size_t)h * g.per_bh + loc];
   if (m.global) {
@@ -228,6 +228,9 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
   if (bad) set_status(p.status, BB_ERR_BAD_TABLE);
   __syncwarp();
   warp_sort128(cand, lane);
+  // Merge equal tiles into the sorted list (mt, mm) in shared memory.
+  int* mt = merged;
+  int* mm = merged + kMaxT;
   int base_pos = 0;
   for (int r = 0; r < 4; ++r) {
     const int e = lane + 32 * r;
@@ -242,13 +245,57 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
     if (head) {
       const int pos = base_pos + __popc(hb & ((1u << lane) - 1));
       if (pos < kMaxT) {
-        L.tile[pos] = (int16_t)(v >> 8);
-        L.mask[pos] = (uint8_t)bits;
+        mt[pos] = v >> 8;
+        mm[pos] = bits;
       }
     }
     base_pos += __popc(hb);
   }
-  if (lane == 0) L.n = min(base_pos, kMaxT);
+  const int n = min(base_pos, kMaxT);
+  __syncwarp();
+  // Visiting order: tiles both 64-row halves of the item attend first, then
+  // tiles of the upper half (groups 0, 1) and of the lower half (groups 2,
+  // 3) alternately, so the half with nothing to do on a tile starts on the
+  // next one (its own) while the other works; results do not depend on the
+  // order.  Each class keeps ascending tile order.
+  int cls[2], rk[2];
+  unsigned cnt_b = 0, cnt_u = 0, cnt_l = 0;
+  for (int r = 0; r < 2; ++r) {
+    const int e = lane + 32 * r;
+    int c = -1;
+    if (e < n) {
+      const bool up = (mm[e] & 0x0F) != 0, lo = (mm[e] & 0xF0) != 0;
+      c = (up && lo) ? 0 : up ? 1 : 2;
+    }
+    const unsigned bb = __ballot_sync(0xFFFFFFFFu, c == 0);
+    const unsigned bu = __ballot_sync(0xFFFFFFFFu, c == 1);
+    const unsigned bl = __ballot_sync(0xFFFFFFFFu, c == 2);
+    const unsigned below = (1u << lane) - 1;
+    cls[r] = c;
+    rk[r] = c == 0 ? cnt_b + __popc(bb & below)
+          : c == 1 ? cnt_u + __popc(bu & below)
+                   : cnt_l + __popc(bl & below);
+    cnt_b += __popc(bb);
+    cnt_u += __popc(bu);
+    cnt_l += __popc(bl);
+  }
+  const int nbo = (int)cnt_b, nu = (int)cnt_u, nl = (int)cnt_l;
+  const int np = min(nu, nl);  // alternating pairs
+  for (int r = 0; r < 2; ++r) {
+    const int e = lane + 32 * r;
+    if (e >= n) continue;
+    int pos;
+    if (cls[r] == 0) {
+      pos = rk[r];
+    } else if (cls[r] == 1) {
+      pos = rk[r] < np ? nbo + 2 * rk[r] : nbo + 2 * np + (rk[r] - np);
+    } else {
+      pos = rk[r] < np ? nbo + 2 * rk[r] + 1 : nbo + 2 * np + (nu - np) + (rk[r] - np);
+    }
+    L.tile[pos] = (int16_t)mt[e];
+    L.mask[pos] = (uint8_t)mm[e];
+  }
+  if (lane == 0) L.n = n;
 }
 
 // Key-side walk of item (h, loc), one warp: the attending query tiles of
@@ -315,7 +362,7 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
   const int id = blockIdx.x * kPlanWarps + warp;
   const int nq = do_q ? nitems : 0;
   if (id < nq) {
-    plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], lane);
+    plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], stage[warp], lane);
   } else if (do_k && id - nq < nitems) {
     const int k = id - nq;
     plan_k_item(p, g, k / g.per_bh, k % g.per_bh, stage[warp], lane);

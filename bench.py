@@ -349,11 +349,14 @@ def run_ours(args, world, rank, local):
     fwd_flops = 4 * pairs * bs * bs * cfg["d"]
     bwd_flops = 10 * pairs * bs * bs * cfg["d"] if backward else 0
     avg = {n: sum(v_) / len(v_) for n, v_ in per_kernel.items()}
+    # Device time per step of each launch name: a name launched more than
+    # once per step (the dK/dV pass at long lengths) is rated over the sum.
+    step_t = {n: sum(v_) / K for n, v_ in per_kernel.items()}
     share = {n: sum(per_kernel[n]) / sum(step_ms) for n in names}
     dom = max(names, key=lambda n: sum(per_kernel[n]))
     peaks, peak_src = load_peaks()
     fl, by = alg.get(kernel_kind(dom), (0, 0))
-    dur_s = avg[dom] / 1e3
+    dur_s = step_t[dom] / 1e3
     bound = kernel_bound(dom)
     if bound == "tensor":
         unit, achieved = "TFLOP/s", fl / dur_s / 1e12
@@ -378,10 +381,10 @@ def run_ours(args, world, rank, local):
                 "kernel": dom, "peak_source": f"{peak_src}: {how}"}
     kernels = {n: {"avg_ms": round(avg[n], 5), "share": round(share[n], 4),
                    "launches": len(per_kernel[n]),
-                   "tflops": (round(alg[kernel_kind(n)][0] / (avg[n] / 1e3)
+                   "tflops": (round(alg[kernel_kind(n)][0] / (step_t[n] / 1e3)
                                     / 1e12, 2)
                               if alg.get(kernel_kind(n), (0, 0))[0] else None),
-                   "gbs": (round(alg[kernel_kind(n)][1] / (avg[n] / 1e3)
+                   "gbs": (round(alg[kernel_kind(n)][1] / (step_t[n] / 1e3)
                                  / 1e9, 1)
                            if alg.get(kernel_kind(n), (0, 0))[1] else None)}
                for n in names}
@@ -618,15 +621,16 @@ def run_sweep(args):
                 # FLOPs by the FlashAttention convention: 4 (fwd) + 10 (bwd)
                 # bs^2 d per attended pair.
                 counted = (4 + 10) * pairs * bs * bs * cfg["d"]
-                names = [bb.bb_attn_launch_name(att.desc, 0, 0)]
+                names = [bb.bb_attn_launch_name(att.desc, 0, i)
+                         for i in range(bb.bb_attn_launch_count(att.desc, 0))]
                 row = {"L": L, "block_size": bs, "r": r, "B": B,
                        "ms": round(ms, 4),
                        "tokens_per_s": round(B * L / (ms / 1e3), 1),
                        "attended_tflops": round(counted / (ms / 1e3) / 1e12, 2),
                        "frac_of_peak": round(counted / (ms / 1e3) / 1e12
                                              / peaks["bf16_tflops"], 4),
-                       "path": "tensor" if names[0].startswith("tc_") else
-                               "cuda-core"}
+                       "path": "tensor" if any(n.startswith("tc_") for n in names)
+                               else "cuda-core"}
                 rows.append(row)
                 print(json.dumps(row), flush=True)
                 del q, k, v, g, out, lse, dq, dk, dv, att

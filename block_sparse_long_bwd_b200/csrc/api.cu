@@ -286,6 +286,10 @@ static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
 static const char* const kBwdTc[] = {"csr_build", "plan", "tc_dq", "tc_dkdv",
                                      "bwd_finish"};
+// At long lengths dK/dV of the global key blocks (hi/lo split) and of the
+// middle windows are separate launches (tc_dkdv_launches).
+static const char* const kBwdTcSplit[] = {"csr_build", "plan", "tc_dq", "tc_dkdv",
+                                          "tc_dkdv", "bwd_finish"};
 
 static int launch_plan(const bb_attn_desc* desc, int pass,
                        const char* const** names, int* n) {
@@ -299,8 +303,9 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     *n = tc ? 3 : 1;
   } else {
     const bool tc = tc_bwd_supported(p);
-    *names = tc ? kBwdTc : kBwdSimt;
-    *n = tc ? 5 : 4;
+    const bool two = tc && tc_dkdv_launches(p) == 2;
+    *names = !tc ? kBwdSimt : two ? kBwdTcSplit : kBwdTc;
+    *n = !tc ? 4 : two ? 6 : 5;
   }
   return BB_OK;
 }

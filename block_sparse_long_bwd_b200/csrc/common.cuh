@@ -102,6 +102,9 @@ int tc_kplan_cap(const Problem& p);
 size_t tc_items_per_bh(const Problem& p);
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s);
 size_t tc_bwd_extra_bytes(const Problem& p);
+// Number of dK/dV launches of the tensor-core backward (1, or 2 at lengths
+// where the global key blocks run with the hi/lo split on their own).
+int tc_dkdv_launches(const Problem& p);
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);
 

@@ -34,6 +34,10 @@ constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // Q, dO, NL, D
 
 struct BwdArgs {
   PairArgs qa;       // items: query side (dq) and, mirrored, key side (dkdv)
+  // Key-side items this dK/dV launch takes: per (b, h) the locs
+  // [kloc0, kloc0 + kgeo.per_bh) (kgeo is qa.geo with per_bh narrowed).
+  Geom kgeo;
+  int kitems, kloc0;
   float* D;          // [B*H*L]
   float* NL;         // [B*H*L]: -lse * log2(e)
   float* dqpart;     // [B*H][n_git][nchunks][128][64]
@@ -539,10 +543,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int kp_issued = 0;
       uint32_t kp_par = 0;
-      ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
-      for (int k = 0; cur.item < ba.qa.items;
-           ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
-        const ItemMeta it = cur.meta(ba.qa.geo, p.H);
+      ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
+      for (int k = 0; cur.item < ba.kitems;
+           ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
+        const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.qa.geo, it, e0, e1);
@@ -602,10 +606,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
     uint32_t g = 0, u = 0;
     bool ok = true;
-    ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < ba.qa.items && ok;
-         ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
-      const ItemMeta it = cur.meta(ba.qa.geo, p.H);
+    ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < ba.kitems && ok;
+         ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
+      const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
       int w0, w1;
       walk_range(p, ba.qa.geo, it, w0, w1);
       const int nwalk = w1 - w0;
@@ -690,10 +694,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t g = 0, u = 0;
-    ItemCursor cur(ba.qa.geo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < ba.qa.items;
-         ++k, cur.next(ba.qa.geo, p.H, gridDim.x)) {
-      const ItemMeta it = cur.meta(ba.qa.geo, p.H);
+    ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
+    for (int k = 0; cur.item < ba.kitems;
+         ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
+      const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
       int e0, e1;
       walk_range(p, ba.qa.geo, it, e0, e1);
@@ -894,6 +898,9 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
 BwdArgs make_bwd_args(const Problem& p) {
   BwdArgs ba;
   ba.qa = make_pair_args(p);
+  ba.kgeo = ba.qa.geo;
+  ba.kitems = ba.qa.items;
+  ba.kloc0 = 0;
   return ba;
 }
 
@@ -902,6 +909,10 @@ BwdArgs make_bwd_args(const Problem& p) {
 bool tc_bwd_supported(const Problem& p) { return tc_shape_ok(p); }
 
 // D, NL: rows floats each; dq partials; dK/dV partials.
+int tc_dkdv_launches(const Problem& p) {
+  return (p.L >= kSplitMinL && make_geom(p.L, p.bs).n_mid > 0) ? 2 : 1;
+}
+
 size_t tc_bwd_extra_bytes(const Problem& p) {
   const size_t rows = (size_t)p.B * p.H * p.L;
   const Geom g = make_geom(p.L, p.bs);
@@ -939,16 +950,39 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   if (e != cudaSuccess) return e;
 
   const size_t smem_kv = 1024 + 4 * kTileBytes + kQStages * kQStageBytes;
-  auto* kv_kernel = p.L >= 16384 ? tc_dkdv_kernel<true> : tc_dkdv_kernel<false>;
-  e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem_kv);
-  if (e != cudaSuccess) return e;
-  kv_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_kv, s>>>(
-      ba, tm.q, tm.k, tm.v, tm.dout);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  e = marks->mark(s);
-  if (e != cudaSuccess) return e;
+  // From kSplitMinL the global key blocks' items (the only ones with the
+  // hi/lo split) run in a launch of their own, the middle windows without.
+  const Geom& g = ba.qa.geo;
+  const int nglob = g.n_git * g.nchunks;
+  struct Part {
+    bool split;
+    int per_bh, loc0;
+  };
+  Part parts[2];
+  int nparts = 0;
+  if (p.L >= kSplitMinL) {
+    parts[nparts++] = {true, nglob, 0};
+    if (g.n_mid > 0) parts[nparts++] = {false, g.n_mid, nglob};
+  } else {
+    parts[nparts++] = {false, g.per_bh, 0};
+  }
+  for (int i = 0; i < nparts; ++i) {
+    BwdArgs bk = ba;
+    bk.kgeo = g;
+    bk.kgeo.per_bh = parts[i].per_bh;
+    bk.kloc0 = parts[i].loc0;
+    bk.kitems = p.B * p.H * parts[i].per_bh;
+    auto* kv_kernel = parts[i].split ? tc_dkdv_kernel<true> : tc_dkdv_kernel<false>;
+    e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_kv);
+    if (e != cudaSuccess) return e;
+    kv_kernel<<<min(bk.kitems, 2 * sms), kThreads, smem_kv, s>>>(
+        bk, tm.q, tm.k, tm.v, tm.dout);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    e = marks->mark(s);
+    if (e != cudaSuccess) return e;
+  }
 
   const size_t frows = (size_t)p.B * p.H * ba.qa.geo.n_git * 128;
   bwd_finish_kernel<<<(unsigned)((frows + 7) / 8), 256, 0, s>>>(ba);

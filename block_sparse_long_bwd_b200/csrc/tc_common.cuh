@@ -29,6 +29,9 @@
 namespace bb {
 
 constexpr int kTile = 64;                             // tokens per tile
+// From this length on, the global key blocks' P^T and dS^T carry a bf16
+// low part in the dK/dV pass (they sum over every query row).
+constexpr int kSplitMinL = 16384;
 constexpr int kMaxT = 64;                             // tiles per item
 constexpr int kChunk = 8;                             // tiles per chunk
 constexpr uint32_t kTileBytes = kTile * kHeadDim * 2; // one 64 x 64 bf16 tile

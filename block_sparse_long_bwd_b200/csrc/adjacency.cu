@@ -359,6 +359,8 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
   const Geom g = make_geom(p.L, p.bs);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nitems = p.H * g.per_bh;
+  // The work counters of the tensor-core launches that follow.
+  if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
   const int id = blockIdx.x * kPlanWarps + warp;
   const int nq = do_q ? nitems : 0;
   if (id < nq) {

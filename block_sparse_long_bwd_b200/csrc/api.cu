@@ -111,6 +111,7 @@ int carve(Problem* p, int pass, void* ws, size_t ws_bytes) {
   if (ws_bytes < w.total) return BB_ERR_WORKSPACE;
   char* base = (char*)ws;
   p->status = (int*)(base + w.status_off);
+  p->sched = (int*)(base + w.status_off + 64);  // same 256-byte region
   if (pass == 1) {
     p->D = (float*)(base + w.D_off);
     p->csr_offs = (int*)(base + w.offs_off);

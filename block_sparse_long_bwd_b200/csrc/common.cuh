@@ -39,6 +39,7 @@ struct Problem {
   void* dv;
   // workspace pieces
   int* status;
+  int* sched;        // [4] work counters of the tensor-core launches (zeroed by the plan kernel)
   float* D;          // [B*H*L] (bwd)
   int* csr_offs;     // [H][nb+1] (bwd)
   int* csr_list;     // [H][csr_cap] (bwd)

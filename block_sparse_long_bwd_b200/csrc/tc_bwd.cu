@@ -38,6 +38,7 @@ struct BwdArgs {
   // [kloc0, kloc0 + kgeo.per_bh) (kgeo is qa.geo with per_bh narrowed).
   Geom kgeo;
   int kitems, kloc0;
+  int* kctr;  // this launch's work counter
   float* D;          // [B*H*L]
   float* NL;         // [B*H*L]: -lse * log2(e)
   float* dqpart;     // [B*H][n_git][nchunks][128][64]
@@ -108,6 +109,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   __shared__ DqBars bars;
   __shared__ TileList lists[2];  // bulk-copy destinations (16-byte aligned)
+  __shared__ int4 item_sh[2];    // (b, h, loc, 1) of the slot's item; w = 0: no more items
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -164,14 +166,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int q_issued = 0;
       uint32_t q_par = 0;
-      ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
-      for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
+      for (int k = 0;; ++k) {
         const int slot = k & 1;
         if (!mbar_wait(&bars.list_empty[slot], ((k >> 1) & 1) ^ 1, &abort_flag,
                        p.status))
           break;
         // Planned key-tile list: one bulk copy into the slot.
-        const ItemMeta m = cur.meta(a.geo, p.H);
+        // Items are taken from the launch's counter (middle windows first);
+        // the slot's (b, h, loc) is published by the list_full arrive.
+        int ib, ih, iloc;
+        if (!next_work(a.geo, p.B, p.H, 0, a.geo.per_bh, p.sched, ib, ih, iloc)) {
+          item_sh[slot] = make_int4(0, 0, 0, 0);
+          mbar_arrive_release(&bars.list_full[slot]);
+          break;
+        }
+        item_sh[slot] = make_int4(ib, ih, iloc, 1);
+        const ItemMeta m = item_meta_at(a.geo, ib, ih, p.H, iloc);
         const TileList& L = lists[slot];
         mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
         bulk_load(&lists[slot],
@@ -230,11 +240,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t qaddr = smem_u32(Qs), gaddr = smem_u32(Gs);
     uint32_t g = 0, u = 0;
     bool ok = true;
-    for (int k = 0, item = blockIdx.x; item < a.items && ok;
-         ++k, item += gridDim.x) {
+    for (int k = 0; ok; ++k) {
       const int slot = k & 1;
       if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
+      if (!item_sh[slot].w) break;
       const int n = lists[slot].n;
       if (!mbar_wait(&bars.q_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
@@ -323,13 +333,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;
-    ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
+    for (int k = 0;; ++k) {
       const int slot = k & 1;
       if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
+      const int4 wi = item_sh[slot];
+      if (!wi.w) break;
       const TileList& L = lists[slot];
-      const ItemMeta im = cur.meta(a.geo, p.H);
+      const ItemMeta im = item_meta_at(a.geo, wi.x, wi.y, p.H, wi.z);
       const int n = L.n;
       const bool rvalid = (im.gvalid >> quarter) & 1;
       const size_t grow = (size_t)im.bh * p.L + (size_t)(rvalid ? im.t[half] : 0) * kTile + r64;
@@ -497,6 +508,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                    const __grid_constant__ CUtensorMap tmG) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ KvBars bars;
+  __shared__ int4 kitem[2];  // (b, h, loc, 1) of item k in slot k & 1; w = 0: no more items
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -543,14 +555,22 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int kp_issued = 0;
       uint32_t kp_par = 0;
-      ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
-      for (int k = 0; cur.item < ba.kitems;
-           ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
-        const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
+      for (int k = 0;; ++k) {
+        if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        // Items are taken from the launch's counter (middle windows first);
+        // the slot's (b, h, loc) is published by the kp_full arrive.
+        int ib, ih, iloc;
+        if (!next_work(ba.qa.geo, p.B, p.H, ba.kloc0, ba.kgeo.per_bh, ba.kctr, ib, ih,
+                       iloc)) {
+          kitem[k & 1] = make_int4(0, 0, 0, 0);
+          mbar_arrive_release(&bars.kp_full);
+          break;
+        }
+        kitem[k & 1] = make_int4(ib, ih, iloc, 1);
+        const ItemMeta it = item_meta_at(ba.qa.geo, ib, ih, p.H, iloc);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.qa.geo, it, e0, e1);
-        if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
         mbar_expect_tx(&bars.kp_full, 2u * nh * kTileBytes);
@@ -606,14 +626,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
     uint32_t g = 0, u = 0;
     bool ok = true;
-    ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < ba.kitems && ok;
-         ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
-      const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
+    for (int k = 0; ok; ++k) {
+      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
+      const int4 wi = kitem[k & 1];
+      if (!wi.w) break;
+      const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
       int w0, w1;
       walk_range(p, ba.qa.geo, it, w0, w1);
       const int nwalk = w1 - w0;
-      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
       tc_fence_after();
       for (int t = 0; t < nwalk;) {
         const int st = g % kQStages;
@@ -694,10 +714,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t g = 0, u = 0;
-    ItemCursor cur(ba.kgeo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < ba.kitems;
-         ++k, cur.next(ba.kgeo, p.H, gridDim.x)) {
-      const ItemMeta it = item_meta_at(ba.qa.geo, cur.b, cur.h, p.H, cur.loc + ba.kloc0);
+    for (int k = 0;; ++k) {
+      // The item of this round: published with its K / V pair (kp_full).
+      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
+      const int4 wi = kitem[k & 1];
+      if (!wi.w) break;
+      const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
       int e0, e1;
       walk_range(p, ba.qa.geo, it, e0, e1);
@@ -901,6 +923,7 @@ BwdArgs make_bwd_args(const Problem& p) {
   ba.kgeo = ba.qa.geo;
   ba.kitems = ba.qa.items;
   ba.kloc0 = 0;
+  ba.kctr = p.sched + 1;
   return ba;
 }
 
@@ -972,6 +995,7 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     bk.kgeo.per_bh = parts[i].per_bh;
     bk.kloc0 = parts[i].loc0;
     bk.kitems = p.B * p.H * parts[i].per_bh;
+    bk.kctr = p.sched + 1 + i;  // sched[0]: dQ
     auto* kv_kernel = parts[i].split ? tc_dkdv_kernel<true> : tc_dkdv_kernel<false>;
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);

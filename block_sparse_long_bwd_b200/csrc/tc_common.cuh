@@ -202,38 +202,33 @@ __host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int
   return item_meta_at(g, bh / H, bh % H, H, item % g.per_bh);
 }
 
-// A CTA's items start, stride: the (b, h, loc) decomposition is stepped
-// forward instead of divided out at every item.
-struct ItemCursor {
-  int item, b, h, loc;
-  int step_bh, step_loc;
-  __device__ __forceinline__ ItemCursor(const Geom& g, int H, int start, int stride) {
-    item = start;
-    const int bh = start / g.per_bh;
-    loc = start % g.per_bh;
-    b = bh / H;
-    h = bh % H;
-    step_bh = stride / g.per_bh;
-    step_loc = stride % g.per_bh;
+// Next work item of a launch, taken from its counter: the locs [loc0, loc0 +
+// nloc) of every (b, h), middle windows first (longer tile lists), then the
+// global chunks, so the short items fill the end of the launch.  False when
+// none is left.
+__device__ __forceinline__ bool next_work(const Geom& g, int B, int H, int loc0, int nloc,
+                                          int* ctr, int& b, int& h, int& loc) {
+  const int nglob = g.n_git * g.nchunks;
+  const int mlo = max(loc0, nglob);
+  const int nmid = max(0, loc0 + nloc - mlo);
+  const int ngl = nloc - nmid;
+  const int BH = B * H;
+  const int w = atomicAdd(ctr, 1);
+  int bh;
+  if (w < BH * nmid) {
+    bh = w / nmid;
+    loc = mlo + w % nmid;
+  } else if (w < BH * nloc) {
+    const int w2 = w - BH * nmid;
+    bh = w2 / ngl;
+    loc = loc0 + w2 % ngl;
+  } else {
+    return false;
   }
-  __device__ __forceinline__ void next(const Geom& g, int H, int stride) {
-    item += stride;
-    loc += step_loc;
-    int dbh = step_bh;
-    if (loc >= g.per_bh) {
-      loc -= g.per_bh;
-      ++dbh;
-    }
-    h += dbh;
-    while (h >= H) {
-      h -= H;
-      ++b;
-    }
-  }
-  __device__ __forceinline__ ItemMeta meta(const Geom& g, int H) const {
-    return item_meta_at(g, b, h, H, loc);
-  }
-};
+  b = bh / H;
+  h = bh % H;
+  return true;
+}
 
 // Plans the key tiles of query-side item (h, loc) into L.  Returns false if
 // the random table held an entry outside [-1, nb) (ignored).

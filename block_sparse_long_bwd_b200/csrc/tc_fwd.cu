@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   __shared__ Bars bars;
   __shared__ TileList lists[2];  // bulk-copy destinations (16-byte aligned)
+  __shared__ int4 item_sh[2];    // (b, h, loc, 1) of the slot's item; w = 0: no more items
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -119,15 +120,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t g = 0;
       int qissued[2] = {0, 0};
       uint32_t qpar[2] = {0, 0};
-      ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
-      for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
+      for (int k = 0;; ++k) {
         const int slot = k & 1;
         const uint32_t ph = (k >> 1) & 1;
         if (!mbar_wait(&bars.list_empty[slot], ph ^ 1, &abort_flag, p.status))
           break;
         // The item's key-tile list was planned before this kernel: one bulk
         // copy into the slot (the producer waits for it like the others).
-        const ItemMeta m = cur.meta(a.geo, p.H);
+        // Items are taken from the launch's counter (middle windows first);
+        // the slot's (b, h, loc) is published by the list_full arrive.
+        int ib, ih, iloc;
+        if (!next_work(a.geo, p.B, p.H, 0, a.geo.per_bh, p.sched, ib, ih, iloc)) {
+          item_sh[slot] = make_int4(0, 0, 0, 0);
+          mbar_arrive_release(&bars.list_full[slot]);
+          break;
+        }
+        item_sh[slot] = make_int4(ib, ih, iloc, 1);
+        const ItemMeta m = item_meta_at(a.geo, ib, ih, p.H, iloc);
         const TileList& L = lists[slot];
         mbar_expect_tx(&bars.list_full[slot], sizeof(TileList));
         bulk_load(&lists[slot],
@@ -189,11 +198,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
     uint32_t g = 0, u = 0;  // K/V stage counter, tile counter
     bool ok = true;
-    for (int k = 0, item = blockIdx.x; item < a.items && ok;
-         ++k, item += gridDim.x) {
+    for (int k = 0; ok; ++k) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
       if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      if (!item_sh[slot].w) break;
       const int n = lists[slot].n;
       if (!mbar_wait(&bars.q_full[slot], ph, &abort_flag, p.status)) break;
       tc_fence_after();
@@ -265,13 +274,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;  // tile counter (same sequence as the MMA warp)
-    ItemCursor cur(a.geo, p.H, blockIdx.x, gridDim.x);
-    for (int k = 0; cur.item < a.items; ++k, cur.next(a.geo, p.H, gridDim.x)) {
+    for (int k = 0;; ++k) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
       if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      const int4 wi = item_sh[slot];
+      if (!wi.w) break;
       const TileList& L = lists[slot];
-      const ItemMeta im = cur.meta(a.geo, p.H);
+      const ItemMeta im = item_meta_at(a.geo, wi.x, wi.y, p.H, wi.z);
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
       bool ok = true;

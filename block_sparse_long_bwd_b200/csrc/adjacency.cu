@@ -305,14 +305,16 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
 // query block at block size 128, else 1), so its region starts at T times
 // the CSR offset of its first key block; global chunks (kChunk query tiles
 // each) follow T x (all CSR entries).
+// offs / list: the head's CSR (global memory, or shared memory when
+// stage is null: the lists are then read in place).
 __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
-                            int* stage, int lane) {
+                            const int* offs, const int* list, int* stage, int* cand,
+                            int lane) {
   const int item = h * g.per_bh + loc;
   KeyWalk w;
-  w.init(g, p.H, p.csr_offs, p.csr_list, p.csr_cap, item);
+  w.init_head(g, p.H, offs, list, item);
   uint32_t* walk = p.kplan + (size_t)h * p.kcap;
   int* kofs = p.kof + 2 * (size_t)item;
-  const int* offs = p.csr_offs + (size_t)h * (g.nb + 1);
   const int T = g.bs == 128 ? 2 : 1;
   int base, cap;
   if (w.global) {
@@ -325,10 +327,71 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
     base = T * offs[jf];
     cap = T * (offs[jl + 1] - offs[jf]);
   }
-  // Stage the (at most four) CSR lists in shared memory when they fit.
+  if (base < 0 || base + cap > p.kcap) {  // cannot happen within the bound
+    if (lane == 0) {
+      set_status(p.status, BB_ERR_BAD_TABLE);
+      kofs[0] = 0;
+      kofs[1] = 0;
+    }
+    return;
+  }
   int total = 0;
   for (int x = 0; x < w.nl; ++x) total += w.ln[x];
-  if (!w.global && total <= kStageCap) {
+  if (!w.global && total * T <= 128) {
+    // Warp-parallel: every (list entry, tile of its query block) as
+    // (tile << 8 | group-half bits), sorted, equal tiles merged.
+    int cum[5];
+    cum[0] = 0;
+    for (int x = 0; x < 4; ++x) cum[x + 1] = cum[x] + (x < w.nl ? w.ln[x] * T : 0);
+    for (int e = lane; e < 128; e += 32) {
+      int v = 0x7FFFFFFF;
+      if (e < cum[w.nl]) {
+        int x = 0;
+        while (e >= cum[x + 1]) ++x;
+        const int k = e - cum[x];
+        const int i = w.lp[x][k / T];  // attending query block
+        int tile, halves;
+        if (g.bs == 32) {
+          tile = i >> 1;
+          halves = 1 << (i & 1);
+        } else if (g.bs == 64) {
+          tile = i;
+          halves = 3;
+        } else {
+          tile = 2 * i + (k % T);
+          halves = 3;
+        }
+        v = (tile << 8) | expand_groups(w.lg[x], halves);
+      }
+      cand[e] = v;
+    }
+    __syncwarp();
+    warp_sort128(cand, lane);
+    int pos0 = 0;
+    for (int r = 0; r < 4; ++r) {
+      const int e = lane + 32 * r;
+      const int v = cand[e];
+      const bool head = v != 0x7FFFFFFF && (e == 0 || (cand[e - 1] >> 8) != (v >> 8));
+      int bits = 0;
+      if (head)
+        for (int x = e; x < 128 && cand[x] != 0x7FFFFFFF && (cand[x] >> 8) == (v >> 8); ++x)
+          bits |= cand[x] & 0xFF;
+      const unsigned hb = __ballot_sync(0xFFFFFFFFu, head);
+      if (head) {
+        const int pos = pos0 + __popc(hb & ((1u << lane) - 1));
+        if (pos < cap) walk[base + pos] = kentry(v >> 8, bits);
+      }
+      pos0 += __popc(hb);
+    }
+    if (lane == 0) {
+      kofs[0] = base;
+      kofs[1] = min(pos0, cap);
+    }
+    return;
+  }
+  // Otherwise one lane merges the lists (staged in shared memory when they
+  // fit).
+  if (stage && !w.global && total <= kStageCap) {
     int off = 0;
     for (int x = 0; x < w.nl; ++x) {
       for (int e = lane; e < w.ln[x]; e += 32) stage[off + e] = w.lp[x][e];
@@ -339,11 +402,6 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
   __syncwarp();
   if (lane == 0) {
     int n = 0, tile, mask;
-    if (base < 0 || base + cap > p.kcap) {  // cannot happen within the bound
-      set_status(p.status, BB_ERR_BAD_TABLE);
-      cap = 0;
-      base = 0;
-    }
     while (n < cap && w.next(tile, mask)) walk[base + n++] = kentry(tile, mask);
     kofs[0] = base;
     kofs[1] = n;
@@ -367,11 +425,149 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
     plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], stage[warp], lane);
   } else if (do_k && id - nq < nitems) {
     const int k = id - nq;
-    plan_k_item(p, g, k / g.per_bh, k % g.per_bh, stage[warp], lane);
+    const int h = k / g.per_bh;
+    plan_k_item(p, g, h, k % g.per_bh, p.csr_offs + (size_t)h * (g.nb + 1),
+                p.csr_list + (size_t)h * p.csr_cap, stage[warp], cand[warp], lane);
   }
 }
 
+// Transposed adjacency of head h built in shared memory by the whole CTA
+// (the same construction as csr_build_kernel): offs[nb + 1], then the lists.
+// Returns the lists' base; sm holds 2 nb + blockDim.x + (nb + 1) + csr_cap
+// ints.
+__device__ int* build_head_csr(const Problem& p, int h, int* sm, int*& offs) {
+  const int nb = p.nb, r = p.r, tid = threadIdx.x, nth = blockDim.x;
+  int* cnt = sm;
+  int* cur = cnt + nb;
+  int* tsum = cur + nb;
+  offs = tsum + nth;
+  int* list = offs + nb + 1;
+  const int32_t* table = p.rand_idx + (size_t)h * nb * r;
+  for (int j = tid; j < nb; j += nth) {
+    int c;
+    if (j == 0 || j == nb - 1) {
+      c = nb;
+    } else {
+      c = 2;  // global query rows 0 and nb-1
+      for (int i = j - 1; i <= j + 1; ++i) c += (i >= 1 && i <= nb - 2);
+    }
+    cnt[j] = c;
+  }
+  __syncthreads();
+  for (int x = tid; x < nb * r; x += nth) {
+    const int i = x / r, a = x % r;
+    if (i == 0 || i == nb - 1) continue;
+    const int j = random_target(table + (size_t)i * r, a, i, nb, p.status);
+    if (j >= 0) atomicAdd(&cnt[j], 1);
+  }
+  __syncthreads();
+  const int chunk = (nb + nth - 1) / nth;
+  const int c0 = tid * chunk, c1 = min(nb, c0 + chunk);
+  int local = 0;
+  for (int j = c0; j < c1; ++j) local += cnt[j];
+  tsum[tid] = local;
+  __syncthreads();
+  for (int step = 1; step < nth; step <<= 1) {
+    int add = tid >= step ? tsum[tid - step] : 0;
+    __syncthreads();
+    tsum[tid] += add;
+    __syncthreads();
+  }
+  int run = tsum[tid] - local;
+  for (int j = c0; j < c1; ++j) {
+    cur[j] = run;
+    offs[j] = run;
+    run += cnt[j];
+  }
+  if (tid == nth - 1) offs[nb] = tsum[nth - 1];
+  __syncthreads();
+  for (int x = tid; x < 2 * nb; x += nth) {
+    const int j = x < nb ? 0 : nb - 1;
+    const int i = x % nb;
+    if (x >= nb && nb == 1) continue;
+    list[cur[j] + i] = i;
+  }
+  for (int j = tid; j < nb; j += nth) {
+    if (j == 0 || j == nb - 1) continue;
+    int pos = atomicAdd(&cur[j], 2 + (j - 1 >= 1) + 1 + (j + 1 <= nb - 2));
+    list[pos++] = 0;
+    list[pos++] = nb - 1;
+    for (int i = j - 1; i <= j + 1; ++i)
+      if (i >= 1 && i <= nb - 2) list[pos++] = i;
+  }
+  for (int x = tid; x < nb * r; x += nth) {
+    const int i = x / r, a = x % r;
+    if (i == 0 || i == nb - 1) continue;
+    const int j = random_target(table + (size_t)i * r, a, i, nb, p.status);
+    if (j >= 0) list[atomicAdd(&cur[j], 1)] = i;
+  }
+  __syncthreads();
+  for (int j = tid; j < nb; j += nth) {
+    if (j == 0 || j == nb - 1) continue;
+    int* L = list + offs[j];
+    const int n = offs[j + 1] - offs[j];
+    for (int a = 1; a < n; ++a) {
+      int x = L[a], c = a - 1;
+      while (c >= 0 && L[c] > x) {
+        L[c + 1] = L[c];
+        --c;
+      }
+      L[c + 1] = x;
+    }
+  }
+  __syncthreads();
+  return list;
+}
+
+constexpr int kFusedWarps = 8;
+
+// Backward plans in one launch: the first qctas CTAs plan query-side items
+// (one warp each); the others each build one head's transposed adjacency in
+// shared memory and plan a slice of that head's key-side items from it
+// (kslices CTAs per head, so no CTA waits for another).
+__global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, int qctas,
+                                                                    int kslices) {
+  extern __shared__ int csr_sm[];
+  __shared__ int cand[kFusedWarps][128];
+  __shared__ int merged[kFusedWarps][128];
+  const Geom g = make_geom(p.L, p.bs);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
+  if ((int)blockIdx.x < qctas) {
+    const int id = blockIdx.x * kFusedWarps + warp;
+    if (id < p.H * g.per_bh)
+      plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], merged[warp], lane);
+    return;
+  }
+  const int kb = blockIdx.x - qctas;
+  const int h = kb / kslices, slice = kb % kslices;
+  int* offs;
+  const int* list = build_head_csr(p, h, csr_sm, offs);
+  for (int loc = slice * kFusedWarps + warp; loc < g.per_bh; loc += kslices * kFusedWarps)
+    plan_k_item(p, g, h, loc, offs, list, nullptr, cand[warp], lane);
+}
+
+size_t fused_plan_smem(const Problem& p) {
+  return (size_t)(2 * p.nb + 32 * kFusedWarps + p.nb + 1 + pair_cap(p.nb, p.r)) * sizeof(int);
+}
+
 }  // namespace
+
+bool tc_bwd_plan_fused(const Problem& p) { return fused_plan_smem(p) <= 160u * 1024u; }
+
+cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s) {
+  const Geom g = make_geom(p.L, p.bs);
+  const int nitems = p.H * g.per_bh;
+  const int qctas = (nitems + kFusedWarps - 1) / kFusedWarps;
+  // About two key-side items per warp.
+  const int kslices = max(1, (g.per_bh + 2 * kFusedWarps - 1) / (2 * kFusedWarps));
+  const size_t smem = fused_plan_smem(p);
+  cudaError_t e = cudaFuncSetAttribute(
+      plan_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  plan_bwd_kernel<<<qctas + p.H * kslices, 32 * kFusedWarps, smem, s>>>(p, qctas, kslices);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s) {
   const size_t rows = (size_t)p.B * p.H * p.L;

@@ -263,9 +263,13 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   if (tc_bwd_supported(p)) {
     TensorMaps tm;
     if (!encode_tensor_maps(p, 1, &tm)) return BB_ERR_CUDA;
-    if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
-    if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
-    if (launch_plan(p, true, s) != cudaSuccess) return BB_ERR_CUDA;
+    if (tc_bwd_plan_fused(p)) {
+      if (launch_plan_bwd(p, s) != cudaSuccess) return BB_ERR_CUDA;
+    } else {
+      if (launch_csr_build(p, s) != cudaSuccess) return BB_ERR_CUDA;
+      if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
+      if (launch_plan(p, true, s) != cudaSuccess) return BB_ERR_CUDA;
+    }
     if (marks->mark(s) != cudaSuccess) return BB_ERR_CUDA;
     if (launch_tc_bwd(p, tm, s, marks) != cudaSuccess) return BB_ERR_CUDA;
   } else {
@@ -285,12 +289,13 @@ static const char* const kFwdSimt[] = {"simt_fwd"};
 static const char* const kFwdTc[] = {"plan", "tc_fwd", "fwd_combine"};
 static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
                                        "simt_dkdv"};
-static const char* const kBwdTc[] = {"csr_build", "plan", "tc_dq", "tc_dkdv",
-                                     "bwd_finish"};
-// At long lengths dK/dV of the global key blocks (hi/lo split) and of the
-// middle windows are separate launches (tc_dkdv_launches).
-static const char* const kBwdTcSplit[] = {"csr_build", "plan", "tc_dq", "tc_dkdv",
-                                          "tc_dkdv", "bwd_finish"};
+// Tensor-core backward: the plans (with each head's transposed adjacency
+// built in shared memory, one launch) or, when a head's adjacency does not
+// fit there, csr_build + plan; then dQ, dK/dV (two launches at long lengths:
+// the global key blocks with the hi/lo split on their own,
+// tc_dkdv_launches), and the merge of the global rows' partials.
+static const char* const kBwdTcTail1[] = {"tc_dq", "tc_dkdv", "bwd_finish"};
+static const char* const kBwdTcTail2[] = {"tc_dq", "tc_dkdv", "tc_dkdv", "bwd_finish"};
 
 static int launch_plan(const bb_attn_desc* desc, int pass,
                        const char* const** names, int* n) {
@@ -303,10 +308,22 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     *names = tc ? kFwdTc : kFwdSimt;
     *n = tc ? 3 : 1;
   } else {
-    const bool tc = tc_bwd_supported(p);
-    const bool two = tc && tc_dkdv_launches(p) == 2;
-    *names = !tc ? kBwdSimt : two ? kBwdTcSplit : kBwdTc;
-    *n = !tc ? 4 : two ? 6 : 5;
+    if (!tc_bwd_supported(p)) {
+      *names = kBwdSimt;
+      *n = 4;
+      return BB_OK;
+    }
+    // Assembled per shape in a small table owned by this translation unit.
+    static thread_local const char* buf[8];
+    int c = 0;
+    if (!tc_bwd_plan_fused(p)) buf[c++] = "csr_build";
+    buf[c++] = "plan";
+    const bool two = tc_dkdv_launches(p) == 2;
+    const char* const* tail = two ? kBwdTcTail2 : kBwdTcTail1;
+    const int nt = two ? 4 : 3;
+    for (int i = 0; i < nt; ++i) buf[c++] = tail[i];
+    *names = buf;
+    *n = c;
   }
   return BB_OK;
 }

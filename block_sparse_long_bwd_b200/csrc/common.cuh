@@ -113,6 +113,11 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
 cudaError_t launch_simt_fwd(const Problem& p, cudaStream_t s);
 cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s);
 cudaError_t launch_csr_build(const Problem& p, cudaStream_t s);
+// Backward plans (query and key side, with each head's transposed adjacency
+// built in shared memory) in one launch; possible when a head's adjacency
+// fits in shared memory (tc_bwd_plan_fused).
+bool tc_bwd_plan_fused(const Problem& p);
+cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s);
 cudaError_t launch_simt_bwd(const Problem& p, cudaStream_t s, EventMarks* marks);
 
 // ---- device helpers -----------------------------------------------------

@@ -301,10 +301,15 @@ struct KeyWalk {
 
   __host__ __device__ void init(const Geom& g, int H, const int* csr_offs,
                                 const int* csr_list, int csr_cap, int item) {
+    const int h = item_meta(g, H, item).h;
+    init_head(g, H, csr_offs + (size_t)h * (g.nb + 1), csr_list + (size_t)h * csr_cap, item);
+  }
+  // Same, given the item's head's CSR offsets [nb + 1] and lists.
+  __host__ __device__ void init_head(const Geom& g, int H, const int* offs, const int* list,
+                                     int item) {
     const ItemMeta m = item_meta(g, H, item);
     bh = m.bh;
     b = m.b;
-    const int h = m.h;
     bs = g.bs;
     pend_tile = -1;
     pend_mask = 0;
@@ -321,8 +326,6 @@ struct KeyWalk {
       end = g.nt < cur + kChunk ? g.nt : cur + kChunk;
       return;
     }
-    const int* offs = csr_offs + (size_t)h * (g.nb + 1);
-    const int* list = csr_list + (size_t)h * csr_cap;
     for (int gr = 0; gr < 4; ++gr) {
       if (!(gvalid & (1 << gr))) continue;
       const int j = block_of(g, t[gr >> 1] * kTile + 32 * (gr & 1));

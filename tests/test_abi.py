@@ -129,17 +129,20 @@ def _names(desc, pass_):
 
 def test_launch_lists_follow_the_dispatch():
     """The launch list a pass reports (what event timing is keyed by): the
-    tensor-core path for bf16 shapes, one dK/dV launch below 16384 tokens and
-    two from there (global key blocks with the hi/lo split on their own),
-    the CUDA-core path for fp32."""
+    tensor-core path for bf16 shapes (backward plans in one launch while a
+    head's transposed adjacency fits in shared memory), one dK/dV launch
+    below 16384 tokens and two from there (global key blocks with the hi/lo
+    split on their own), the CUDA-core path for fp32."""
     import torch
     short = bb.make_desc(2, 4, 4096, 64, 64, 3, torch.bfloat16)
     assert _names(short, 0) == ["plan", "tc_fwd", "fwd_combine"]
-    assert _names(short, 1) == ["csr_build", "plan", "tc_dq", "tc_dkdv", "bwd_finish"]
+    assert _names(short, 1) == ["plan", "tc_dq", "tc_dkdv", "bwd_finish"]
     for bs in (32, 64, 128):
         long_ = bb.make_desc(1, 2, 16384, 64, bs, 3, torch.bfloat16)
-        assert _names(long_, 1) == ["csr_build", "plan", "tc_dq", "tc_dkdv", "tc_dkdv",
-                                    "bwd_finish"], bs
+        assert _names(long_, 1) == ["plan", "tc_dq", "tc_dkdv", "tc_dkdv", "bwd_finish"], bs
     f32 = bb.make_desc(1, 2, 1024, 64, 64, 3, torch.float32)
     assert _names(f32, 0) == ["simt_fwd"]
     assert _names(f32, 1) == ["bwd_pre", "csr_build", "simt_dq", "simt_dkdv"]
+    # A head's adjacency too large for shared memory: CSR built separately.
+    huge = bb.make_desc(1, 1, 131072, 64, 32, 3, torch.bfloat16)
+    assert _names(huge, 1)[:2] == ["csr_build", "plan"]

@@ -896,6 +896,9 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
   const size_t grow = bh * p.L + (size_t)t[row >> 6] * kTile + (row & 63);
   const size_t ib = (bh * g.n_git + gi) * g.nchunks;
   float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+  // Unrolled so that several chunks' loads are in flight at once (the sums
+  // keep the chunk order).
+#pragma unroll 8
   for (int c = 0; c < g.nchunks; ++c) {
     const float2 x = reinterpret_cast<const float2*>(
         ba.dqpart + ((ib + c) * 128 + row) * 64)[lane];

@@ -501,9 +501,12 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
   item_rows(g, true, gi, t, gvalid);
   if (!((gvalid >> (row >> 5)) & 1)) return;
   const float* base = p.part + ((bh * g.n_git + gi) * g.nchunks * 128 + row) * kPartStride;
+  // Unrolled so that several chunks' loads are in flight at once.
   float M = -INFINITY;
+#pragma unroll 8
   for (int c = 0; c < g.nchunks; ++c) M = fmaxf(M, base[(size_t)c * 128 * kPartStride + 64]);
   float Lsum = 0.f, o0 = 0.f, o1 = 0.f;
+#pragma unroll 8
   for (int c = 0; c < g.nchunks; ++c) {
     const float* src = base + (size_t)c * 128 * kPartStride;
     const float w = ex2(src[64] - M);

@@ -176,6 +176,44 @@ __device__ __forceinline__ void warp_sort128(int* v, int lane) {
   }
 }
 
+// Bitonic sort of 64 ints held two per lane (element lane in a, lane + 32
+// in b), by shuffles: no shared memory and no barriers.
+__device__ __forceinline__ void warp_sort64(int& a, int& b, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j == 32) {  // partners in the same lane (only for k = 64: ascending)
+        const int lo = min(a, b), hi = max(a, b);
+        a = lo;
+        b = hi;
+      } else {
+        const int oa = __shfl_xor_sync(0xFFFFFFFFu, a, j);
+        const int ob = __shfl_xor_sync(0xFFFFFFFFu, b, j);
+        const bool lower = (lane & j) == 0;
+        const bool upa = (lane & k) == 0, upb = ((lane + 32) & k) == 0;
+        a = (lower == upa) ? min(a, oa) : max(a, oa);
+        b = (lower == upb) ? min(b, ob) : max(b, ob);
+      }
+    }
+  }
+}
+
+// Sorts cand[0..128); when every real entry sits in cand[0..64) (the rest
+// being the 0x7FFFFFFF filler), in registers.
+__device__ __forceinline__ void warp_sort_cand(int* cand, int used, int lane) {
+  if (used <= 64) {
+    int a = cand[lane], b = cand[lane + 32];
+    __syncwarp();
+    warp_sort64(a, b, lane);
+    cand[lane] = a;
+    cand[lane + 32] = b;
+    __syncwarp();
+  } else {
+    warp_sort128(cand, lane);
+  }
+}
+
 // Query-side plan of item (h, loc), one warp: every (group, attended block,
 // tile) candidate as (tile << 8 | mask bits), sorted, equal tiles merged.
 __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
@@ -227,7 +265,7 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
   }
   if (bad) set_status(p.status, BB_ERR_BAD_TABLE);
   __syncwarp();
-  warp_sort128(cand, lane);
+  warp_sort_cand(cand, 4 * S * T, lane);
   // Merge equal tiles into the sorted list (mt, mm) in shared memory.
   int* mt = merged;
   int* mm = merged + kMaxT;
@@ -366,7 +404,7 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
       cand[e] = v;
     }
     __syncwarp();
-    warp_sort128(cand, lane);
+    warp_sort_cand(cand, cum[w.nl], lane);
     int pos0 = 0;
     for (int r = 0; r < 4; ++r) {
       const int e = lane + 32 * r;
@@ -559,8 +597,9 @@ cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s) {
   const Geom g = make_geom(p.L, p.bs);
   const int nitems = p.H * g.per_bh;
   const int qctas = (nitems + kFusedWarps - 1) / kFusedWarps;
-  // About two key-side items per warp.
-  const int kslices = max(1, (g.per_bh + 2 * kFusedWarps - 1) / (2 * kFusedWarps));
+  // One key-side item per warp (each CTA rebuilds its head's small
+  // adjacency, so more CTAs per head cost only parallel work).
+  const int kslices = max(1, (g.per_bh + kFusedWarps - 1) / kFusedWarps);
   const size_t smem = fused_plan_smem(p);
   cudaError_t e = cudaFuncSetAttribute(
       plan_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

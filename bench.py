@@ -49,12 +49,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 # captured, that file, the workload captured).  Another workload or a
 # changed source reports null.
 NCU_TRAFFIC = {
-    # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, 1 launch)
-    "tc_fwd": (147637504 + 31209472, "59074614694c826e", "tc_fwd.cu",
+    # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, 1 launch;
+    # hashes refreshed after comment-only edits of the sources)
+    "tc_fwd": (147637504 + 31209472, "0f41c4d9c5be114a", "tc_fwd.cu",
                "large_train_l4096"),
-    "tc_dq": (224994560 + 33675264, "10b1282167afe315", "tc_bwd.cu",
+    "tc_dq": (224994560 + 33675264, "44becb5d0e98a1ed", "tc_bwd.cu",
               "large_train_l4096"),
-    "tc_dkdv": (200701696 + 64869376, "10b1282167afe315", "tc_bwd.cu",
+    "tc_dkdv": (200701696 + 64869376, "44becb5d0e98a1ed", "tc_bwd.cu",
                 "large_train_l4096"),
 }
 

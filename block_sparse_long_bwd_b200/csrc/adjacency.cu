@@ -1,5 +1,9 @@
-// Backward preprocessing: D = rowsum(dO * O) and the transposed block
-// adjacency (for each key block j, the sorted query blocks i with j in A(i)).
+// Planning and preprocessing: the tensor-core kernels' tile plans (query
+// side: each item's merged, ordered key tiles with group masks; key side:
+// each item's walk of attending query tiles), the transposed block
+// adjacency (for each key block j, the sorted query blocks i with j in A(i);
+// built per head in shared memory by the backward's planning launch, or in
+// global memory), and D = rowsum(dO * O) for the CUDA-core backward.
 #include "tc_common.cuh"
 
 namespace bb {

@@ -1,22 +1,25 @@
-// Tensor-core backward of the block-sparse attention (bf16 I/O, block 64,
-// d 64) for sm_100a.  Probabilities are recomputed from the forward's lse
-// (P = exp(S - lse)), so nothing of size pairs x bs^2 is stored.
+// Tensor-core backward of the block-sparse attention (bf16 I/O, blocks of
+// 32, 64 or 128 tokens, d 64) for sm_100a.  Probabilities are recomputed
+// from the forward's lse (P = exp(S - lse)), so nothing of size pairs x bs^2
+// is stored.  Items (see tc_common.cuh) are taken from a per-launch counter.
 //
-// tc_dq_kernel: query-side items (as in the forward: middle 128-row windows
-//   and chunks of the global rows; see tc_common.cuh).  Per key block j of the item:
-//   S = Q K_j^T and dP = dO V_j^T into TMEM; one thread per row forms
+// tc_dq_kernel: query-side items (as in the forward).  Per key tile of the
+//   item: S = Q K^T and dP = dO V^T into TMEM; one thread per row forms
 //   dS = P (dP - D) (D = <dO, O> of the row, computed at the start of the
 //   item and also written to the workspace with -lse*log2(e) for the next
-//   kernel); dS (bf16) goes back to TMEM and dQ += dS K_j accumulates in
-//   TMEM across the item.  Global rows write fp32 partials per chunk.
+//   kernel) into dS columns of its own, so the next tile's S and dP are
+//   computed as soon as this tile's have been read; dQ += dS K accumulates
+//   in TMEM across the item.  Global rows write fp32 partials per chunk.
 // tc_dkdv_kernel: key-side items take 128 key rows (a middle window of two
-//   key tiles) and walk the merged transposed adjacency lists (the query
-//   blocks that attend their key blocks, from the CSR), as query tiles with
-//   a group/half mask; the global key blocks, attended by every query block,
-//   are split into chunks of query tiles.  Per query block i: S^T = K_pair Q_i^T and dP^T = V_pair dO_i^T;
-//   P^T and dS^T (bf16) back to TMEM; dV += P^T dO_i and dK += dS^T Q_i
-//   accumulate in TMEM.  Each key row is owned by exactly one item (or one
-//   chunk partial), so there are no atomics.
+//   key tiles) and walk the planned query tiles that attend them (from the
+//   transposed adjacency), each with a group/half mask; the global key
+//   blocks, attended by every query block, are split into chunks of query
+//   tiles.  Per query tile: S^T = K_pair Q^T and dP^T = V_pair dO^T; P^T and
+//   dS^T (bf16) back over them in TMEM; dV += P^T dO and dK += dS^T Q
+//   accumulate in TMEM.  From kSplitMinL the global key blocks run in a
+//   launch of their own with a bf16 low part of P^T and dS^T.  Each key row
+//   is owned by exactly one item (or one chunk partial), so there are no
+//   atomics on data.
 // bwd_finish_kernel: sums the chunk partials of the global query rows (dQ)
 //   and of the global key blocks (dK, dV) in a fixed order.
 #include "tc_common.cuh"

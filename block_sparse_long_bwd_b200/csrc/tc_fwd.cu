@@ -1,6 +1,7 @@
-// Tensor-core forward of the block-sparse attention (bf16 I/O, block 64,
-// d 64) for sm_100a: TMA tile loads, tcgen05 MMAs with TMEM accumulators and
-// an online softmax, in a persistent warp-specialised kernel.
+// Tensor-core forward of the block-sparse attention (bf16 I/O, blocks of
+// 32, 64 or 128 tokens, d 64) for sm_100a: TMA tile loads, tcgen05 MMAs with
+// TMEM accumulators and an online softmax, in a persistent warp-specialised
+// kernel.
 //
 // Work item = 128 query rows of one (b, h) in one 128-row MMA tile (see
 // tc_common.cuh): a middle window streams the union of its row groups'
@@ -8,13 +9,16 @@
 // 32 columns; a global item streams a chunk of all key tiles for the rows of
 // blocks 0 and nb-1 and writes partial (O, m, l) that fwd_combine_kernel
 // merges.  Blocks of 32, 64 and 128 tokens all map onto 64-token tiles.
+// Items are taken from a per-launch counter (middle windows first).
 //
-// Roles (192 threads): warp 0 lane 0 issues TMA loads (Q pair once per item,
-// K and V per key block through a kNST-stage ring); warp 1 lane 0 issues the
-// MMAs (S = Q K^T into one of two TMEM S buffers, then O_part = P V with P
-// read from TMEM); warps 2-5 run the softmax, one thread per tile row: load
-// S from TMEM, fold scale, key mask and running max, write P (bf16) back
-// over S, and accumulate O_part into registers with the rescale factor.
+// Roles (192 threads): warp 0 lane 0 takes the next item, bulk-copies its
+// planned tile list and issues the TMA loads (Q pair once per item, K and V
+// per key tile through a kNST-stage ring); warp 1 lane 0 issues the MMAs
+// (S = Q K^T into one of two TMEM S buffers, O += P V with P read from one
+// of two TMEM P buffers); warps 2-5 run the softmax, one thread per tile
+// row: load S, fold scale, masks and the lazy running max, write P (bf16
+// pairs) and rescale O in TMEM when the max moves; at the end of an item
+// they normalise O and store it through shared memory with a TMA store.
 #include "tc_common.cuh"
 
 namespace bb {

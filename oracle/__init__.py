@@ -2,12 +2,17 @@
 
 from .bigbird_oracle import (  # noqa: F401
     DEFAULT_MASK_VALUE,
+    Dropout,
     SplitMix64,
     attended_blocks,
     backward,
     block_probs,
+    dropout_keep,
+    dropout_scale,
+    dropout_threshold,
     forward,
     pair_count,
+    philox4x32_10,
     rand_table,
     random_candidates,
 )

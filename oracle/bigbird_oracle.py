@@ -44,6 +44,17 @@ Readings taken where the pages are silent (each listed in the design doc):
   Fisher-Yates shuffle draws r_eff = min(r, |cand|) of them; the chosen ids
   are written sorted ascending, unused slots and rows 0 and nb-1 hold -1.
 
+* Attention dropout ([GC] sections "BigBirdEncoder 的关键参数", which lists
+  attention_dropout_rate = 0.1, and "梯度检查点的实现方式", which requires
+  stateless, seeded dropout so a recomputed forward draws the same noise):
+  the dropout multiplies the attended softmax probabilities by 0 (dropped)
+  or 1 / keep probability (kept); the lse is that of the undropped softmax.
+  The keep decision of element (b, h, t, u) is this library's own
+  specification (the pages give no generator): Philox4x32-10 (Salmon et
+  al., SC 2011) with counter (u >> 4, t, h, b) and the 64-bit seed as key;
+  byte u & 15 of its 16 little-endian output bytes is compared with the
+  rate rounded to 1/256 (dropped when below).
+
 The backward pass is the gradient of the forward's definition (the pages do
 not spell it out; the pages' layer trains with autodiff and recomputation):
 D_t = <dO_t, o_t>, dS_tu = p_tu (<dO_t, v_u> - D_t), dq_t = scale sum_u
@@ -54,7 +65,10 @@ masked softmax attention, torch fp64 autograd, finite differences, library
 SDPA on the shapes where the pattern is dense, a closed-form adjacency
 read-out and invariants; tests/test_rand_table.py checks the generator
 against the published SplitMix64 outputs and the table's defining
-properties.
+properties; tests/test_dropout_oracle.py checks the dropout generator
+against the published Philox4x32-10 known-answer vectors and the dropped
+forward and backward against dense torch fp64 with autograd and finite
+differences.
 """
 
 import math
@@ -121,6 +135,112 @@ def attended_blocks(i, num_blocks, rand_row):
     return sorted(j for j in s if 0 <= j < num_blocks)
 
 
+# ---------------------------------------------------------------------------
+# Seeded attention dropout.
+#
+# [GC] section "BigBirdEncoder 的关键参数" lists attention_dropout_rate (0.1 by
+# default) beside the ordinary dropout rate; section "梯度检查点的实现方式"
+# explains that, under recomputation, the dropout must be stateless and
+# seeded so that the recomputed forward draws the same noise.  Readings
+# (listed in the design doc): the dropout acts on the softmax probabilities of the
+# attended keys (the usual attention dropout), the lse stays that of the
+# undropped softmax, and the keep decision of element (b, h, t, u) is a pure
+# function of (seed, b, h, t, u), drawn from Philox4x32-10 as specified below.
+# ---------------------------------------------------------------------------
+
+_MASK32 = 0xFFFFFFFF
+# Philox4x32 constants from the published generator (J. K. Salmon,
+# M. A. Moraes, R. O. Dror and D. E. Shaw, "Parallel random numbers: as easy
+# as 1, 2, 3", SC 2011): the two round multipliers and the two Weyl
+# increments of the key schedule.
+_PHILOX_M0 = 0xD2511F53
+_PHILOX_M1 = 0xCD9E8D57
+_PHILOX_W0 = 0x9E3779B9
+_PHILOX_W1 = 0xBB67AE85
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds on arrays of counters.
+
+    ctr: four arrays (broadcastable, values < 2**32) c0..c3; key: two ints
+    k0, k1.  Returns the four output words as uint64 arrays holding 32-bit
+    values.  Each round multiplies c0 by M0 and c2 by M1 into 64-bit
+    products; the new words are (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2),
+    hi(M0 c0) ^ c3 ^ k1, lo(M0 c0)); between rounds the key advances by the
+    Weyl increments (W0, W1) modulo 2**32."""
+    c = [np.asarray(x, dtype=np.uint64) & np.uint64(_MASK32) for x in ctr]
+    c = list(np.broadcast_arrays(*c))
+    k0 = int(key[0]) & _MASK32
+    k1 = int(key[1]) & _MASK32
+    m32 = np.uint64(_MASK32)
+    sh = np.uint64(32)
+    for rnd in range(10):
+        if rnd:
+            k0 = (k0 + _PHILOX_W0) & _MASK32
+            k1 = (k1 + _PHILOX_W1) & _MASK32
+        p0 = c[0] * np.uint64(_PHILOX_M0)  # < 2**64: exact in uint64
+        p1 = c[2] * np.uint64(_PHILOX_M1)
+        c = [(p1 >> sh) ^ c[1] ^ np.uint64(k0), p1 & m32,
+             (p0 >> sh) ^ c[3] ^ np.uint64(k1), p0 & m32]
+    return c
+
+
+def dropout_threshold(rate):
+    """Byte threshold of a dropout rate: the rate rounded to the nearest
+    multiple of 1/256 (halves up), as an integer thr in [0, 255]; an element
+    is dropped when its byte is below thr."""
+    rate = float(rate)
+    if not 0.0 <= rate < 1.0:
+        raise ValueError("dropout rate must be in [0, 1)")
+    thr = int(math.floor(rate * 256.0 + 0.5))
+    if thr > 255:
+        raise ValueError("dropout rate rounds to 1")
+    return thr
+
+
+def dropout_scale(rate):
+    """Factor applied to kept probabilities: 1 / keep probability, with the
+    keep probability (256 - thr) / 256 of the rounded rate, so the dropped
+    probabilities are unbiased."""
+    return 256.0 / (256 - dropout_threshold(rate))
+
+
+def dropout_keep(seed, b, h, rows, cols, rate):
+    """bool [len(rows), len(cols)] keep decisions of query tokens rows and key
+    tokens cols of batch b, head h.
+
+    Element (b, h, t, u) draws Philox4x32-10 with counter
+    (u >> 4, t, h, b) and key (seed mod 2**32, seed >> 32); the 16 output
+    bytes, taken little-endian from the words in order, belong to the key
+    tokens 16 (u >> 4) .. 16 (u >> 4) + 15, and byte u & 15 decides.  The
+    element is kept when its byte is >= dropout_threshold(rate)."""
+    thr = dropout_threshold(rate)
+    seed = int(seed) & _MASK64
+    t = np.asarray(rows, dtype=np.uint64)[:, None]
+    u = np.asarray(cols, dtype=np.uint64)[None, :]
+    words = philox4x32_10((u >> np.uint64(4), t, np.uint64(h), np.uint64(b)),
+                          (seed & _MASK32, seed >> 32))
+    j = (u & np.uint64(15)).astype(np.int64)
+    w = np.choose(np.broadcast_to(j >> 2, words[0].shape), words)
+    byte = (w >> (np.uint64(8) * (u & np.uint64(3)))) & np.uint64(0xFF)
+    return byte >= np.uint64(thr)
+
+
+class Dropout:
+    """Attention dropout of one call: rate in [0, 1) and a 64-bit seed."""
+
+    def __init__(self, rate, seed):
+        dropout_threshold(rate)  # validates
+        self.rate = float(rate)
+        self.seed = int(seed) & _MASK64
+
+    def factors(self, b, h, rows, cols):
+        """[len(rows), len(cols)] multipliers of the probabilities: the
+        scale where kept, 0 where dropped."""
+        keep = dropout_keep(self.seed, b, h, rows, cols, self.rate)
+        return np.where(keep, dropout_scale(self.rate), 0.0)
+
+
 def _prep(x):
     return np.asarray(x, dtype=np.float64)
 
@@ -161,11 +281,13 @@ def block_probs(q, k, key_mask, table, block_size, b, h, i, scale=None,
 
 
 def forward(q, k, v, key_mask, table, block_size, scale=None,
-            mask_value=DEFAULT_MASK_VALUE):
+            mask_value=DEFAULT_MASK_VALUE, dropout=None):
     """Block-sparse attention forward: (o [B,H,L,d], lse [B,H,L]) in fp64.
 
     q, k, v: [B, H, L, d] (any float dtype, read as fp64); key_mask: None or
-    [B, L] with nonzero = attend; table: int [H, nb, r]."""
+    [B, L] with nonzero = attend; table: int [H, nb, r].  dropout: None or a
+    Dropout; o then sums the kept probabilities times the dropout scale,
+    while lse stays that of the undropped softmax."""
     q = _prep(q)
     k = _prep(k)
     v = _prep(v)
@@ -181,17 +303,23 @@ def forward(q, k, v, key_mask, table, block_size, scale=None,
             for i in range(nb):
                 cols, p, l = block_probs(q, k, key_mask, table, bs, b, h, i,
                                          scale, mask_value)
+                if dropout is not None:
+                    p = p * dropout.factors(b, h, np.arange(i * bs, (i + 1) * bs),
+                                            cols)
                 o[b, h, i * bs:(i + 1) * bs] = p @ v[b, h, cols]
                 lse[b, h, i * bs:(i + 1) * bs] = l
     return o, lse
 
 
 def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
-             mask_value=DEFAULT_MASK_VALUE):
+             mask_value=DEFAULT_MASK_VALUE, dropout=None):
     """Gradient of forward's o with respect to q, k, v for upstream dout.
 
     Returns (dq, dk, dv), each [B, H, L, d] fp64.  Probabilities and o are
-    recomputed here from the definition, in fp64."""
+    recomputed here from the definition, in fp64.  With dropout (factors
+    m_tu: the scale where kept, 0 where dropped) o_t = sum_u m_tu p_tu v_u,
+    so D_t = <dO_t, o_t> still, dS_tu = p_tu (m_tu <dO_t, v_u> - D_t) and
+    dv_u = sum_t m_tu p_tu dO_t."""
     q = _prep(q)
     k = _prep(k)
     v = _prep(v)
@@ -213,14 +341,18 @@ def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
                 vc = v[b, h, cols]
                 kc = k[b, h, cols]
                 do_i = dout[b, h, rows]
-                o_i = p @ vc
+                m = 1.0
+                if dropout is not None:
+                    m = dropout.factors(b, h, np.arange(i * bs, (i + 1) * bs),
+                                        cols)
+                o_i = (m * p) @ vc
                 D = (do_i * o_i).sum(axis=1)
-                dP = do_i @ vc.T
+                dP = m * (do_i @ vc.T)
                 dS = p * (dP - D[:, None])
                 dq[b, h, rows] = scale * (dS @ kc)
                 # cols holds each key token once, so fancy-index += is exact.
                 dk[b, h, cols] += scale * (dS.T @ q[b, h, rows])
-                dv[b, h, cols] += p.T @ do_i
+                dv[b, h, cols] += (m * p).T @ do_i
     return dq, dk, dv
 
 

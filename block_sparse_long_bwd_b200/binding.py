@@ -34,7 +34,8 @@ class bb_attn_desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("L", ctypes.c_int),
                 ("d", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("r", ctypes.c_int), ("dtype", ctypes.c_int),
-                ("scale", ctypes.c_float), ("mask_value", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("mask_value", ctypes.c_float),
+                ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_uint64)]
 
 
 _lib = None
@@ -98,10 +99,12 @@ def bb_abi_version():
     return lib().bb_abi_version()
 
 
-def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0):
+def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0,
+              dropout=0.0, dropout_seed=0):
     if isinstance(dtype, torch.dtype):
         dtype = {torch.float32: BB_F32, torch.bfloat16: BB_BF16}[dtype]
-    return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value)
+    return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value,
+                        dropout, dropout_seed & ((1 << 64) - 1))
 
 
 def _check(code, what):
@@ -167,9 +170,11 @@ def _cuda_tensor(t, name, dtype=None):
         raise ValueError(f"{name} must be {dtype}")
 
 
-def desc_for(q, block_size, r, scale=0.0, mask_value=0.0):
+def desc_for(q, block_size, r, scale=0.0, mask_value=0.0, dropout=0.0,
+             dropout_seed=0):
     B, H, L, d = q.shape
-    return make_desc(B, H, L, d, block_size, r, q.dtype, scale, mask_value)
+    return make_desc(B, H, L, d, block_size, r, q.dtype, scale, mask_value,
+                     dropout, dropout_seed)
 
 
 def bb_attn_fwd(desc, q, k, v, key_mask, rand_idx, out, lse, workspace,
@@ -243,9 +248,10 @@ class Attention:
     library; every call below goes straight to the C entry points."""
 
     def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
-                 device="cuda", scale=0.0, mask_value=0.0):
+                 device="cuda", scale=0.0, mask_value=0.0, dropout=0.0,
+                 dropout_seed=0):
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
-                              mask_value)
+                              mask_value, dropout, dropout_seed)
         self.dtype = dtype
         nb = L // block_size
         self.table_host = bb_rand_attn_build(seed, H, nb, r)

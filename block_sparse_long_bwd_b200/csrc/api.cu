@@ -94,6 +94,11 @@ int make_problem(const bb_attn_desc* desc, Problem* p) {
   if (p->L % p->bs != 0) return BB_ERR_INVALID;
   if (!isfinite(desc->scale) || !isfinite(desc->mask_value))
     return BB_ERR_INVALID;
+  // Dropout rate in [0, 1), rounded to 1/256; a rate that rounds to 1 would
+  // drop everything (infinite scale).
+  if (!(desc->dropout >= 0.f && desc->dropout < 1.f)) return BB_ERR_INVALID;
+  const double thr = floor((double)desc->dropout * 256.0 + 0.5);
+  if (thr > 255.0) return BB_ERR_INVALID;
   if (p->d != kHeadDim) return BB_ERR_UNSUPPORTED;
   if (p->bs != 32 && p->bs != 64 && p->bs != 128) return BB_ERR_UNSUPPORTED;
   p->nb = p->L / p->bs;
@@ -101,6 +106,9 @@ int make_problem(const bb_attn_desc* desc, Problem* p) {
   if (p->H > 65535 || p->B > 65535) return BB_ERR_UNSUPPORTED;
   p->scale = desc->scale != 0.f ? desc->scale : 1.0f / sqrtf((float)p->d);
   p->mask_value = desc->mask_value != 0.f ? desc->mask_value : -10000.0f;
+  p->drop_thr = (uint32_t)thr;
+  p->drop_scale = (float)(256.0 / (256.0 - thr));
+  p->drop_seed = desc->dropout_seed;
   return BB_OK;
 }
 

@@ -22,6 +22,10 @@ struct Problem {
   int B, H, L, d, bs, r, nb, dtype;
   float scale;       // resolved (never 0)
   float mask_value;  // resolved (never 0)
+  // attention dropout: byte threshold (0: off), 1 / keep probability, seed
+  uint32_t drop_thr;
+  float drop_scale;
+  uint64_t drop_seed;
   // inputs
   const void* q;
   const void* k;

@@ -7,8 +7,10 @@
 // value block in shared memory, with an online softmax in the log2 domain.
 // Backward: dQ per query block as above; dK/dV per key block over the
 // transposed block adjacency (CSR, built by csr_build_kernel), without
-// atomics.
+// atomics.  With dropout each element's keep decision is drawn on its own
+// (one Philox call per element; these kernels are the fp32 correctness path).
 #include "common.cuh"
+#include "dropout.cuh"
 
 namespace bb {
 namespace {
@@ -111,15 +113,18 @@ __global__ void __launch_bounds__(BS) simt_fwd_kernel(Problem p) {
 #pragma unroll
       for (int u = 0; u < kChunk; ++u) {
         const float pu = exp2f(s[u] - mn);
-        l += pu;
+        l += pu;  // the lse is that of the undropped softmax
+        float pw = pu;
+        if (p.drop_thr)
+          pw = keep_one(p, b, h, i * BS + tid, j * BS + c0 + u) ? pu * p.drop_scale : 0.f;
         const float4* v4 = reinterpret_cast<const float4*>(Vs + (c0 + u) * kHeadDim);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           float4 x = v4[c];
-          o[4 * c + 0] = fmaf(pu, x.x, o[4 * c + 0]);
-          o[4 * c + 1] = fmaf(pu, x.y, o[4 * c + 1]);
-          o[4 * c + 2] = fmaf(pu, x.z, o[4 * c + 2]);
-          o[4 * c + 3] = fmaf(pu, x.w, o[4 * c + 3]);
+          o[4 * c + 0] = fmaf(pw, x.x, o[4 * c + 0]);
+          o[4 * c + 1] = fmaf(pw, x.y, o[4 * c + 1]);
+          o[4 * c + 2] = fmaf(pw, x.z, o[4 * c + 2]);
+          o[4 * c + 3] = fmaf(pw, x.w, o[4 * c + 3]);
         }
       }
       m = mn;
@@ -177,7 +182,10 @@ __global__ void __launch_bounds__(BS) simt_dq_kernel(Problem p) {
     for (int u = 0; u < BS; ++u) {
       const float* kr = Ks + u * kHeadDim;
       const float pu = exp2f(dot64(q, kr) + koff[u] - lse2);
-      const float ds = pu * (dot64(g, Vs + u * kHeadDim) - Dt);
+      float dpv = dot64(g, Vs + u * kHeadDim);
+      if (p.drop_thr)
+        dpv = keep_one(p, b, h, i * BS + tid, j * BS + u) ? dpv * p.drop_scale : 0.f;
+      const float ds = pu * (dpv - Dt);
       const float4* k4 = reinterpret_cast<const float4*>(kr);
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
@@ -247,16 +255,22 @@ __global__ void __launch_bounds__(2 * BS) simt_dkdv_kernel(Problem p) {
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       dp += __shfl_xor_sync(0xffffffffu, dp, 1);
       const float pu = exp2f(s + ko - lse2[t]);
+      float pw = pu;
+      if (p.drop_thr) {
+        const float m = keep_one(p, b, h, i * BS + t, j * BS + u) ? p.drop_scale : 0.f;
+        dp *= m;
+        pw = pu * m;
+      }
       const float ds = pu * (dp - Ds[t]);
       const float4* q4 = reinterpret_cast<const float4*>(qt);
       const float4* g4 = reinterpret_cast<const float4*>(gt);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         float4 a = g4[c], qq = q4[c];
-        dv[4 * c + 0] = fmaf(pu, a.x, dv[4 * c + 0]);
-        dv[4 * c + 1] = fmaf(pu, a.y, dv[4 * c + 1]);
-        dv[4 * c + 2] = fmaf(pu, a.z, dv[4 * c + 2]);
-        dv[4 * c + 3] = fmaf(pu, a.w, dv[4 * c + 3]);
+        dv[4 * c + 0] = fmaf(pw, a.x, dv[4 * c + 0]);
+        dv[4 * c + 1] = fmaf(pw, a.y, dv[4 * c + 1]);
+        dv[4 * c + 2] = fmaf(pw, a.z, dv[4 * c + 2]);
+        dv[4 * c + 3] = fmaf(pw, a.w, dv[4 * c + 3]);
         dk[4 * c + 0] = fmaf(ds, qq.x, dk[4 * c + 0]);
         dk[4 * c + 1] = fmaf(ds, qq.y, dk[4 * c + 1]);
         dk[4 * c + 2] = fmaf(ds, qq.z, dk[4 * c + 2]);

@@ -22,6 +22,7 @@
 //   atomics on data.
 // bwd_finish_kernel: sums the chunk partials of the global query rows (dQ)
 //   and of the global key blocks (dK, dV) in a fixed order.
+#include "dropout.cuh"
 #include "tc_common.cuh"
 
 namespace bb {
@@ -96,6 +97,21 @@ __device__ __forceinline__ void dq_ds_half(const uint32_t (&pv)[32], const uint3
   }
 }
 
+// Dropout form of dq_ds_half: dS = P (m dP - D), m = 1 / keep probability
+// where kept (bit e of keep), 0 where dropped.
+__device__ __forceinline__ void dq_ds_half_drop(const uint32_t (&pv)[32],
+                                                const uint32_t (&dp)[32], float Dr, float sc,
+                                                uint32_t keep, uint32_t* out) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float m0 = ((keep >> e) & 1u) ? sc : 0.f;
+    const float m1 = ((keep >> (e + 1)) & 1u) ? sc : 0.f;
+    const float d0 = __uint_as_float(pv[e]) * fmaf(m0, __uint_as_float(dp[e]), -Dr);
+    const float d1 = __uint_as_float(pv[e + 1]) * fmaf(m1, __uint_as_float(dp[e + 1]), -Dr);
+    out[e >> 1] = pack_bf16(d0, d1);
+  }
+}
+
 struct DqBars {
   uint64_t list_full[2], list_empty[2];
   uint64_t q_full, q_empty;
@@ -103,6 +119,7 @@ struct DqBars {
   uint64_t s_full, s_free, dp_free, p_full, dq_done, dq_full, dq_empty;
 };
 
+template <bool kDrop>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_dq_kernel(const __grid_constant__ BwdArgs ba,
                  const __grid_constant__ CUtensorMap tmQ,
@@ -346,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const ItemMeta im = item_meta_at(a.geo, wi.x, wi.y, p.H, wi.z);
       const int n = L.n;
       const bool rvalid = (im.gvalid >> quarter) & 1;
-      const size_t grow = (size_t)im.bh * p.L + (size_t)(rvalid ? im.t[half] : 0) * kTile + r64;
+      const int tq = (rvalid ? im.t[half] : 0) * kTile + r64;  // query token
+      const size_t grow = (size_t)im.bh * p.L + tq;
       float nl2 = 0.f, Dr = 0.f;
       if (rvalid) {
         nl2 = -p.lse[grow] * kLog2e;
@@ -385,13 +403,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free);
         const uint64_t kb = (m2 && p.key_mask) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
+        const uint64_t db =
+            (kDrop && m2) ? keep_row64(p, im.b, im.h, tq, L.tile[t]) : 0ull;
         if (m2 & 1) dq_p_half(s0, kb, 0, c, nl2, mvl);
         if (m2 & 2) dq_p_half(s1, kb, 32, c, nl2, mvl);
         uint32_t dS[32];
         if (m2 & 1) {
           tmem_ld32(tDP + lane_off, dp);
           tmem_ld_wait();
-          dq_ds_half(s0, dp, Dr, dS);
+          if (kDrop)
+            dq_ds_half_drop(s0, dp, Dr, p.drop_scale, (uint32_t)db, dS);
+          else
+            dq_ds_half(s0, dp, Dr, dS);
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) dS[e] = 0u;
@@ -404,7 +427,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.dp_free);
         if (m2 & 2) {
-          dq_ds_half(s1, dp, Dr, dS + 16);
+          if (kDrop)
+            dq_ds_half_drop(s1, dp, Dr, p.drop_scale, (uint32_t)(db >> 32), dS + 16);
+          else
+            dq_ds_half(s1, dp, Dr, dS + 16);
         } else {
 #pragma unroll
           for (int e = 0; e < 16; ++e) dS[16 + e] = 0u;
@@ -502,7 +528,9 @@ struct KvBars {
 // lengths where they sum over enough query rows (>= 16K) for bf16 products
 // to cost accuracy.  A template flag keeps the low parts out of the shorter
 // lengths' register budget.
-template <bool kSplit>
+// kDrop: seeded attention dropout (P^T kept times 1 / keep probability for
+// dV; dS^T = P^T (m dP^T - D)).
+template <bool kSplit, bool kDrop>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_dkdv_kernel(const __grid_constant__ BwdArgs ba,
                    const __grid_constant__ CUtensorMap tmQ,
@@ -736,6 +764,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
       for (int e = e0; e < e1; ++e) {
         const int mask = (int)(nxt >> 16);
+        const int qtile = (int)(nxt & 0xFFFFu);
         if (e + 1 < e1) nxt = __ldg(walk + e + 1);
         const int st = g % kQStages;
         if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
@@ -754,6 +783,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float* NLs =
             reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
         const float* Ds = NLs + 64;
+        // Dropout keep bits of this lane's key against the tile's 64 query
+        // tokens (m2 is uniform over the warp, as the shuffles need).
+        uint32_t keep[2] = {0u, 0u};
+        if (kDrop && m2)
+          keep_cols64(p, it.b, it.h, (int)(ktok & ~(size_t)31), qtile * kTile, lane, keep[0],
+                      keep[1]);
         // Per query-column half hc (32 columns): read S^T and dP^T, then
         // write P^T and dS^T (bf16 pairs, 16 columns) over the columns just
         // read: high parts at 32 hc, low parts (global items) at 32 hc + 16.
@@ -782,12 +817,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                     add2(make_float2(nls[x], nls[x + 1]), off2));
                 pv[x] = ex2(a.x);
                 pv[x + 1] = ex2(a.y);
-                const float2 d = mul2(
-                    make_float2(pv[x], pv[x + 1]),
-                    sub2(make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
-                         make_float2(dds[x], dds[x + 1])));
-                dv[x] = d.x;
-                dv[x + 1] = d.y;
+                if (kDrop) {
+                  // m = 1 / keep probability where kept, 0 where dropped:
+                  // dS = P (m dP - D), and m P enters dV.
+                  const float m0 = ((keep[hc] >> (e + x)) & 1u) ? p.drop_scale : 0.f;
+                  const float m1 = ((keep[hc] >> (e + x + 1)) & 1u) ? p.drop_scale : 0.f;
+                  dv[x] = pv[x] * fmaf(m0, __uint_as_float(dp[e + x]), -dds[x]);
+                  dv[x + 1] = pv[x + 1] * fmaf(m1, __uint_as_float(dp[e + x + 1]), -dds[x + 1]);
+                  pv[x] *= m0;
+                  pv[x + 1] *= m1;
+                } else {
+                  const float2 d = mul2(
+                      make_float2(pv[x], pv[x + 1]),
+                      sub2(make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
+                           make_float2(dds[x], dds[x + 1])));
+                  dv[x] = d.x;
+                  dv[x + 1] = d.y;
+                }
               }
 #pragma unroll
               for (int x = 0; x < 2; ++x) {
@@ -968,10 +1014,12 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   const size_t smem_dq = 1024 + (4 + 2 * kKvStages) * kTileBytes;
+  const bool drop = p.drop_thr != 0;
+  auto* dq_kernel = drop ? tc_dq_kernel<true> : tc_dq_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(
-      tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
+      dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
   if (e != cudaSuccess) return e;
-  tc_dq_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_dq, s>>>(
+  dq_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_dq, s>>>(
       ba, tm.q, tm.k, tm.v, tm.dout);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1002,7 +1050,10 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     bk.kloc0 = parts[i].loc0;
     bk.kitems = p.B * p.H * parts[i].per_bh;
     bk.kctr = p.sched + 1 + i;  // sched[0]: dQ
-    auto* kv_kernel = parts[i].split ? tc_dkdv_kernel<true> : tc_dkdv_kernel<false>;
+    auto* kv_kernel = parts[i].split ? (drop ? tc_dkdv_kernel<true, true>
+                                             : tc_dkdv_kernel<true, false>)
+                                     : (drop ? tc_dkdv_kernel<false, true>
+                                             : tc_dkdv_kernel<false, false>);
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);
     if (e != cudaSuccess) return e;

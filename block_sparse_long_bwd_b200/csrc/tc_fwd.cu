@@ -19,6 +19,7 @@
 // row: load S, fold scale, masks and the lazy running max, write P (bf16
 // pairs) and rescale O in TMEM when the max moves; at the end of an item
 // they normalise O and store it through shared memory with a TMA store.
+#include "dropout.cuh"
 #include "tc_common.cuh"
 
 namespace bb {
@@ -63,6 +64,9 @@ __device__ __forceinline__ float max64(const float* z) {
   return fmax3(a, b, fmaxf(n[6], n[7]));
 }
 
+// kDrop: seeded attention dropout on the probabilities that enter P V (the
+// row sums, hence the lse, stay those of the undropped softmax).
+template <bool kDrop>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
@@ -288,6 +292,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       const ItemMeta im = item_meta_at(a.geo, wi.x, wi.y, p.H, wi.z);
       const int n = L.n;
       float m = -INFINITY, l = 0.f;
+      // Query token of this row (dropout counters; any row when invalid).
+      const int tq = (((im.gvalid >> quarter) & 1) ? im.t[half] : 0) * kTile + (row & 63);
       bool ok = true;
       for (int t = 0; t < n; ++t) {
         const uint32_t uu = u + t;
@@ -377,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int e = 0; e < 4; ++e) sum2[e] = make_float2(0.f, 0.f);
           const float cc = scaled ? 1.f : c;
           const float2 cc2 = make_float2(cc, cc), nm2 = make_float2(-m, -m);
+          const uint64_t db = kDrop ? keep_row64(p, im.b, im.h, tq, L.tile[t]) : 0ull;
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t Ph[16];
@@ -385,7 +392,14 @@ __global__ void __launch_bounds__(kThreads, 2)
               const float2 a = fma2(make_float2(z[32 * hh + e], z[32 * hh + e + 1]), cc2, nm2);
               const float2 pp = make_float2(ex2(a.x), ex2(a.y));
               sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pp);
-              Ph[e >> 1] = pack_bf16(pp.x, pp.y);
+              if (kDrop) {
+                // Kept probabilities times 1 / keep probability, dropped 0.
+                const int col = 32 * hh + e;
+                Ph[e >> 1] = pack_bf16(((db >> col) & 1ull) ? pp.x * p.drop_scale : 0.f,
+                                       ((db >> (col + 1)) & 1ull) ? pp.y * p.drop_scale : 0.f);
+              } else {
+                Ph[e >> 1] = pack_bf16(pp.x, pp.y);
+              }
             }
             tmem_st16(tP + 16 * hh, Ph);
           }
@@ -542,14 +556,15 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
   const PairArgs a = make_pair_args(p);
   const size_t smem = 1024 + (2 * 2 + 2 * kNST) * kTileBytes;
+  auto* kernel = p.drop_thr ? tc_fwd_kernel<true> : tc_fwd_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(
-      tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = min(a.items, 2 * sms);
-  tc_fwd_kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v, tm.out32);
+  kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v, tm.out32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = marks->mark(s);

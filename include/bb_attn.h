@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define BB_ABI_VERSION 1
+#define BB_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define BB_API __attribute__((visibility("default")))
@@ -69,12 +69,31 @@ typedef enum { BB_F32 = 0, BB_BF16 = 1 } bb_dtype;
  * scale == 0 selects 1/sqrt(d) (key_dim = hidden / heads, as the pages'
  * layer sets it).  mask_value == 0 selects -10000, the pages' offset for
  * masked positions.  The scale multiplies <q, k> before the offset is added;
- * the offset is not scaled. */
+ * the offset is not scaled.
+ *
+ * dropout is the attention-dropout rate in [0, 1) ([gitcode page] sections
+ * "BigBirdEncoder 的关键参数", attention_dropout_rate, and "梯度检查点的实现方式",
+ * which asks for stateless seeded dropout so a recomputation draws the same
+ * noise).  It acts on the attended softmax probabilities: kept ones are
+ * multiplied by 1 / keep probability, dropped ones by 0; the lse output stays
+ * that of the undropped softmax.  The rate is rounded to the nearest multiple
+ * of 1/256 (thr = floor(256 rate + 1/2), keep probability (256 - thr) / 256);
+ * a rate that rounds to 0 disables dropout, one that rounds to 1 is
+ * BB_ERR_INVALID.  The keep decision of element (b, h, query token t, key
+ * token u) is a pure function of dropout_seed and (b, h, t, u): Philox4x32-10
+ * (Salmon, Moraes, Dror and Shaw, SC 2011) with counter words
+ * (u >> 4, t, h, b) and key words (seed mod 2^32, seed >> 32) gives 16 bytes,
+ * little-endian from its four output words in order, for key tokens
+ * 16 (u >> 4) .. 16 (u >> 4) + 15; byte u & 15 keeps the element when it is
+ * >= thr.  The backward must be called with the forward's dropout and
+ * dropout_seed. */
 typedef struct {
   int B, H, L, d, block_size, r;
   int dtype;
   float scale;
   float mask_value;
+  float dropout;
+  uint64_t dropout_seed;
 } bb_attn_desc;
 
 /* Random block table ([gitcode page] section "随机块掩码是如何生成的": per

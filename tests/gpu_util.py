@@ -14,13 +14,15 @@ ATOL = {"f32": 2e-5, "bf16": 1e-2}
 
 
 def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
-            scale=0.0, mask_value=0.0, table=None):
+            scale=0.0, mask_value=0.0, table=None, dropout=0.0,
+            dropout_seed=0):
     """Forward (and backward) through the C ABI; returns CPU tensors."""
     dev = torch.device("cuda")
     B, H, L = cfg["B"], cfg["H"], cfg["L"]
     att = bb.Attention(B, H, L, cfg["block_size"], cfg["r"],
                        synth.torch_dtype(cfg["dtype"]), d=cfg["d"],
-                       seed=table_seed, scale=scale, mask_value=mask_value)
+                       seed=table_seed, scale=scale, mask_value=mask_value,
+                       dropout=dropout, dropout_seed=dropout_seed)
     if table is not None:
         att.table_host = torch.as_tensor(table, dtype=torch.int32)
         att.table = att.table_host.to(dev)
@@ -39,20 +41,36 @@ def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
                  else v_) for k_, v_ in res.items()}
 
 
+class _SliceDropout(oracle.Dropout):
+    """The oracle's dropout for a (b, h) slice run as a 1 x 1 problem: the
+    keep rule is drawn at the slice's own (b, h)."""
+
+    def __init__(self, rate, seed, b, h):
+        super().__init__(rate, seed)
+        self.b0, self.h0 = b, h
+
+    def factors(self, b, h, rows, cols):
+        return super().factors(self.b0 + b, self.h0 + h, rows, cols)
+
+
 def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
-                 mask_value=oracle.DEFAULT_MASK_VALUE):
-    """Oracle on the (b, h) slice: rows of one (b, h) depend on nothing else."""
+                 mask_value=oracle.DEFAULT_MASK_VALUE, dropout=0.0,
+                 dropout_seed=0):
+    """Oracle on the (b, h) slice: rows of one (b, h) depend on nothing else
+    (the dropout decisions are drawn at the slice's own b and h)."""
     sl = lambda x: x[b:b + 1, h:h + 1].double().numpy()
     km = inp["key_mask"]
     km = None if km is None else km[b:b + 1].numpy()
     tab = np.asarray(table)[h:h + 1]
+    drop = _SliceDropout(dropout, dropout_seed, b, h) if dropout else None
     o, lse = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), km, tab,
-                            cfg["block_size"], scale, mask_value)
+                            cfg["block_size"], scale, mask_value, drop)
     res = {"out": o[0, 0], "lse": lse[0, 0]}
     if backward:
         dq, dk, dv = oracle.backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
                                      sl(inp["dout"]), km, tab,
-                                     cfg["block_size"], scale, mask_value)
+                                     cfg["block_size"], scale, mask_value,
+                                     drop)
         res.update(dq=dq[0, 0], dk=dk[0, 0], dv=dv[0, 0])
     return res
 

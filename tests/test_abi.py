@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
     assert "bb_attn_fwd" in names and "bb_attn_bwd" in names
     for name in names:
         assert hasattr(lib, name), name
-    assert bb.bb_abi_version() == 1
+    assert bb.bb_abi_version() == 2
 
 
 @pytest.mark.parametrize("seed,H,nb,r", [
@@ -75,6 +75,9 @@ def test_workspace_size_and_validation():
         (dict(L=500), -1), (dict(B=0), -1), (dict(r=-1), -1),
         (dict(dtype=7), -1), (dict(d=128), -2), (dict(block_size=16), -2),
         (dict(r=33), -2), (dict(L=64 * 8193), -2),
+        # dropout outside [0, 1), NaN, or a rate that rounds to 1 (256/256)
+        (dict(dropout=1.0), -1), (dict(dropout=-0.1), -1),
+        (dict(dropout=float("nan")), -1), (dict(dropout=255.6 / 256), -1),
     ]
     lib = bb.lib()
     for kw, code in bad:
@@ -82,6 +85,9 @@ def test_workspace_size_and_validation():
         got = lib.bb_attn_workspace_size(ctypes.byref(_desc(**kw)), 0,
                                          ctypes.byref(n))
         assert got == code, (kw, got)
+    for rate in (0.1, 0.5, 255.4 / 256):  # valid rates, any seed
+        assert bb.bb_attn_workspace_size(
+            _desc(dropout=rate, dropout_seed=2**64 - 1), 1) == n1
     n = ctypes.c_size_t(0)
     assert lib.bb_attn_workspace_size(None, 0, ctypes.byref(n)) == -1
     assert lib.bb_attn_workspace_size(ctypes.byref(_desc()), 2,

@@ -1,7 +1,7 @@
 """Benchmark of the block-sparse attention hot path (forward + backward).
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                [--workload NAME]
+                [--workload NAME] [--dropout RATE [--dropout-seed S]]
 
 One step = one forward + backward pass of the whole hot path over one batch
 of the named synthetic workload (default: BigBird-large attention layer at
@@ -68,6 +68,10 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=10)
+    # Seeded attention dropout on the attended probabilities (rate in [0, 1);
+    # 0, the default, is the plain operation the headline line times).
+    ap.add_argument("--dropout", type=float, default=0.0)
+    ap.add_argument("--dropout-seed", type=int, default=0)
     # Profiling runs (ncu) only: leave out the end-to-end and CPU legs.
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
@@ -273,7 +277,8 @@ def run_ours(args, world, rank, local):
 
     inp = synth.make_inputs(cfg, with_grad=backward)
     att = bb.Attention(B, H, L, bs, r, dt, d=cfg["d"], seed=synth.TABLE_SEED,
-                       device=dev)
+                       device=dev, dropout=args.dropout,
+                       dropout_seed=args.dropout_seed)
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     g = inp["dout"].to(dev) if backward else None
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
@@ -383,7 +388,7 @@ def run_ours(args, world, rank, local):
         peak, how = peaks["hbm_gbs"], "HBM copy"
     traffic = None
     tr = NCU_TRAFFIC.get(dom)
-    if (tr is not None and args.workload == tr[3] and
+    if (tr is not None and args.workload == tr[3] and not args.dropout and
             tr[1] == src_hash(os.path.join(ROOT, "block_sparse_long_bwd_b200",
                                            "csrc", tr[2]))):
         traffic = tr[0]
@@ -418,6 +423,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": args.workload, "B": B, "H": H, "L": L,
                    "block_size": bs, "d": cfg["d"], "r": r,
                    "mask": cfg["mask"], "passes": cfg["passes"],
+                   "dropout": args.dropout,
                    "global_batch": B * world, "seq_len": L,
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (256 MiB write, untimed)"},
@@ -434,7 +440,8 @@ def run_ours(args, world, rank, local):
     }
     if rank == 0:
         result["cpu_baseline"] = None if args.skip_cpu else cpu_baseline(
-            cfg, att.table_host.numpy(), backward, budget_s=12.0)
+            cfg, att.table_host.numpy(), backward, budget_s=12.0,
+            dropout=(args.dropout, args.dropout_seed))
         print(json.dumps(result), flush=True)
 
 
@@ -545,10 +552,12 @@ def run_e2e(args, cfg, att, inp, dev, backward, world):
                       "step s+1 in and s-1 out overlap the compute of s)"}
 
 
-def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None):
+def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None,
+                 dropout=(0.0, 0)):
     """The fp64 oracle, as it stands, on (b, h) slices of the workload until
     the time budget is spent; scaled to tokens/s of the whole workload
-    (each slice is 1/(B*H) of it)."""
+    (each slice is 1/(B*H) of it).  dropout: (rate, seed) of the timed
+    call."""
     import oracle
     try:
         from threadpoolctl import threadpool_info
@@ -567,13 +576,15 @@ def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None):
                                     batch_slice=slice(b, b + 1))
             km = None if inp["key_mask"] is None else inp["key_mask"].numpy()
             for h in range(H):
+                drop = (oracle.Dropout(dropout[0], dropout[1], b0=b, h0=h)
+                        if dropout[0] else None)
                 t0 = time.perf_counter()
                 oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
-                               km, table[h:h + 1], bs)
+                               km, table[h:h + 1], bs, dropout=drop)
                 if backward:
                     oracle.backward(f(inp["q"], h), f(inp["k"], h),
                                     f(inp["v"], h), f(inp["dout"], h), km,
-                                    table[h:h + 1], bs)
+                                    table[h:h + 1], bs, dropout=drop)
                 t_used += time.perf_counter() - t0
                 done += 1
                 if t_used >= budget_s or (max_slices and done >= max_slices):
@@ -604,11 +615,14 @@ def run_reference(args, world, rank):
 
     def step(s):
         h = s % H
+        drop = (oracle.Dropout(args.dropout, args.dropout_seed, b0=0, h0=h)
+                if args.dropout else None)
         oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), km,
-                       table[h:h + 1], bs)
+                       table[h:h + 1], bs, dropout=drop)
         if backward:
             oracle.backward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
-                            f(inp["dout"], h), km, table[h:h + 1], bs)
+                            f(inp["dout"], h), km, table[h:h + 1], bs,
+                            dropout=drop)
 
     for s in range(args.warmup):
         step(s)
@@ -633,6 +647,7 @@ def run_reference(args, world, rank):
         "dtype": "f64", "data": "synthetic (seeded N(0,1) inputs)",
         "config": {"workload": args.workload, "B": B, "H": H, "L": L,
                    "block_size": bs, "d": cfg["d"], "r": r,
+                   "dropout": args.dropout,
                    "global_batch": B, "seq_len": L},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                          "cores": cores, "kind": "oracle", "sample": sample},

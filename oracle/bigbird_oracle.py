@@ -227,17 +227,23 @@ def dropout_keep(seed, b, h, rows, cols, rate):
 
 
 class Dropout:
-    """Attention dropout of one call: rate in [0, 1) and a 64-bit seed."""
+    """Attention dropout of one call: rate in [0, 1) and a 64-bit seed.
 
-    def __init__(self, rate, seed):
+    b0, h0: index offsets for a (b, h) slice computed as a problem of its
+    own, so that its decisions are those of batch b0 + b, head h0 + h of the
+    whole call."""
+
+    def __init__(self, rate, seed, b0=0, h0=0):
         dropout_threshold(rate)  # validates
         self.rate = float(rate)
         self.seed = int(seed) & _MASK64
+        self.b0, self.h0 = int(b0), int(h0)
 
     def factors(self, b, h, rows, cols):
         """[len(rows), len(cols)] multipliers of the probabilities: the
         scale where kept, 0 where dropped."""
-        keep = dropout_keep(self.seed, b, h, rows, cols, self.rate)
+        keep = dropout_keep(self.seed, self.b0 + b, self.h0 + h, rows, cols,
+                            self.rate)
         return np.where(keep, dropout_scale(self.rate), 0.0)
 
 

@@ -41,18 +41,6 @@ def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
                  else v_) for k_, v_ in res.items()}
 
 
-class _SliceDropout(oracle.Dropout):
-    """The oracle's dropout for a (b, h) slice run as a 1 x 1 problem: the
-    keep rule is drawn at the slice's own (b, h)."""
-
-    def __init__(self, rate, seed, b, h):
-        super().__init__(rate, seed)
-        self.b0, self.h0 = b, h
-
-    def factors(self, b, h, rows, cols):
-        return super().factors(self.b0 + b, self.h0 + h, rows, cols)
-
-
 def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
                  mask_value=oracle.DEFAULT_MASK_VALUE, dropout=0.0,
                  dropout_seed=0):
@@ -62,7 +50,8 @@ def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
     km = inp["key_mask"]
     km = None if km is None else km[b:b + 1].numpy()
     tab = np.asarray(table)[h:h + 1]
-    drop = _SliceDropout(dropout, dropout_seed, b, h) if dropout else None
+    drop = (oracle.Dropout(dropout, dropout_seed, b0=b, h0=h)
+            if dropout else None)
     o, lse = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), km, tab,
                             cfg["block_size"], scale, mask_value, drop)
     res = {"out": o[0, 0], "lse": lse[0, 0]}

@@ -241,3 +241,24 @@ def test_dropout_output_is_unbiased_over_seeds():
     mean = acc / n
     se = np.sqrt(np.maximum(sq / n - mean * mean, 0) / n) + 1e-12
     assert np.max(np.abs(mean - o0) / se) < 6.0
+
+
+def test_slice_offsets_reproduce_the_whole_call():
+    """A (b, h) slice run as its own problem with offsets (b, h) draws the
+    decisions of the whole call's batch b, head h."""
+    q, k, v, dout, km, table = _case(48, 2, 3, 6, 4, 8, 2, True, False)
+    whole = oracle.Dropout(0.3, 77)
+    o, _ = oracle.forward(q, k, v, km, table, 4, dropout=whole)
+    g = oracle.backward(q, k, v, dout, km, table, 4, dropout=whole)
+    for b in range(2):
+        for h in range(3):
+            sl = lambda x: x[b:b + 1, h:h + 1]
+            part = oracle.Dropout(0.3, 77, b0=b, h0=h)
+            kmb = km[b:b + 1]
+            os_, _ = oracle.forward(sl(q), sl(k), sl(v), kmb, table[h:h + 1],
+                                    4, dropout=part)
+            np.testing.assert_array_equal(os_[0, 0], o[b, h])
+            gs = oracle.backward(sl(q), sl(k), sl(v), sl(dout), kmb,
+                                 table[h:h + 1], 4, dropout=part)
+            for a, c in zip(gs, g):
+                np.testing.assert_array_equal(a[0, 0], c[b, h])

@@ -56,6 +56,9 @@ def lib():
         L.bb_rand_attn_build.argtypes = [ctypes.c_uint64, ctypes.c_int,
                                          ctypes.c_int, ctypes.c_int, _P]
         L.bb_rand_attn_build.restype = ctypes.c_int
+        L.bb_rand_attn_build_ex.argtypes = [ctypes.c_uint64] + [
+            ctypes.c_int] * 5 + [_P]
+        L.bb_rand_attn_build_ex.restype = ctypes.c_int
         L.bb_attn_workspace_size.argtypes = [
             ctypes.POINTER(bb_attn_desc), ctypes.c_int,
             ctypes.POINTER(ctypes.c_size_t)]
@@ -118,6 +121,19 @@ def bb_rand_attn_build(seed, heads, num_blocks, r):
     _check(lib().bb_rand_attn_build(seed, heads, num_blocks, r,
                                     out.data_ptr() if out.numel() else None),
            "bb_rand_attn_build")
+    return out
+
+
+def bb_rand_attn_build_ex(seed, heads, num_blocks, r, max_blocks=0,
+                          last_block=0):
+    """int32 CPU tensor [heads, num_blocks, r] drawn for a table of
+    max_blocks blocks with random ids capped below last_block (see
+    include/bb_attn.h)."""
+    out = torch.empty((heads, num_blocks, r), dtype=torch.int32)
+    _check(lib().bb_rand_attn_build_ex(seed, heads, num_blocks, r, max_blocks,
+                                       last_block,
+                                       out.data_ptr() if out.numel() else None),
+           "bb_rand_attn_build_ex")
     return out
 
 
@@ -249,12 +265,20 @@ class Attention:
 
     def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
                  device="cuda", scale=0.0, mask_value=0.0, dropout=0.0,
-                 dropout_seed=0):
+                 dropout_seed=0, max_rand_mask_length=0, last_idx=0):
+        """max_rand_mask_length, last_idx (tokens; 0 = off): the pages'
+        layer options for the random table (drawn for the maximum length,
+        random blocks before token last_idx); seed: the layer index there."""
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
                               mask_value, dropout, dropout_seed)
         self.dtype = dtype
         nb = L // block_size
-        self.table_host = bb_rand_attn_build(seed, H, nb, r)
+        if max_rand_mask_length or last_idx:
+            self.table_host = bb_rand_attn_build_ex(
+                seed, H, nb, r, max_rand_mask_length // block_size,
+                last_idx // block_size)
+        else:
+            self.table_host = bb_rand_attn_build(seed, H, nb, r)
         self.table = self.table_host.to(device)
         self.ws_fwd = torch.empty(bb_attn_workspace_size(self.desc, 0),
                                   dtype=torch.uint8, device=device)

@@ -156,22 +156,28 @@ const char* bb_status_str(int status) {
   }
 }
 
-int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
-                       int32_t* out_host) {
-  if (heads < 0 || num_blocks < 0 || r < 0) return BB_ERR_INVALID;
+int bb_rand_attn_build_ex(uint64_t seed, int heads, int num_blocks, int r,
+                          int max_blocks, int last_block, int32_t* out_host) {
+  if (heads < 0 || num_blocks < 0 || r < 0 || max_blocks < 0 || last_block < 0)
+    return BB_ERR_INVALID;
+  // The rows are drawn as for a table of nbb blocks; the first num_blocks
+  // rows are kept.
+  const int nbb = max_blocks ? max_blocks : num_blocks;
+  if (nbb < num_blocks) return BB_ERR_INVALID;
   const size_t n = (size_t)heads * num_blocks * r;
   if (n == 0) return BB_OK;
   if (!out_host) return BB_ERR_INVALID;
   std::vector<int32_t> cand;
-  cand.reserve(num_blocks);
+  cand.reserve(nbb);
   for (int h = 0; h < heads; ++h) {
     for (int i = 0; i < num_blocks; ++i) {
       int32_t* row = out_host + ((size_t)h * num_blocks + i) * r;
       for (int a = 0; a < r; ++a) row[a] = -1;
       if (i == 0 || i == num_blocks - 1) continue;
       cand.clear();
-      for (int j = 1; j <= num_blocks - 2; ++j)
-        if (j < i - 1 || j > i + 1) cand.push_back(j);
+      for (int j = 1; j <= nbb - 2; ++j)
+        if ((j < i - 1 || j > i + 1) && (last_block == 0 || j < last_block))
+          cand.push_back(j);
       const int m = (int)cand.size();
       const int r_eff = r < m ? r : m;
       SplitMix64 g{seed ^ (((uint64_t)(uint32_t)h << 32) | (uint64_t)(uint32_t)i)};
@@ -180,11 +186,21 @@ int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
         const int t = a + (int)(u % (uint64_t)(m - a));
         std::swap(cand[a], cand[t]);
       }
-      std::sort(cand.begin(), cand.begin() + r_eff);
-      for (int a = 0; a < r_eff; ++a) row[a] = cand[a];
+      // Keep the ids of this table's middle blocks: one at or past its last
+      // (global) block is dropped, which leaves the attended set unchanged
+      // or removes a block the shorter sequence does not have.
+      int k = 0;
+      for (int a = 0; a < r_eff; ++a)
+        if (cand[a] <= num_blocks - 2) row[k++] = cand[a];
+      std::sort(row, row + k);
     }
   }
   return BB_OK;
+}
+
+int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
+                       int32_t* out_host) {
+  return bb_rand_attn_build_ex(seed, heads, num_blocks, r, 0, 0, out_host);
 }
 
 int bb_attn_workspace_size(const bb_attn_desc* desc, int pass, size_t* bytes) {

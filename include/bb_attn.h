@@ -111,6 +111,32 @@ typedef struct {
 BB_API int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
                        int32_t* out_host);
 
+/* Random block table with the options of the pages' layer ([gitcode page]
+ * section "随机块掩码是如何生成的": the table is fixed per head when the layer
+ * is built, for its maximum length, with random blocks capped by
+ * last_idx = 1024 tokens, and the first L / block_size - 2 middle rows are
+ * used at run time; section "网络实现：从配置文件到编码器": the maximum
+ * length is max_rand_mask_length = max_position_embeddings and the seed is
+ * the layer index).
+ *   max_blocks  rows are drawn as for a table of max_blocks blocks
+ *               (max_rand_mask_length / block_size; >= num_blocks), and the
+ *               first num_blocks rows are returned; 0 = num_blocks
+ *   last_block  random candidates are restricted to ids < last_block
+ *               (last_idx / block_size); 0 = no cap
+ * Row i (0 < i < num_blocks - 1) draws, exactly as bb_rand_attn_build does
+ * (same SplitMix64 stream and partial Fisher-Yates shuffle), r_eff =
+ * min(r, |cand(i)|) ids from cand(i) = {j in [1, max_blocks - 2] :
+ * |j - i| > 1, and j < last_block when last_block > 0}, then keeps those
+ * <= num_blocks - 2, sorted
+ * ascending, with -1 in the remaining slots.  Dropping an id past the
+ * shorter table's middle blocks leaves the attended set unchanged (its last
+ * block is global) or removes a block the sequence does not have.  With
+ * max_blocks = 0 and last_block = 0 the result equals bb_rand_attn_build.
+ * Returns BB_ERR_INVALID for a negative argument, max_blocks < num_blocks,
+ * or a NULL out_host (unless the table is empty).  Host only. */
+BB_API int bb_rand_attn_build_ex(uint64_t seed, int heads, int num_blocks, int r,
+                                 int max_blocks, int last_block, int32_t* out_host);
+
 /* Bytes of device workspace bb_attn_fwd (pass 0) or bb_attn_bwd (pass 1)
  * needs for `desc`; written to *bytes.  Host only. */
 BB_API int bb_attn_workspace_size(const bb_attn_desc* desc, int pass, size_t* bytes);

@@ -44,6 +44,14 @@ Readings taken where the pages are silent (each listed in the design doc):
   Fisher-Yates shuffle draws r_eff = min(r, |cand|) of them; the chosen ids
   are written sorted ascending, unused slots and rows 0 and nb-1 hold -1.
 
+* The pages' layer draws its table once for the maximum length
+  (max_rand_mask_length = max_position_embeddings), with random blocks
+  restricted to tokens before last_idx = 1024, and uses its first rows for
+  a shorter sequence ([GC] 随机块掩码是如何生成的).  Both are options of
+  rand_table (off by default): rows drawn for max_blocks blocks with ids
+  below last_block; a row keeps the drawn ids that are middle blocks of the
+  shorter table (an id at its last block is global already, one past it
+  does not exist).
 * Attention dropout ([GC] sections "BigBirdEncoder 的关键参数", which lists
   attention_dropout_rate = 0.1, and "梯度检查点的实现方式", which requires
   stateless, seeded dropout so a recomputed forward draws the same noise):
@@ -107,21 +115,34 @@ def random_candidates(i, num_blocks):
     return [j for j in range(1, num_blocks - 1) if abs(j - i) > 1]
 
 
-def rand_table(seed, heads, num_blocks, r):
-    """int32 [heads, num_blocks, r] random block table (spec in module doc)."""
-    if heads < 0 or num_blocks < 0 or r < 0:
+def rand_table(seed, heads, num_blocks, r, max_blocks=0, last_block=0):
+    """int32 [heads, num_blocks, r] random block table (spec in module doc).
+
+    max_blocks, last_block (0 = off): the options of the pages' layer ([GC]
+    随机块掩码是如何生成的: the table is drawn once for the maximum length,
+    with random blocks before token last_idx, and its first rows are used
+    for a shorter sequence).  Row i is drawn as in a table of max_blocks
+    blocks whose candidates are also below last_block; it keeps the drawn
+    ids that are middle blocks of this table (<= num_blocks - 2), sorted."""
+    if heads < 0 or num_blocks < 0 or r < 0 or max_blocks < 0 or last_block < 0:
         raise ValueError("negative size")
+    nbb = max_blocks or num_blocks
+    if nbb < num_blocks:
+        raise ValueError("max_blocks below num_blocks")
     table = np.full((heads, num_blocks, r), -1, dtype=np.int32)
     for h in range(heads):
         for i in range(1, num_blocks - 1):
-            cand = random_candidates(i, num_blocks)
+            cand = random_candidates(i, nbb)
+            if last_block:
+                cand = [j for j in cand if j < last_block]
             r_eff = min(r, len(cand))
             rng = SplitMix64((int(seed) ^ ((h << 32) | i)) & _MASK64)
             for kk in range(r_eff):
                 u = rng.next()
                 t = kk + u % (len(cand) - kk)
                 cand[kk], cand[t] = cand[t], cand[kk]
-            table[h, i, :r_eff] = sorted(cand[:r_eff])
+            kept = sorted(j for j in cand[:r_eff] if j <= num_blocks - 2)
+            table[h, i, :len(kept)] = kept
     return table
 
 

@@ -49,6 +49,28 @@ def test_rand_table_bit_exact_vs_oracle(seed, H, nb, r):
     assert np.array_equal(got, want)
 
 
+@pytest.mark.parametrize("seed,H,nb,r,mx,last", [
+    (0, 12, 16, 3, 64, 16), (3, 12, 32, 3, 64, 16), (11, 12, 64, 3, 64, 16),
+    (5, 4, 40, 6, 41, 0), (7, 4, 33, 9, 0, 12), (2**64 - 1, 2, 8, 3, 8, 3),
+    (1, 3, 1, 3, 5, 0), (1, 3, 3, 2, 64, 0)])
+def test_rand_table_layer_options_bit_exact_vs_oracle(seed, H, nb, r, mx, last):
+    got = bb.bb_rand_attn_build_ex(seed, H, nb, r, mx, last).numpy()
+    want = oracle.rand_table(seed, H, nb, r, max_blocks=mx, last_block=last)
+    assert np.array_equal(got, want)
+
+
+def test_rand_table_layer_options_off_equal_the_base_call():
+    assert np.array_equal(bb.bb_rand_attn_build_ex(4, 3, 48, 3, 0, 0).numpy(),
+                          bb.bb_rand_attn_build(4, 3, 48, 3).numpy())
+    lib = bb.lib()
+    buf = (ctypes.c_int32 * 64)()
+    assert lib.bb_rand_attn_build_ex(0, 1, 32, 2, 16, 0, buf) == -1  # mx < nb
+    assert lib.bb_rand_attn_build_ex(0, 1, 32, 2, 0, -1, buf) == -1
+    assert lib.bb_rand_attn_build_ex(0, 1, 32, 2, -1, 0, buf) == -1
+    assert lib.bb_rand_attn_build_ex(0, 1, 32, 2, 64, 16, None) == -1
+    assert lib.bb_rand_attn_build_ex(0, 0, 32, 2, 64, 16, None) == 0  # empty
+
+
 def test_rand_table_errors():
     lib = bb.lib()
     assert lib.bb_rand_attn_build(0, -1, 4, 3, None) == -1

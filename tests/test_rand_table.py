@@ -68,3 +68,82 @@ def test_table_uniform_chi_square():
     assert obs.sum() == 6000 * r
     p = stats.chisquare(obs).pvalue
     assert p > 1e-3, p
+
+
+# ---- the layer's table options: drawn for the maximum length, capped ----
+
+def test_layer_options_off_is_the_base_table():
+    for nb, r in ((16, 3), (33, 9), (5, 2)):
+        assert np.array_equal(oracle.rand_table(9, 3, nb, r, 0, 0),
+                              oracle.rand_table(9, 3, nb, r))
+        assert np.array_equal(oracle.rand_table(9, 3, nb, r, nb, 0),
+                              oracle.rand_table(9, 3, nb, r))
+
+
+@pytest.mark.parametrize("nb,nbb,r", [(16, 64, 3), (32, 64, 3), (3, 64, 2),
+                                      (40, 41, 6), (64, 64, 3)])
+def test_truncation_keeps_the_prefix_of_the_full_build(nb, nbb, r):
+    """Rows of a table drawn for nbb blocks and kept for nb are the rows of
+    the full nbb-block table restricted to this table's middle blocks."""
+    full = oracle.rand_table(3, 4, nbb, r)
+    part = oracle.rand_table(3, 4, nb, r, max_blocks=nbb)
+    for h in range(4):
+        assert (part[h, 0] == -1).all() and (part[h, nb - 1] == -1).all()
+        for i in range(1, nb - 1):
+            want = sorted(j for j in full[h, i].tolist()
+                          if 0 <= j <= nb - 2)
+            got = part[h, i]
+            assert got[:len(want)].tolist() == want
+            assert (got[len(want):] == -1).all()
+
+
+@pytest.mark.parametrize("nb,last,r", [(64, 16, 3), (64, 16, 6), (32, 4, 3),
+                                       (64, 1, 3), (20, 30, 2)])
+def test_cap_keeps_random_blocks_below_last_block(nb, last, r):
+    t = oracle.rand_table(11, 3, nb, r, last_block=last)
+    for h in range(3):
+        for i in range(1, nb - 1):
+            cand = [j for j in range(1, nb - 1) if abs(j - i) > 1 and j < last]
+            r_eff = min(r, len(cand))
+            row = t[h, i]
+            chosen = row[:r_eff].tolist()
+            assert (row[r_eff:] == -1).all()
+            assert len(set(chosen)) == r_eff and all(c in cand for c in chosen)
+            assert chosen == sorted(chosen)
+
+
+def test_pages_configuration_stays_inside_short_sequences():
+    """The pages' layer: block 64, table for 4096 tokens, random blocks
+    before token 1024, seed = layer index; every kept id is a middle block
+    of the running sequence, below 16, off the row's window."""
+    for layer in range(12):
+        for L in (1024, 2048, 4096):
+            nb = L // 64
+            t = oracle.rand_table(layer, 12, nb, 3, max_blocks=64,
+                                  last_block=16)
+            ids = t[t >= 0]
+            assert ids.min() >= 1 and ids.max() <= min(15, nb - 2)
+            for i in range(1, nb - 1):
+                for j in t[:, i][t[:, i] >= 0].tolist():
+                    assert abs(j - i) > 1
+
+
+def test_capped_choice_uniform_chi_square():
+    """Over many seeds a capped row chooses each allowed candidate equally
+    often."""
+    nb, i, r, last = 64, 30, 3, 16
+    cand = [j for j in range(1, nb - 1) if abs(j - i) > 1 and j < last]
+    counts = dict.fromkeys(cand, 0)
+    n = 3000
+    for s in range(n):
+        for j in oracle.rand_table(s, 1, nb, r, last_block=last)[0, i]:
+            counts[int(j)] += 1
+    assert sum(counts.values()) == n * r
+    assert stats.chisquare(list(counts.values())).pvalue > 1e-4
+
+
+def test_layer_options_reject_bad_arguments():
+    with pytest.raises(ValueError):
+        oracle.rand_table(0, 1, 32, 3, max_blocks=16)
+    with pytest.raises(ValueError):
+        oracle.rand_table(0, 1, 32, 3, last_block=-1)

@@ -34,8 +34,11 @@ Readings taken where the pages are silent (each listed in the design doc):
   applied before the offset; the offset is not scaled.  Blocks outside A(i)
   are absent (as if -inf), masked keys inside A(i) get the finite offset.
 * lse_t = ln sum_u exp(s_tu) over the attended keys (natural log).
-* The key mask is key-side only: query rows of padding are computed like
-  any other row.
+* The key mask is key-side only by default: query rows of padding are
+  computed like any other row.  The optional query_mask (the from-side mask
+  BigBirdMasks derives from the same input mask, [GC]
+  随机块掩码是如何生成的) zeroes the output rows of padding tokens, so they
+  pass no gradient.
 * The random table follows this library's own specification (the pages'
   NumPy stream is not given): per head h and middle row i, the candidates are
   the ascending block ids j in [1, nb-2] with |j - i| > 1; a SplitMix64
@@ -76,7 +79,8 @@ against the published SplitMix64 outputs and the table's defining
 properties; tests/test_dropout_oracle.py checks the dropout generator
 against the published Philox4x32-10 known-answer vectors and the dropped
 forward and backward against dense torch fp64 with autograd and finite
-differences.
+differences; tests/test_query_mask_oracle.py does the same for the query
+mask.
 """
 
 import math
@@ -307,14 +311,25 @@ def block_probs(q, k, key_mask, table, block_size, b, h, i, scale=None,
     return cols, e / z, (m + np.log(z))[:, 0]
 
 
+def _query_factors(query_mask, B, L):
+    """[B, L] 1.0 for real query tokens, 0.0 for padding (None: all real)."""
+    if query_mask is None:
+        return np.ones((B, L))
+    return (np.asarray(query_mask).reshape(B, L) != 0).astype(np.float64)
+
+
 def forward(q, k, v, key_mask, table, block_size, scale=None,
-            mask_value=DEFAULT_MASK_VALUE, dropout=None):
+            mask_value=DEFAULT_MASK_VALUE, dropout=None, query_mask=None):
     """Block-sparse attention forward: (o [B,H,L,d], lse [B,H,L]) in fp64.
 
     q, k, v: [B, H, L, d] (any float dtype, read as fp64); key_mask: None or
     [B, L] with nonzero = attend; table: int [H, nb, r].  dropout: None or a
     Dropout; o then sums the kept probabilities times the dropout scale,
-    while lse stays that of the undropped softmax."""
+    while lse stays that of the undropped softmax.  query_mask: None or
+    [B, L], nonzero = real token: rows of padding tokens output zero (the
+    from-side mask of [GC] 随机块掩码是如何生成的, where BigBirdMasks derives
+    the from and to masks of the attention from the same input mask); their
+    lse is still the row's normaliser."""
     q = _prep(q)
     k = _prep(k)
     v = _prep(v)
@@ -323,6 +338,7 @@ def forward(q, k, v, key_mask, table, block_size, scale=None,
     if L % bs:
         raise ValueError("L must be a multiple of block_size")
     nb = L // bs
+    qf = _query_factors(query_mask, B, L)
     o = np.zeros((B, H, L, d))
     lse = np.zeros((B, H, L))
     for b in range(B):
@@ -333,20 +349,23 @@ def forward(q, k, v, key_mask, table, block_size, scale=None,
                 if dropout is not None:
                     p = p * dropout.factors(b, h, np.arange(i * bs, (i + 1) * bs),
                                             cols)
-                o[b, h, i * bs:(i + 1) * bs] = p @ v[b, h, cols]
-                lse[b, h, i * bs:(i + 1) * bs] = l
+                rows = slice(i * bs, (i + 1) * bs)
+                o[b, h, rows] = qf[b, rows][:, None] * (p @ v[b, h, cols])
+                lse[b, h, rows] = l
     return o, lse
 
 
 def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
-             mask_value=DEFAULT_MASK_VALUE, dropout=None):
+             mask_value=DEFAULT_MASK_VALUE, dropout=None, query_mask=None):
     """Gradient of forward's o with respect to q, k, v for upstream dout.
 
     Returns (dq, dk, dv), each [B, H, L, d] fp64.  Probabilities and o are
     recomputed here from the definition, in fp64.  With dropout (factors
     m_tu: the scale where kept, 0 where dropped) o_t = sum_u m_tu p_tu v_u,
     so D_t = <dO_t, o_t> still, dS_tu = p_tu (m_tu <dO_t, v_u> - D_t) and
-    dv_u = sum_t m_tu p_tu dO_t."""
+    dv_u = sum_t m_tu p_tu dO_t.  With query_mask the output row of a
+    padding token is multiplied by 0, so its dO_t enters as 0: its dq is 0
+    and it adds nothing to dk, dv."""
     q = _prep(q)
     k = _prep(k)
     v = _prep(v)
@@ -356,6 +375,7 @@ def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
     nb = L // bs
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    qf = _query_factors(query_mask, B, L)
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)
     dv = np.zeros_like(v)
@@ -367,7 +387,7 @@ def backward(q, k, v, dout, key_mask, table, block_size, scale=None,
                 rows = slice(i * bs, (i + 1) * bs)
                 vc = v[b, h, cols]
                 kc = k[b, h, cols]
-                do_i = dout[b, h, rows]
+                do_i = qf[b, rows][:, None] * dout[b, h, rows]
                 m = 1.0
                 if dropout is not None:
                     m = dropout.factors(b, h, np.arange(i * bs, (i + 1) * bs),

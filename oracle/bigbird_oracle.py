@@ -22,7 +22,7 @@ Sources (web pages; titles and sections):
   (ai-papers.xuzou.cn), section "方法适配": queries/keys are blockified and the
   attended block budget per query block is constant, so work is linear in L.
 
-Readings taken where the pages are silent (each listed in the design doc):
+Readings taken where the pages are silent:
 
 * The attended set A(i) of query block i is a SET of key blocks: rows 0 and
   nb-1 (global) attend every block; every other row attends
@@ -167,7 +167,7 @@ def attended_blocks(i, num_blocks, rand_row):
 # default) beside the ordinary dropout rate; section "梯度检查点的实现方式"
 # explains that, under recomputation, the dropout must be stateless and
 # seeded so that the recomputed forward draws the same noise.  Readings
-# (listed in the design doc): the dropout acts on the softmax probabilities of the
+# taken: the dropout acts on the softmax probabilities of the
 # attended keys (the usual attention dropout), the lse stays that of the
 # undropped softmax, and the keep decision of element (b, h, t, u) is a pure
 # function of (seed, b, h, t, u), drawn from Philox4x32-10 as specified below.

@@ -257,6 +257,20 @@ def bb_attn_check_status(workspace, stream=None):
     return lib().bb_attn_check_status(_ptr(workspace), _stream_ptr(stream))
 
 
+def make_table(seed, H, L, block_size, r, max_rand_mask_length=0,
+               last_idx=0):
+    """Random block table [H, L // block_size, r] (int32, CPU) for a call of
+    length L.  max_rand_mask_length, last_idx: the pages' layer options in
+    tokens (0 = off), converted to blocks by floor division; seed is the
+    layer index there."""
+    nb = L // block_size
+    if max_rand_mask_length or last_idx:
+        return bb_rand_attn_build_ex(seed, H, nb, r,
+                                     max_rand_mask_length // block_size,
+                                     last_idx // block_size)
+    return bb_rand_attn_build(seed, H, nb, r)
+
+
 class Attention:
     """Convenience wrapper holding the table and workspaces for one shape.
 
@@ -272,13 +286,8 @@ class Attention:
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
                               mask_value, dropout, dropout_seed)
         self.dtype = dtype
-        nb = L // block_size
-        if max_rand_mask_length or last_idx:
-            self.table_host = bb_rand_attn_build_ex(
-                seed, H, nb, r, max_rand_mask_length // block_size,
-                last_idx // block_size)
-        else:
-            self.table_host = bb_rand_attn_build(seed, H, nb, r)
+        self.table_host = make_table(seed, H, L, block_size, r,
+                                     max_rand_mask_length, last_idx)
         self.table = self.table_host.to(device)
         self.ws_fwd = torch.empty(bb_attn_workspace_size(self.desc, 0),
                                   dtype=torch.uint8, device=device)

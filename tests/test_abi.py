@@ -71,6 +71,19 @@ def test_rand_table_layer_options_off_equal_the_base_call():
     assert lib.bb_rand_attn_build_ex(0, 0, 32, 2, 64, 16, None) == 0  # empty
 
 
+def test_binding_table_options_in_tokens():
+    """The binding's table helper takes the pages' options in tokens: a
+    4096-token table with random blocks before token 1024, layer 7, used at
+    L = 2048 with block 64."""
+    got = bb.make_table(7, 12, 2048, 64, 3, max_rand_mask_length=4096,
+                        last_idx=1024).numpy()
+    assert np.array_equal(got, oracle.rand_table(7, 12, 32, 3, 64, 16))
+    assert np.array_equal(bb.make_table(7, 12, 2048, 64, 3).numpy(),
+                          oracle.rand_table(7, 12, 32, 3))
+    with pytest.raises(bb.BBError):
+        bb.make_table(7, 12, 2048, 64, 3, max_rand_mask_length=1024)
+
+
 def test_rand_table_errors():
     lib = bb.lib()
     assert lib.bb_rand_attn_build(0, -1, 4, 3, None) == -1

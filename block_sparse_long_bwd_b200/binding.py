@@ -16,6 +16,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbbattn.so")
 
 BB_OK = 0
+BB_ERR_TIMEOUT = -5
+BB_ERR_BAD_TABLE = -6
 BB_F32 = 0
 BB_BF16 = 1
 STATUS = {0: "BB_OK", -1: "BB_ERR_INVALID", -2: "BB_ERR_UNSUPPORTED",
@@ -90,6 +92,9 @@ def lib():
         L.bb_attn_fwd_noalloc.restype = ctypes.c_int
         L.bb_attn_check_status.argtypes = [_P, _P]
         L.bb_attn_check_status.restype = ctypes.c_int
+        L.bb_debug_wait_probe.argtypes = [_P, ctypes.c_size_t, ctypes.c_int,
+                                          _P]
+        L.bb_debug_wait_probe.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -269,6 +274,16 @@ def make_table(seed, H, L, block_size, r, max_rand_mask_length=0,
                                      max_rand_mask_length // block_size,
                                      last_idx // block_size)
     return bb_rand_attn_build(seed, H, nb, r)
+
+
+def bb_debug_wait_probe(workspace, armed, stream=None):
+    """Failure-detection self-test (see include/bb_attn.h): armed, a device
+    wait runs out and leaves BB_ERR_TIMEOUT in the workspace's status word;
+    read it with bb_attn_check_status."""
+    _cuda_tensor(workspace, "workspace")
+    _check(lib().bb_debug_wait_probe(
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        int(armed), _stream_ptr(stream)), "bb_debug_wait_probe")
 
 
 class Attention:

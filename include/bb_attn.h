@@ -240,6 +240,19 @@ BB_API int bb_attn_check_status(const void* workspace, void* stream);
 /* Static description of a status code (never NULL). */
 BB_API const char* bb_status_str(int status);
 
+/* Failure-detection self-test.  Launches one small kernel on `stream` that
+ * waits on an mbarrier through the bounded wait every tensor-core kernel
+ * uses (limit 2 s).  armed = 1: nothing completes the barrier, so the wait
+ * runs out, writes BB_ERR_TIMEOUT into the status word at the start of
+ * `workspace` (any buffer of >= 256 bytes, 16-byte aligned) and returns;
+ * the kernel exits normally and the context stays usable.  armed = 0: the
+ * barrier completes at once and the status word stays BB_OK.  Asynchronous:
+ * read the result with bb_attn_check_status(workspace, stream).  Returns
+ * BB_ERR_INVALID for a NULL, misaligned or short workspace or armed not 0/1,
+ * BB_ERR_CUDA if the launch fails. */
+BB_API int bb_debug_wait_probe(void* workspace, size_t ws_bytes, int armed,
+                               void* stream);
+
 /* BB_ABI_VERSION of the loaded library. */
 BB_API int bb_abi_version(void);
 

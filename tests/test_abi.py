@@ -84,6 +84,16 @@ def test_binding_table_options_in_tokens():
         bb.make_table(7, 12, 2048, 64, 3, max_rand_mask_length=1024)
 
 
+def test_wait_probe_rejects_bad_arguments_on_host():
+    """Invalid arguments are refused before any launch (fake pointers)."""
+    lib = bb.lib()
+    good = 1 << 20
+    assert lib.bb_debug_wait_probe(None, 256, 1, None) == -1
+    assert lib.bb_debug_wait_probe(good + 4, 256, 1, None) == -1
+    assert lib.bb_debug_wait_probe(good, 255, 1, None) == -1
+    assert lib.bb_debug_wait_probe(good, 256, 2, None) == -1
+
+
 def test_rand_table_errors():
     lib = bb.lib()
     assert lib.bb_rand_attn_build(0, -1, 4, 3, None) == -1

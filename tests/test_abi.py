@@ -194,6 +194,17 @@ def test_launch_lists_follow_the_dispatch():
     f32 = bb.make_desc(1, 2, 1024, 64, 64, 3, torch.float32)
     assert _names(f32, 0) == ["simt_fwd"]
     assert _names(f32, 1) == ["bwd_pre", "csr_build", "simt_dq", "simt_dkdv"]
+    # bf16 shapes outside the tensor-core bounds: L not a multiple of 64,
+    # r past the planner bound (27 at block 64, 11 at blocks 32 and 128).
+    for B, H, L, bs, r in ((1, 2, 96, 32, 2), (1, 1, 1024, 64, 28),
+                           (1, 1, 1024, 32, 12), (1, 1, 1024, 128, 12)):
+        d_ = bb.make_desc(B, H, L, 64, bs, r, torch.bfloat16)
+        assert _names(d_, 0) == ["simt_fwd"], (L, bs, r)
+        assert _names(d_, 1) == ["bwd_pre", "csr_build", "simt_dq",
+                                 "simt_dkdv"], (L, bs, r)
+    for bs, r in ((64, 27), (32, 11), (128, 11)):  # the largest on the tensor cores
+        d_ = bb.make_desc(1, 1, 1024, 64, bs, r, torch.bfloat16)
+        assert _names(d_, 0) == ["plan", "tc_fwd", "fwd_combine"], (bs, r)
     # A head's adjacency too large for shared memory: CSR built separately.
     huge = bb.make_desc(1, 1, 131072, 64, 32, 3, torch.bfloat16)
     assert _names(huge, 1)[:2] == ["csr_build", "plan"]

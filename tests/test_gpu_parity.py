@@ -57,6 +57,10 @@ SMALL = [
     (2, 1, 2048, 128, 3, "bf16", "random5"),
     (1, 1, 1152, 128, 2, "f32", "tail"),
     (1, 5, 2112, 64, 6, "bf16", None),
+    # bf16 outside the tensor-core bounds (CUDA-core kernels, bf16 I/O):
+    (1, 2, 96, 32, 2, "bf16", "tail"),      # L not a multiple of 64
+    (1, 1, 1024, 64, 28, "bf16", None),     # r past the planner bound
+    (1, 1, 1024, 32, 12, "bf16", "random5"),
 ]
 
 

@@ -107,6 +107,30 @@ def pairs_per_head(nb, table_h):
     return total
 
 
+def valid_key_fraction(nb, bs, table, key_mask):
+    """Share of the pattern's attended (query, key) products whose key is
+    not masked: per batch row b, each attended block pair counts the valid
+    keys of its key block instead of bs.  1.0 without a mask."""
+    if key_mask is None:
+        return 1.0
+    km = key_mask.numpy().astype(bool)
+    B = km.shape[0]
+    valid = km.reshape(B, nb, bs).sum(axis=2)  # [B, nb] valid keys per block
+    full = got = 0
+    for h in range(table.shape[0]):
+        for i in range(nb):
+            if i == 0 or i == nb - 1:
+                blocks = range(nb)
+            else:
+                s = {0, nb - 1, i - 1, i, i + 1}
+                s.update(int(j) for j in table[h, i] if 0 <= j < nb)
+                blocks = sorted(s)
+            for j in blocks:
+                full += B * bs
+                got += int(valid[:, j].sum())
+    return got / full
+
+
 def load_peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
@@ -363,6 +387,7 @@ def run_ours(args, world, rank, local):
     pairs = sum(pairs_per_head(nb, att.table_host[h].numpy())
                 for h in range(H)) * B
     alg = algorithmic(cfg, pairs)
+    vkf = valid_key_fraction(nb, bs, att.table_host.numpy(), inp["key_mask"])
     fwd_flops = 4 * pairs * bs * bs * cfg["d"]
     bwd_flops = 10 * pairs * bs * bs * cfg["d"] if backward else 0
     avg = {n: sum(v_) / len(v_) for n, v_ in per_kernel.items()}
@@ -431,7 +456,10 @@ def run_ours(args, world, rank, local):
             "fwd": round(fwd_flops * world / (sum(sum(per_kernel[n]) for n in names[:n_fwd]) / K / 1e3) / 1e12, 2),
             "fwd_bwd": round((fwd_flops + bwd_flops) * world / (ms_per_step / 1e3) / 1e12, 2),
             "convention": "4*bs^2*d per attended block pair fwd, 10*bs^2*d bwd",
-            "pairs": pairs},
+            "pairs": pairs,
+            # the same rates counting only products with an unmasked key
+            "valid_key_fraction": round(vkf, 4),
+            "fwd_valid_keys": round(vkf * fwd_flops * world / (sum(sum(per_kernel[n]) for n in names[:n_fwd]) / K / 1e3) / 1e12, 2)},
         "roofline": roofline,
         "kernels": kernels,
         "gpu_launches": K * (n_fwd + n_bwd),

@@ -37,7 +37,8 @@ class bb_attn_desc(ctypes.Structure):
                 ("d", ctypes.c_int), ("block_size", ctypes.c_int),
                 ("r", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("scale", ctypes.c_float), ("mask_value", ctypes.c_float),
-                ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_uint64)]
+                ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_uint64),
+                ("mask_queries", ctypes.c_int)]
 
 
 _lib = None
@@ -108,11 +109,12 @@ def bb_abi_version():
 
 
 def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0,
-              dropout=0.0, dropout_seed=0):
+              dropout=0.0, dropout_seed=0, mask_queries=0):
     if isinstance(dtype, torch.dtype):
         dtype = {torch.float32: BB_F32, torch.bfloat16: BB_BF16}[dtype]
     return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value,
-                        dropout, dropout_seed & ((1 << 64) - 1))
+                        dropout, dropout_seed & ((1 << 64) - 1),
+                        int(mask_queries))
 
 
 def _check(code, what):
@@ -294,12 +296,13 @@ class Attention:
 
     def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
                  device="cuda", scale=0.0, mask_value=0.0, dropout=0.0,
-                 dropout_seed=0, max_rand_mask_length=0, last_idx=0):
+                 dropout_seed=0, max_rand_mask_length=0, last_idx=0,
+                 mask_queries=0):
         """max_rand_mask_length, last_idx (tokens; 0 = off): the pages'
         layer options for the random table (drawn for the maximum length,
         random blocks before token last_idx); seed: the layer index there."""
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
-                              mask_value, dropout, dropout_seed)
+                              mask_value, dropout, dropout_seed, mask_queries)
         self.dtype = dtype
         self.table_host = make_table(seed, H, L, block_size, r,
                                      max_rand_mask_length, last_idx)

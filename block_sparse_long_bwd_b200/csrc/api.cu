@@ -109,6 +109,8 @@ int make_problem(const bb_attn_desc* desc, Problem* p) {
   p->drop_thr = (uint32_t)thr;
   p->drop_scale = (float)(256.0 / (256.0 - thr));
   p->drop_seed = desc->dropout_seed;
+  if (desc->mask_queries != 0 && desc->mask_queries != 1) return BB_ERR_INVALID;
+  p->mask_q = desc->mask_queries;  // cleared at the call when key_mask is NULL
   return BB_OK;
 }
 
@@ -231,6 +233,7 @@ static int fwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   p.k = k;
   p.v = v;
   p.key_mask = key_mask;
+  if (!key_mask) p.mask_q = 0;
   p.rand_idx = rand_idx;
   p.out = out;
   p.lse_out = lse;
@@ -276,6 +279,7 @@ static int bwd_impl(const bb_attn_desc* desc, const void* q, const void* k,
   p.lse = lse;
   p.dout = dout;
   p.key_mask = key_mask;
+  if (!key_mask) p.mask_q = 0;
   p.rand_idx = rand_idx;
   p.dq = dq;
   p.dk = dk;

@@ -26,6 +26,7 @@ struct Problem {
   uint32_t drop_thr;
   float drop_scale;
   uint64_t drop_seed;
+  int mask_q;  // 1: key_mask also zeroes the output rows of padding tokens
   // inputs
   const void* q;
   const void* k;

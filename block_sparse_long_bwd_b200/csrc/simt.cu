@@ -130,7 +130,9 @@ __global__ void __launch_bounds__(BS) simt_fwd_kernel(Problem p) {
       m = mn;
     }
   }
-  const float inv = 1.f / l;
+  // Query-side mask: the output row of a padding token is 0.
+  const bool qpad = p.mask_q && !p.key_mask[(size_t)b * p.L + (size_t)i * BS + tid];
+  const float inv = qpad ? 0.f : 1.f / l;
   T* Og = static_cast<T*>(p.out) + (bh * p.L + (size_t)i * BS + tid) * kHeadDim;
 #pragma unroll
   for (int c = 0; c < kHeadDim; ++c) Og[c] = from_f<T>(o[c] * inv);
@@ -167,7 +169,10 @@ __global__ void __launch_bounds__(BS) simt_dq_kernel(Problem p) {
     g[c] = to_f(static_cast<const T*>(p.dout)[row * kHeadDim + c]);
     dq[c] = 0.f;
   }
-  const float lse2 = p.lse[row] * kLog2e;
+  // Query-side mask: a padding token's p is 0 (lse taken as +inf).
+  const float lse2 = (p.mask_q && !p.key_mask[(size_t)b * p.L + (size_t)i * BS + tid])
+                         ? INFINITY
+                         : p.lse[row] * kLog2e;
   const float Dt = p.D[row];
   __syncthreads();
   const int n = global_row ? nb : nlist;
@@ -242,7 +247,10 @@ __global__ void __launch_bounds__(2 * BS) simt_dkdv_kernel(Problem p) {
       Gs[x] = to_f(Gb[(size_t)i * BS * kHeadDim + x]);
     }
     if (tid < BS) {
-      lse2[tid] = p.lse[bh * p.L + (size_t)i * BS + tid] * kLog2e;
+      // Query-side mask: a padding token's p is 0 (lse taken as +inf).
+      lse2[tid] = (p.mask_q && !p.key_mask[(size_t)b * p.L + (size_t)i * BS + tid])
+                      ? INFINITY
+                      : p.lse[bh * p.L + (size_t)i * BS + tid] * kLog2e;
       Ds[tid] = p.D[bh * p.L + (size_t)i * BS + tid];
     }
     __syncthreads();

@@ -368,6 +368,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       float nl2 = 0.f, Dr = 0.f;
       if (rvalid) {
         nl2 = -p.lse[grow] * kLog2e;
+        // Query-side mask: a padding token's P is 0 (NL = -inf), so its dS
+        // is 0 here and in the dK/dV pass, which reads NL.
+        if (p.mask_q && !p.key_mask[(size_t)im.b * p.L + tq]) nl2 = -INFINITY;
         const __nv_bfloat16* Or = static_cast<const __nv_bfloat16*>(p.o) + grow * kHeadDim;
         const __nv_bfloat16* Gr = static_cast<const __nv_bfloat16*>(p.dout) + grow * kHeadDim;
 #pragma unroll

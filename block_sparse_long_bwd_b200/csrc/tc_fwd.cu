@@ -427,7 +427,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const int r64 = row & 63;
       const bool write = (im.gvalid >> quarter) & 1;
-      const float inv = im.global ? 1.f : 1.f / l;
+      float inv = im.global ? 1.f : 1.f / l;
+      // Query-side mask: the output row of a padding token is 0 (global
+      // rows are zeroed when their chunks are combined).
+      if (p.mask_q && write && !im.global && !p.key_mask[(size_t)im.b * p.L + tq]) inv = 0.f;
       const size_t grow = (size_t)im.bh * p.L + (size_t)(write ? im.t[half] : 0) * kTile + r64;
       float* part = p.part +
                     ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) * 128 +
@@ -533,8 +536,11 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
     o0 = fmaf(w, o.x, o0);
     o1 = fmaf(w, o.y, o1);
   }
-  const float inv = 1.f / Lsum;
-  const size_t grow = bh * p.L + (size_t)t[row >> 6] * kTile + (row & 63);
+  const size_t tok = (size_t)t[row >> 6] * kTile + (row & 63);
+  const size_t grow = bh * p.L + tok;
+  // Query-side mask: the output row of a padding token is 0.
+  const float inv =
+      (p.mask_q && !p.key_mask[(bh / p.H) * p.L + tok]) ? 0.f : 1.f / Lsum;
   reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.out) +
                               grow * kHeadDim)[lane] =
       pack_bf16(o0 * inv, o1 * inv);

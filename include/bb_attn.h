@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define BB_ABI_VERSION 2
+#define BB_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define BB_API __attribute__((visibility("default")))
@@ -86,7 +86,15 @@ typedef enum { BB_F32 = 0, BB_BF16 = 1 } bb_dtype;
  * little-endian from its four output words in order, for key tokens
  * 16 (u >> 4) .. 16 (u >> 4) + 15; byte u & 15 keeps the element when it is
  * >= thr.  The backward must be called with the forward's dropout and
- * dropout_seed. */
+ * dropout_seed.
+ *
+ * mask_queries (0 or 1): with a key_mask, 1 also masks the query side, as
+ * the pages' BigBirdMasks derives its from-side mask from the same input
+ * mask ([gitcode page] "随机块掩码是如何生成的"): the output rows of padding
+ * tokens are 0, so they pass no gradient (their dq rows are 0 and they add
+ * nothing to dk, dv); their lse is still the row's normaliser.  The
+ * backward must be called with the forward's mask_queries.  Ignored without
+ * a key_mask. */
 typedef struct {
   int B, H, L, d, block_size, r;
   int dtype;
@@ -94,6 +102,7 @@ typedef struct {
   float mask_value;
   float dropout;
   uint64_t dropout_seed;
+  int mask_queries;
 } bb_attn_desc;
 
 /* Random block table ([gitcode page] section "随机块掩码是如何生成的": per

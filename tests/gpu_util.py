@@ -15,14 +15,15 @@ ATOL = {"f32": 2e-5, "bf16": 1e-2}
 
 def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
             scale=0.0, mask_value=0.0, table=None, dropout=0.0,
-            dropout_seed=0):
+            dropout_seed=0, mask_queries=0):
     """Forward (and backward) through the C ABI; returns CPU tensors."""
     dev = torch.device("cuda")
     B, H, L = cfg["B"], cfg["H"], cfg["L"]
     att = bb.Attention(B, H, L, cfg["block_size"], cfg["r"],
                        synth.torch_dtype(cfg["dtype"]), d=cfg["d"],
                        seed=table_seed, scale=scale, mask_value=mask_value,
-                       dropout=dropout, dropout_seed=dropout_seed)
+                       dropout=dropout, dropout_seed=dropout_seed,
+                       mask_queries=mask_queries)
     if table is not None:
         att.table_host = torch.as_tensor(table, dtype=torch.int32)
         att.table = att.table_host.to(dev)
@@ -43,7 +44,7 @@ def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
 
 def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
                  mask_value=oracle.DEFAULT_MASK_VALUE, dropout=0.0,
-                 dropout_seed=0):
+                 dropout_seed=0, mask_queries=0):
     """Oracle on the (b, h) slice: rows of one (b, h) depend on nothing else
     (the dropout decisions are drawn at the slice's own b and h)."""
     sl = lambda x: x[b:b + 1, h:h + 1].double().numpy()
@@ -52,14 +53,15 @@ def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,
     tab = np.asarray(table)[h:h + 1]
     drop = (oracle.Dropout(dropout, dropout_seed, b0=b, h0=h)
             if dropout else None)
+    qm = km if (mask_queries and km is not None) else None
     o, lse = oracle.forward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), km, tab,
-                            cfg["block_size"], scale, mask_value, drop)
+                            cfg["block_size"], scale, mask_value, drop, qm)
     res = {"out": o[0, 0], "lse": lse[0, 0]}
     if backward:
         dq, dk, dv = oracle.backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
                                      sl(inp["dout"]), km, tab,
                                      cfg["block_size"], scale, mask_value,
-                                     drop)
+                                     drop, qm)
         res.update(dq=dq[0, 0], dk=dk[0, 0], dv=dv[0, 0])
     return res
 

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
     assert "bb_attn_fwd" in names and "bb_attn_bwd" in names
     for name in names:
         assert hasattr(lib, name), name
-    assert bb.bb_abi_version() == 2
+    assert bb.bb_abi_version() == 3
 
 
 @pytest.mark.parametrize("seed,H,nb,r", [
@@ -123,6 +123,7 @@ def test_workspace_size_and_validation():
         # dropout outside [0, 1), NaN, or a rate that rounds to 1 (256/256)
         (dict(dropout=1.0), -1), (dict(dropout=-0.1), -1),
         (dict(dropout=float("nan")), -1), (dict(dropout=255.6 / 256), -1),
+        (dict(mask_queries=2), -1), (dict(mask_queries=-1), -1),
     ]
     lib = bb.lib()
     for kw, code in bad:

@@ -2,6 +2,7 @@
 
 python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                 [--workload NAME] [--dropout RATE [--dropout-seed S]]
+                [--mask-queries]
 
 One step = one forward + backward pass of the whole hot path over one batch
 of the named synthetic workload (default: BigBird-large attention layer at
@@ -72,6 +73,9 @@ def parse():
     # 0, the default, is the plain operation the headline line times).
     ap.add_argument("--dropout", type=float, default=0.0)
     ap.add_argument("--dropout-seed", type=int, default=0)
+    # With a masked workload: the key mask also zeroes the output rows of
+    # padding tokens (off by default).
+    ap.add_argument("--mask-queries", action="store_true")
     # Profiling runs (ncu) only: leave out the end-to-end and CPU legs.
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
@@ -302,7 +306,8 @@ def run_ours(args, world, rank, local):
     inp = synth.make_inputs(cfg, with_grad=backward)
     att = bb.Attention(B, H, L, bs, r, dt, d=cfg["d"], seed=synth.TABLE_SEED,
                        device=dev, dropout=args.dropout,
-                       dropout_seed=args.dropout_seed)
+                       dropout_seed=args.dropout_seed,
+                       mask_queries=int(args.mask_queries))
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     g = inp["dout"].to(dev) if backward else None
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
@@ -414,6 +419,7 @@ def run_ours(args, world, rank, local):
     traffic = None
     tr = NCU_TRAFFIC.get(dom)
     if (tr is not None and args.workload == tr[3] and not args.dropout and
+            not args.mask_queries and
             tr[1] == src_hash(os.path.join(ROOT, "block_sparse_long_bwd_b200",
                                            "csrc", tr[2]))):
         traffic = tr[0]
@@ -449,6 +455,7 @@ def run_ours(args, world, rank, local):
                    "block_size": bs, "d": cfg["d"], "r": r,
                    "mask": cfg["mask"], "passes": cfg["passes"],
                    "dropout": args.dropout,
+                   "mask_queries": bool(args.mask_queries),
                    "global_batch": B * world, "seq_len": L,
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (256 MiB write, untimed)"},
@@ -469,7 +476,8 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         result["cpu_baseline"] = None if args.skip_cpu else cpu_baseline(
             cfg, att.table_host.numpy(), backward, budget_s=12.0,
-            dropout=(args.dropout, args.dropout_seed))
+            dropout=(args.dropout, args.dropout_seed),
+            mask_queries=args.mask_queries)
         print(json.dumps(result), flush=True)
 
 
@@ -581,7 +589,7 @@ def run_e2e(args, cfg, att, inp, dev, backward, world):
 
 
 def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None,
-                 dropout=(0.0, 0)):
+                 dropout=(0.0, 0), mask_queries=False):
     """The fp64 oracle, as it stands, on (b, h) slices of the workload until
     the time budget is spent; scaled to tokens/s of the whole workload
     (each slice is 1/(B*H) of it).  dropout: (rate, seed) of the timed
@@ -606,13 +614,16 @@ def cpu_baseline(cfg, table, backward, budget_s=12.0, max_slices=None,
             for h in range(H):
                 drop = (oracle.Dropout(dropout[0], dropout[1], b0=b, h0=h)
                         if dropout[0] else None)
+                qm = km if mask_queries else None
                 t0 = time.perf_counter()
                 oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
-                               km, table[h:h + 1], bs, dropout=drop)
+                               km, table[h:h + 1], bs, dropout=drop,
+                               query_mask=qm)
                 if backward:
                     oracle.backward(f(inp["q"], h), f(inp["k"], h),
                                     f(inp["v"], h), f(inp["dout"], h), km,
-                                    table[h:h + 1], bs, dropout=drop)
+                                    table[h:h + 1], bs, dropout=drop,
+                                    query_mask=qm)
                 t_used += time.perf_counter() - t0
                 done += 1
                 if t_used >= budget_s or (max_slices and done >= max_slices):
@@ -645,12 +656,13 @@ def run_reference(args, world, rank):
         h = s % H
         drop = (oracle.Dropout(args.dropout, args.dropout_seed, b0=0, h0=h)
                 if args.dropout else None)
+        qm = km if args.mask_queries else None
         oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), km,
-                       table[h:h + 1], bs, dropout=drop)
+                       table[h:h + 1], bs, dropout=drop, query_mask=qm)
         if backward:
             oracle.backward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h),
                             f(inp["dout"], h), km, table[h:h + 1], bs,
-                            dropout=drop)
+                            dropout=drop, query_mask=qm)
 
     for s in range(args.warmup):
         step(s)
@@ -676,6 +688,7 @@ def run_reference(args, world, rank):
         "config": {"workload": args.workload, "B": B, "H": H, "L": L,
                    "block_size": bs, "d": cfg["d"], "r": r,
                    "dropout": args.dropout,
+                   "mask_queries": bool(args.mask_queries),
                    "global_batch": B, "seq_len": L},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                          "cores": cores, "kind": "oracle", "sample": sample},

@@ -189,6 +189,11 @@ def test_launch_lists_follow_the_dispatch():
     short = bb.make_desc(2, 4, 4096, 64, 64, 3, torch.bfloat16)
     assert _names(short, 0) == ["plan", "tc_fwd", "fwd_combine"]
     assert _names(short, 1) == ["plan", "tc_dq", "tc_dkdv", "bwd_finish"]
+    # dropout and the query mask change the kernels' variants, not the list
+    opt = bb.make_desc(2, 4, 4096, 64, 64, 3, torch.bfloat16, dropout=0.1,
+                       dropout_seed=3, mask_queries=1)
+    assert _names(opt, 0) == _names(short, 0)
+    assert _names(opt, 1) == _names(short, 1)
     for bs in (32, 64, 128):
         long_ = bb.make_desc(1, 2, 16384, 64, bs, 3, torch.bfloat16)
         assert _names(long_, 1) == ["plan", "tc_dq", "tc_dkdv", "tc_dkdv", "bwd_finish"], bs

@@ -69,3 +69,34 @@ def test_c_table_equals_oracle_on_random_arguments(seed, H, nb, r, extra,
     got = bb.bb_rand_attn_build_ex(seed, H, nb, r, mx, last).numpy()
     want = oracle.rand_table(seed, H, nb, r, max_blocks=mx, last_block=last)
     assert np.array_equal(got, want)
+
+
+@settings(**SETTINGS)
+@given(problems(), st.sampled_from([0.0, 0.1, 0.5]), st.booleans(),
+       st.integers(0, 2**64 - 1))
+def test_oracle_options_equal_dense_autograd_on_random_shapes(prob, rate,
+                                                              qmask, dseed):
+    """Dropout and the query mask on random shapes: the oracle against dense
+    softmax attention with the same keep factors and masked output rows."""
+    from test_dropout_oracle import _dense_dropout
+    B, H, nb, bs, d, r, masked, seed, own = prob
+    q, k, v, dout, km, table = _inputs(*prob)
+    L = nb * bs
+    qm = None
+    if qmask:
+        qm = (np.random.default_rng(seed + 7).random((B, L)) > 0.3).astype(
+            np.uint8)
+    drop = oracle.Dropout(rate, dseed)
+    o, _ = oracle.forward(q, k, v, km, table, bs, dropout=drop, query_mask=qm)
+    dq, dk, dv = oracle.backward(q, k, v, dout, km, table, bs, dropout=drop,
+                                 query_mask=qm)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True)
+                  for x in (q, k, v))
+    od, _ = _dense_dropout(tq, tk, tv, km, table, bs, 1.0 / math.sqrt(d),
+                           -10000.0, drop)
+    if qm is not None:
+        od = od * torch.from_numpy(qm.astype(np.float64))[:, None, :, None]
+    np.testing.assert_allclose(o, od.detach().numpy(), atol=1e-12, rtol=0)
+    (od * torch.from_numpy(dout)).sum().backward()
+    for got, want in ((dq, tq), (dk, tk), (dv, tv)):
+        np.testing.assert_allclose(got, want.grad.numpy(), atol=1e-10, rtol=0)

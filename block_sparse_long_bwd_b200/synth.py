@@ -7,8 +7,9 @@ Recipe (identical for the CUDA path and the oracle):
   as fp32 N(0, 1) of shape [B, H, L, d], then cast to the workload dtype
   (bf16 by round-to-nearest-even).  The oracle reads the same cast values.
 * key mask (uint8 [B, L], 1 = attend) from ``numpy.random.default_rng(S+1)``:
-  - "tail": per sequence a valid length drawn uniformly from the multiples
-    of 64 in [L/2, L]; keys at t >= length are masked;
+  - "tail": per sequence a valid length drawn uniformly from
+    L/2, L/2 + 64, ... (<= L) -- the multiples of 64 in [L/2, L] when L/2
+    is one, as at L = 4096; keys at t >= length are masked;
   - "random5": exactly round(0.05 L) key positions per sequence, drawn
     uniformly without replacement, are masked;
   - None: no mask (all keys attended).

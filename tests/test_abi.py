@@ -214,3 +214,39 @@ def test_launch_lists_follow_the_dispatch():
     # A head's adjacency too large for shared memory: CSR built separately.
     huge = bb.make_desc(1, 1, 131072, 64, 32, 3, torch.bfloat16)
     assert _names(huge, 1)[:2] == ["csr_build", "plan"]
+
+
+def test_host_calls_are_reentrant_across_threads():
+    """The host-only entry points called concurrently from several threads
+    (ctypes releases the GIL during the call) give the single-thread
+    results: the table builder, workspace sizing and the launch-name
+    lookup (thread-local name buffer)."""
+    import threading
+
+    import torch
+    want_t = bb.bb_rand_attn_build_ex(123, 4, 256, 6, 300, 100).numpy()
+    d_short = bb.make_desc(2, 4, 4096, 64, 64, 3, torch.bfloat16)
+    d_f32 = bb.make_desc(1, 2, 1024, 64, 64, 3, torch.float32)
+    want_n = (_names(d_short, 1), _names(d_f32, 1))
+    want_w = bb.bb_attn_workspace_size(d_short, 1)
+    errors = []
+
+    def worker(i):
+        try:
+            for _ in range(20):
+                t = bb.bb_rand_attn_build_ex(123, 4, 256, 6, 300, 100).numpy()
+                assert np.array_equal(t, want_t)
+                d = d_short if i % 2 else d_f32
+                names = [bb.bb_attn_launch_name(d, 1, k)
+                         for k in range(bb.bb_attn_launch_count(d, 1))]
+                assert names == want_n[0 if i % 2 else 1]
+                assert bb.bb_attn_workspace_size(d_short, 1) == want_w
+        except Exception as e:  # noqa: BLE001 - reported below
+            errors.append(e)
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(8)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors

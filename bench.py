@@ -51,7 +51,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 # changed source reports null.
 NCU_TRAFFIC = {
     # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, 1 launch;
-    # hashes refreshed after comment-only edits of the sources)
+    # hashes of the sources the counters were taken on: they no longer match
+    # since the dropout and query-mask variants, so the figure reads null
+    # until a new capture)
     "tc_fwd": (147637504 + 31209472, "0f41c4d9c5be114a", "tc_fwd.cu",
                "large_train_l4096"),
     "tc_dq": (224994560 + 33675264, "44becb5d0e98a1ed", "tc_bwd.cu",
@@ -148,7 +150,8 @@ def src_hash(path):
     csrc = os.path.dirname(path)
     h = hashlib.sha256()
     for p in [path] + [os.path.join(csrc, n) for n in
-                       ("tc_common.cuh", "sm100.cuh", "common.cuh")]:
+                       ("tc_common.cuh", "sm100.cuh", "common.cuh",
+                        "dropout.cuh")]:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -12,7 +12,9 @@
  * attended set A(i) is a set (each key block once).  For key token u of an
  * attended block the score is
  *     s = scale * <q, k_u> + (key_mask[b][u] ? 0 : mask_value)
- * and the row softmax over the attended keys weights V.
+ * and the row softmax over the attended keys weights V.  Options (see
+ * bb_attn_desc): seeded attention dropout on the attended probabilities,
+ * and a query-side mask that zeroes the output rows of padding tokens.
  *
  * Conventions shared by every call:
  *  - All tensors are dense, row-major, contiguous.  Q, K, V, O, dO, dQ, dK
@@ -28,7 +30,8 @@
  *    without synchronising.  Launch errors are returned; faults detected by a
  *    kernel (a wait that ran out, a corrupt random table) are written to a
  *    status word at the start of the workspace, read by bb_attn_check_status.
- *  - Calls are re-entrant and thread-safe (no global mutable state); two
+ *  - Calls are re-entrant and thread-safe (no global mutable state; the one
+ *    exception is bb_attn_fwd_noalloc's built-in scratch, see there); two
  *    calls may share a workspace only if they are ordered on the GPU.
  *  - Results are deterministic run to run: no floating-point atomics.
  */

@@ -81,6 +81,9 @@ def parse():
     # Profiling runs (ncu) only: leave out the end-to-end and CPU legs.
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
+    # Leave out the sub-records (the other workloads and the sweep, timed
+    # after the headline on rank 0).
+    ap.add_argument("--skip-sub", action="store_true")
     # Sweep mode: one line per (L, block, r) point of the length / block /
     # random-count sweep (B*L = 32768 tokens, H = 12), then the linear-in-L
     # check; not the headline line.
@@ -476,6 +479,8 @@ def run_ours(args, world, rank, local):
         "clocks": clocks,
         "e2e": e2e,
     }
+    if rank == 0 and not args.skip_sub and args.workload == DEFAULT_WORKLOAD:
+        result["sub"] = sub_records(dev, peaks)
     if rank == 0:
         result["cpu_baseline"] = None if args.skip_cpu else cpu_baseline(
             cfg, att.table_host.numpy(), backward, budget_s=12.0,
@@ -700,13 +705,76 @@ def run_reference(args, world, rank):
     }), flush=True)
 
 
-def run_sweep(args):
-    """fwd+bwd tokens/s and attended TFLOP/s per sweep point (device-timed,
-    CUDA events around each step, L2 flushed between steps), then the
-    linear-in-L check: at fixed (block, r), tokens/s within +-15 % of its
-    median over L."""
+def time_sweep_point(L, bs, r, steps, dev, flush, peaks):
+    """fwd+bwd of one sweep point, device-timed (CUDA events around each
+    step on the launching stream, L2 flushed between steps)."""
     from block_sparse_long_bwd_b200 import binding as bb
 
+    cfg = synth.sweep_point(L, bs, r)
+    B, H = cfg["B"], cfg["H"]
+    inp = synth.make_inputs(cfg)
+    att = bb.Attention(B, H, L, bs, r, torch.bfloat16, device=dev)
+    q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        att.forward(q, k, v, None, out=out, lse=lse, stream=stream)
+        att.backward(q, k, v, out, lse, g, None, dq=dq, dk=dk, dv=dv,
+                     stream=stream)
+
+    for _ in range(3):
+        step()
+    tot = 0.0
+    for s_ in range(steps):
+        flush.fill_(s_ & 0xFF)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / steps
+    pairs = sum(pairs_per_head(L // bs, att.table_host[h].numpy())
+                for h in range(H)) * B
+    # FLOPs by the FlashAttention convention: 4 (fwd) + 10 (bwd) bs^2 d per
+    # attended pair.
+    counted = (4 + 10) * pairs * bs * bs * cfg["d"]
+    names = [bb.bb_attn_launch_name(att.desc, 0, i)
+             for i in range(bb.bb_attn_launch_count(att.desc, 0))]
+    return {"L": L, "block_size": bs, "r": r, "B": B,
+            "ms": round(ms, 4),
+            "tokens_per_s": round(B * L / (ms / 1e3), 1),
+            "attended_tflops": round(counted / (ms / 1e3) / 1e12, 2),
+            "frac_of_peak": round(counted / (ms / 1e3) / 1e12
+                                  / peaks["bf16_tflops"], 4),
+            "path": "tensor" if any(n.startswith("tc_") for n in names)
+                    else "cuda-core"}
+
+
+def linear_in_L(rows):
+    """At fixed (block, r): tokens/s over L within +-15 % of its median."""
+    checks = []
+    for bs in synth.SWEEP_BS:
+        for r in synth.SWEEP_R:
+            tp = [x["tokens_per_s"] for x in rows
+                  if x["block_size"] == bs and x["r"] == r]
+            if not tp:
+                continue
+            med = statistics.median(tp)
+            dev_ = max(abs(t / med - 1) for t in tp)
+            checks.append({"block_size": bs, "r": r,
+                           "max_dev_from_median": round(dev_, 3),
+                           "linear_in_L": dev_ <= 0.15})
+    return checks
+
+
+def run_sweep(args):
+    """fwd+bwd tokens/s and attended TFLOP/s per sweep point, one JSON line
+    each, then the linear-in-L check."""
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks, _ = load_peaks()
@@ -715,62 +783,112 @@ def run_sweep(args):
     for bs in synth.SWEEP_BS:
         for r in synth.SWEEP_R:
             for L in synth.SWEEP_L:
-                cfg = synth.sweep_point(L, bs, r)
-                B, H = cfg["B"], cfg["H"]
-                inp = synth.make_inputs(cfg)
-                att = bb.Attention(B, H, L, bs, r, torch.bfloat16, device=dev)
-                q, k, v, g = (inp[n].to(dev) for n in ("q", "k", "v", "dout"))
-                out = torch.empty_like(q)
-                lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
-                dq, dk, dv = (torch.empty_like(q) for _ in range(3))
-
-                def step():
-                    att.forward(q, k, v, None, out=out, lse=lse)
-                    att.backward(q, k, v, out, lse, g, None, dq=dq, dk=dk, dv=dv)
-
-                for _ in range(3):
-                    step()
-                tot = 0.0
-                for s_ in range(args.sweep_steps):
-                    flush.fill_(s_ & 0xFF)
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record()
-                    step()
-                    e1.record()
-                    e1.synchronize()
-                    tot += e0.elapsed_time(e1)
-                ms = tot / args.sweep_steps
-                pairs = sum(pairs_per_head(L // bs, att.table_host[h].numpy())
-                            for h in range(H)) * B
-                # FLOPs by the FlashAttention convention: 4 (fwd) + 10 (bwd)
-                # bs^2 d per attended pair.
-                counted = (4 + 10) * pairs * bs * bs * cfg["d"]
-                names = [bb.bb_attn_launch_name(att.desc, 0, i)
-                         for i in range(bb.bb_attn_launch_count(att.desc, 0))]
-                row = {"L": L, "block_size": bs, "r": r, "B": B,
-                       "ms": round(ms, 4),
-                       "tokens_per_s": round(B * L / (ms / 1e3), 1),
-                       "attended_tflops": round(counted / (ms / 1e3) / 1e12, 2),
-                       "frac_of_peak": round(counted / (ms / 1e3) / 1e12
-                                             / peaks["bf16_tflops"], 4),
-                       "path": "tensor" if any(n.startswith("tc_") for n in names)
-                               else "cuda-core"}
+                row = time_sweep_point(L, bs, r, args.sweep_steps, dev, flush,
+                                       peaks)
                 rows.append(row)
                 print(json.dumps(row), flush=True)
-                del q, k, v, g, out, lse, dq, dk, dv, att
                 torch.cuda.empty_cache()
-    checks = []
+    print(json.dumps({"sweep_linear_in_L": linear_in_L(rows)}), flush=True)
+
+
+def time_workload(name, steps, dev, flush):
+    """Device time per step of a named workload (its own passes: forward
+    only for the BigBird-base layer), per launch and in total, with the
+    attended FLOP rates; L2 flushed between steps."""
+    from block_sparse_long_bwd_b200 import binding as bb
+
+    cfg = workload(name)
+    backward = cfg["passes"] == "fwd+bwd"
+    B, H, L, bs, r = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"], cfg["r"]
+    inp = synth.make_inputs(cfg, with_grad=backward)
+    att = bb.Attention(B, H, L, bs, r, synth.torch_dtype(cfg["dtype"]),
+                       d=cfg["d"], device=dev)
+    q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
+    g = inp["dout"].to(dev) if backward else None
+    km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    n_fwd = bb.bb_attn_launch_count(att.desc, 0)
+    n_bwd = bb.bb_attn_launch_count(att.desc, 1) if backward else 0
+    names = ([bb.bb_attn_launch_name(att.desc, 0, i) for i in range(n_fwd)]
+             + [bb.bb_attn_launch_name(att.desc, 1, i) for i in range(n_bwd)])
+    stream = torch.cuda.current_stream(dev)
+
+    def events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    def step(ev_f=None, ev_b=None):
+        att.forward(q, k, v, km, out=out, lse=lse, stream=stream, events=ev_f)
+        if backward:
+            att.backward(q, k, v, out, lse, g, km, dq=dq, dk=dk, dv=dv,
+                         stream=stream, events=ev_b)
+
+    for _ in range(3):
+        step()
+    evf = [events(n_fwd + 1) for _ in range(steps)]
+    evb = [events(n_bwd + 1) for _ in range(steps)] if backward else None
+    torch.cuda.synchronize(dev)
+    for s_ in range(steps):
+        flush.fill_(s_ & 0xFF)
+        step(evf[s_], evb[s_] if backward else None)
+    torch.cuda.synchronize(dev)
+    per = {n: 0.0 for n in names}
+    fwd_ms = tot = 0.0
+    for s_ in range(steps):
+        for i, n in enumerate(names[:n_fwd]):
+            per[n] += evf[s_][i].elapsed_time(evf[s_][i + 1])
+        fwd_ms += evf[s_][0].elapsed_time(evf[s_][-1])
+        tot += evf[s_][0].elapsed_time(evf[s_][-1])
+        if backward:
+            for i, n in enumerate(names[n_fwd:]):
+                per[n] += evb[s_][i].elapsed_time(evb[s_][i + 1])
+            tot += evb[s_][0].elapsed_time(evb[s_][-1])
+    ms = tot / steps
+    fwd_ms /= steps
+    pairs = sum(pairs_per_head(L // bs, att.table_host[h].numpy())
+                for h in range(H)) * B
+    unit = pairs * bs * bs * cfg["d"]
+    vkf = valid_key_fraction(L // bs, bs, att.table_host.numpy(),
+                             inp["key_mask"])
+    rec = {"workload": name, "passes": cfg["passes"], "steps": steps,
+           "ms_per_step": round(ms, 5),
+           "tokens_per_s": round(B * L / (ms / 1e3), 1),
+           "attended_tflops_fwd": round(4 * unit / (fwd_ms / 1e3) / 1e12, 2),
+           "valid_key_fraction": round(vkf, 4),
+           "kernels_ms": {n: round(per[n] / steps, 5) for n in names}}
+    if backward:
+        rec["attended_tflops_fwd_bwd"] = round(14 * unit / (ms / 1e3) / 1e12, 2)
+    if "tc_fwd" in per:
+        rec["tc_fwd_tflops"] = round(4 * unit / (per["tc_fwd"] / steps / 1e3)
+                                     / 1e12, 2)
+    return rec
+
+
+def sub_records(dev, peaks, sweep_steps=5):
+    """The other workloads and the sweep, timed in the same run after the
+    headline: the BigBird-base forward (its padded batch), the 16K pattern
+    (fwd+bwd), and every sweep point with the linear-in-L verdict."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    subs = {n: time_workload(n, 10, dev, flush)
+            for n in ("base_fwd_l4096", "long_l16384")}
+    rows = []
     for bs in synth.SWEEP_BS:
         for r in synth.SWEEP_R:
-            tp = [x["tokens_per_s"] for x in rows
-                  if x["block_size"] == bs and x["r"] == r]
-            med = statistics.median(tp)
-            dev_ = max(abs(t / med - 1) for t in tp)
-            checks.append({"block_size": bs, "r": r,
-                           "max_dev_from_median": round(dev_, 3),
-                           "linear_in_L": dev_ <= 0.15})
-    print(json.dumps({"sweep_linear_in_L": checks}), flush=True)
+            for L in synth.SWEEP_L:
+                rows.append(time_sweep_point(L, bs, r, sweep_steps, dev, flush,
+                                             peaks))
+                torch.cuda.empty_cache()
+    subs["sweep"] = {"steps_per_point": sweep_steps,
+                     "points": [{k_: x[k_] for k_ in ("L", "block_size", "r",
+                                                      "ms", "tokens_per_s",
+                                                      "attended_tflops")}
+                                for x in rows],
+                     "linear_in_L": linear_in_L(rows)}
+    return subs
 
 
 def main():

@@ -16,6 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbbattn.so")
 
 BB_OK = 0
+BB_ERR_WORKSPACE = -4
 BB_ERR_TIMEOUT = -5
 BB_ERR_BAD_TABLE = -6
 BB_F32 = 0
@@ -38,7 +39,7 @@ class bb_attn_desc(ctypes.Structure):
                 ("r", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("scale", ctypes.c_float), ("mask_value", ctypes.c_float),
                 ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_uint64),
-                ("mask_queries", ctypes.c_int)]
+                ("mask_queries", ctypes.c_int), ("grad_fp32", ctypes.c_int)]
 
 
 _lib = None
@@ -91,6 +92,8 @@ def lib():
         L.bb_attn_fwd_noalloc.argtypes = [ctypes.POINTER(bb_attn_desc)] + [
             _P] * 8
         L.bb_attn_fwd_noalloc.restype = ctypes.c_int
+        L.bb_attn_noalloc_status.argtypes = [_P]
+        L.bb_attn_noalloc_status.restype = ctypes.c_int
         L.bb_attn_check_status.argtypes = [_P, _P]
         L.bb_attn_check_status.restype = ctypes.c_int
         L.bb_debug_wait_probe.argtypes = [_P, ctypes.c_size_t, ctypes.c_int,
@@ -109,12 +112,20 @@ def bb_abi_version():
 
 
 def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0,
-              dropout=0.0, dropout_seed=0, mask_queries=0):
+              dropout=0.0, dropout_seed=0, mask_queries=0, grad_fp32=0):
     if isinstance(dtype, torch.dtype):
         dtype = {torch.float32: BB_F32, torch.bfloat16: BB_BF16}[dtype]
     return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value,
                         dropout, dropout_seed & ((1 << 64) - 1),
-                        int(mask_queries))
+                        int(mask_queries), int(grad_fp32))
+
+
+def grad_dtype(desc):
+    """torch dtype of dq, dk, dv for `desc` (fp32 when grad_fp32 is set or
+    the I/O dtype is fp32, else bf16)."""
+    if desc.grad_fp32 or desc.dtype == BB_F32:
+        return torch.float32
+    return torch.bfloat16
 
 
 def _check(code, what):
@@ -241,8 +252,10 @@ def bb_attn_fwd_noalloc(desc, q, k, v, key_mask, rand_idx, out, lse,
 def bb_attn_bwd(desc, q, k, v, out, lse, dout, key_mask, rand_idx, dq, dk, dv,
                 workspace, stream=None, events=None):
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out),
-                    ("dout", dout), ("dq", dq), ("dk", dk), ("dv", dv)):
+                    ("dout", dout)):
         _cuda_tensor(t, name, q.dtype)
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _cuda_tensor(t, name, grad_dtype(desc))
     _cuda_tensor(lse, "lse", torch.float32)
     _cuda_tensor(workspace, "workspace")
     if key_mask is not None:
@@ -258,6 +271,12 @@ def bb_attn_bwd(desc, q, k, v, out, lse, dout, key_mask, rand_idx, dq, dk, dv,
     else:
         arr, n = _event_array(events)
         _check(lib().bb_attn_bwd_events(*args, arr, n), "bb_attn_bwd_events")
+
+
+def bb_attn_noalloc_status(stream=None):
+    """Status word the last bb_attn_fwd_noalloc left in the built-in
+    scratch (waits for the stream)."""
+    return lib().bb_attn_noalloc_status(_stream_ptr(stream))
 
 
 def bb_attn_check_status(workspace, stream=None):
@@ -297,12 +316,14 @@ class Attention:
     def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
                  device="cuda", scale=0.0, mask_value=0.0, dropout=0.0,
                  dropout_seed=0, max_rand_mask_length=0, last_idx=0,
-                 mask_queries=0):
+                 mask_queries=0, grad_fp32=0):
         """max_rand_mask_length, last_idx (tokens; 0 = off): the pages'
         layer options for the random table (drawn for the maximum length,
-        random blocks before token last_idx); seed: the layer index there."""
+        random blocks before token last_idx); seed: the layer index there.
+        grad_fp32: the backward writes dq, dk, dv as fp32."""
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
-                              mask_value, dropout, dropout_seed, mask_queries)
+                              mask_value, dropout, dropout_seed, mask_queries,
+                              grad_fp32)
         self.dtype = dtype
         self.table_host = make_table(seed, H, L, block_size, r,
                                      max_rand_mask_length, last_idx)
@@ -325,9 +346,10 @@ class Attention:
 
     def backward(self, q, k, v, out, lse, dout, key_mask=None, dq=None,
                  dk=None, dv=None, stream=None, events=None):
-        dq = torch.empty_like(q) if dq is None else dq
-        dk = torch.empty_like(k) if dk is None else dk
-        dv = torch.empty_like(v) if dv is None else dv
+        gd = grad_dtype(self.desc)
+        dq = torch.empty_like(q, dtype=gd) if dq is None else dq
+        dk = torch.empty_like(k, dtype=gd) if dk is None else dk
+        dv = torch.empty_like(v, dtype=gd) if dv is None else dv
         bb_attn_bwd(self.desc, q, k, v, out, lse, dout, key_mask, self.table,
                     dq, dk, dv, self.ws_bwd, stream, events)
         return dq, dk, dv

@@ -111,6 +111,8 @@ int make_problem(const bb_attn_desc* desc, Problem* p) {
   p->drop_seed = desc->dropout_seed;
   if (desc->mask_queries != 0 && desc->mask_queries != 1) return BB_ERR_INVALID;
   p->mask_q = desc->mask_queries;  // cleared at the call when key_mask is NULL
+  if (desc->grad_fp32 != 0 && desc->grad_fp32 != 1) return BB_ERR_INVALID;
+  p->grad_f32 = (p->dtype == BB_F32) ? 1 : desc->grad_fp32;
   return BB_OK;
 }
 

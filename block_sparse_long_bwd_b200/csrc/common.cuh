@@ -27,6 +27,7 @@ struct Problem {
   float drop_scale;
   uint64_t drop_seed;
   int mask_q;  // 1: key_mask also zeroes the output rows of padding tokens
+  int grad_f32;  // 1: dq, dk, dv are written as fp32 (else in dtype)
   // inputs
   const void* q;
   const void* k;
@@ -138,6 +139,16 @@ __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) {
   return __float2bfloat16_rn(x);
+}
+
+// Element i of a gradient output: fp32 when the call asked for fp32
+// gradients, else the I/O type T (rounded to nearest even from x).
+template <typename T>
+__device__ __forceinline__ void store_grad(const Problem& p, void* base, size_t i, float x) {
+  if (p.grad_f32)
+    static_cast<float*>(base)[i] = x;
+  else
+    static_cast<T*>(base)[i] = from_f<T>(x);
 }
 
 // Record the first non-OK status of a call (integer atomic, not a result).

@@ -202,9 +202,9 @@ __global__ void __launch_bounds__(BS) simt_dq_kernel(Problem p) {
       }
     }
   }
-  T* dQg = static_cast<T*>(p.dq) + row * kHeadDim;
+  const size_t q0 = (size_t)row * kHeadDim;
 #pragma unroll
-  for (int c = 0; c < kHeadDim; ++c) dQg[c] = from_f<T>(dq[c] * p.scale);
+  for (int c = 0; c < kHeadDim; ++c) store_grad<T>(p, p.dq, q0 + c, dq[c] * p.scale);
 }
 
 // dK/dV for key block j over the query blocks of its CSR list.  Two threads
@@ -287,12 +287,11 @@ __global__ void __launch_bounds__(2 * BS) simt_dkdv_kernel(Problem p) {
     }
   }
   // Qs held q * scale * log2(e); dk = scale * sum ds q = sum ds (Qs / log2 e).
-  T* dKg = static_cast<T*>(p.dk) + krow * kHeadDim + half * 32;
-  T* dVg = static_cast<T*>(p.dv) + krow * kHeadDim + half * 32;
+  const size_t k0 = (size_t)krow * kHeadDim + half * 32;
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
-    dKg[c] = from_f<T>(dk[c] * (1.0f / kLog2e));
-    dVg[c] = from_f<T>(dv[c]);
+    store_grad<T>(p, p.dk, k0 + c, dk[c] * (1.0f / kLog2e));
+    store_grad<T>(p, p.dv, k0 + c, dv[c]);
   }
 }
 

@@ -60,6 +60,35 @@ __device__ __forceinline__ void ld_bf16x8_as_f(const __nv_bfloat16* p,
   }
 }
 
+// One 64-element gradient row (fp32 bit patterns, columns 0-31 in lo and
+// 32-63 in hi) times mul, stored as bf16 (rounded to nearest even) or, when
+// the call asked for fp32 gradients, as fp32.
+__device__ __forceinline__ void store_grad_row(const Problem& p, void* base, size_t row,
+                                               const uint32_t (&lo)[32],
+                                               const uint32_t (&hi)[32], float mul) {
+  if (p.grad_f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + row * kHeadDim);
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      const uint32_t* src = v < 8 ? lo + 4 * v : hi + 4 * (v - 8);
+      dst[v] = make_float4(__uint_as_float(src[0]) * mul, __uint_as_float(src[1]) * mul,
+                           __uint_as_float(src[2]) * mul, __uint_as_float(src[3]) * mul);
+    }
+    return;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + row * kHeadDim);
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    const uint32_t* src = v < 4 ? lo + 8 * v : hi + 8 * (v - 4);
+    uint4 w;
+    w.x = pack_bf16(__uint_as_float(src[0]) * mul, __uint_as_float(src[1]) * mul);
+    w.y = pack_bf16(__uint_as_float(src[2]) * mul, __uint_as_float(src[3]) * mul);
+    w.z = pack_bf16(__uint_as_float(src[4]) * mul, __uint_as_float(src[5]) * mul);
+    w.w = pack_bf16(__uint_as_float(src[6]) * mul, __uint_as_float(src[7]) * mul);
+    dst[v] = w;
+  }
+}
+
 // ======================= dQ =======================
 
 // P = 2^(S c + NL) of 32 key columns (col0: 0 or 32 within the tile) of
@@ -469,18 +498,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive(&bars.dq_empty);
       if (rvalid) {
         if (!im.global) {
-          uint4* dst = reinterpret_cast<uint4*>(
-              static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint32_t* src = v < 4 ? q0 + 8 * v : q1 + 8 * (v - 4);
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(src[0]) * p.scale, __uint_as_float(src[1]) * p.scale);
-            w.y = pack_bf16(__uint_as_float(src[2]) * p.scale, __uint_as_float(src[3]) * p.scale);
-            w.z = pack_bf16(__uint_as_float(src[4]) * p.scale, __uint_as_float(src[5]) * p.scale);
-            w.w = pack_bf16(__uint_as_float(src[6]) * p.scale, __uint_as_float(src[7]) * p.scale);
-            dst[v] = w;
-          }
+          store_grad_row(p, p.dq, grow, q0, q1, p.scale);
         } else {
           float4* dst = reinterpret_cast<float4*>(
               ba.dqpart + ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) *
@@ -883,24 +901,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive(&bars.acc_empty);
       if (rvalid) {
         if (!it.global) {
-          uint4* dk = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dk) + krow * kHeadDim);
-          uint4* dv = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dv) + krow * kHeadDim);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint32_t* sk = v < 4 ? k0 + 8 * v : k1 + 8 * (v - 4);
-            const uint32_t* sv = v < 4 ? v0 + 8 * v : v1 + 8 * (v - 4);
-            uint4 w;
-            w.x = pack_bf16(__uint_as_float(sk[0]) * p.scale, __uint_as_float(sk[1]) * p.scale);
-            w.y = pack_bf16(__uint_as_float(sk[2]) * p.scale, __uint_as_float(sk[3]) * p.scale);
-            w.z = pack_bf16(__uint_as_float(sk[4]) * p.scale, __uint_as_float(sk[5]) * p.scale);
-            w.w = pack_bf16(__uint_as_float(sk[6]) * p.scale, __uint_as_float(sk[7]) * p.scale);
-            dk[v] = w;
-            w.x = pack_bf16(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
-            w.y = pack_bf16(__uint_as_float(sv[2]), __uint_as_float(sv[3]));
-            w.z = pack_bf16(__uint_as_float(sv[4]), __uint_as_float(sv[5]));
-            w.w = pack_bf16(__uint_as_float(sv[6]), __uint_as_float(sv[7]));
-            dv[v] = w;
-          }
+          store_grad_row(p, p.dk, krow, k0, k1, p.scale);
+          store_grad_row(p, p.dv, krow, v0, v1, 1.0f);
         } else {
           float4* dst = reinterpret_cast<float4*>(
               ba.kvpart + ((((size_t)it.bh * ba.qa.geo.n_git + it.gi) * ba.qa.geo.nchunks +
@@ -963,6 +965,15 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
     k1 += xk.y;
     v0 += xv.x;
     v1 += xv.y;
+  }
+  if (p.grad_f32) {
+    reinterpret_cast<float2*>(static_cast<float*>(p.dq) + grow * kHeadDim)[lane] =
+        make_float2(q0 * p.scale, q1 * p.scale);
+    reinterpret_cast<float2*>(static_cast<float*>(p.dk) + grow * kHeadDim)[lane] =
+        make_float2(k0 * p.scale, k1 * p.scale);
+    reinterpret_cast<float2*>(static_cast<float*>(p.dv) + grow * kHeadDim)[lane] =
+        make_float2(v0, v1);
+    return;
   }
   reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim)[lane] =
       pack_bf16(q0 * p.scale, q1 * p.scale);

@@ -18,8 +18,9 @@
  *
  * Conventions shared by every call:
  *  - All tensors are dense, row-major, contiguous.  Q, K, V, O, dO, dQ, dK
- *    and dV are [B][H][L][d] in the descriptor's dtype (fp32 or bf16); the
- *    blocked view [B][H][nb][block_size][d] of the pages is the same memory.
+ *    and dV are [B][H][L][d] in the descriptor's dtype (fp32 or bf16; dQ,
+ *    dK and dV in fp32 instead when grad_fp32 = 1); the blocked view
+ *    [B][H][nb][block_size][d] of the pages is the same memory.
  *    lse and the workspace's fp32 arrays are fp32.
  *  - Pointers named *_host are host memory; every other pointer is device
  *    memory of the current CUDA device.  The caller owns every buffer; the
@@ -45,7 +46,7 @@
 extern "C" {
 #endif
 
-#define BB_ABI_VERSION 3
+#define BB_ABI_VERSION 4
 
 #if defined(__GNUC__)
 #define BB_API __attribute__((visibility("default")))
@@ -97,7 +98,18 @@ typedef enum { BB_F32 = 0, BB_BF16 = 1 } bb_dtype;
  * tokens are 0, so they pass no gradient (their dq rows are 0 and they add
  * nothing to dk, dv); their lse is still the row's normaliser.  The
  * backward must be called with the forward's mask_queries.  Ignored without
- * a key_mask. */
+ * a key_mask.
+ *
+ * grad_fp32 (0 or 1; backward only): 1 writes dq, dk and dv as fp32 instead
+ * of the dtype.  The kernels accumulate in fp32 either way; with bf16 the
+ * stored gradient is that fp32 value rounded to nearest even, bit for bit.
+ * Why it matters: the gradients of the two global key blocks sum over every
+ * query row, so their magnitude grows with the square root of L (about 5
+ * at L = 32768 and 10 at L = 131072 for unit-variance inputs), and above 4
+ * bf16's own spacing (1/32, then 1/16 above 8) alone exceeds an absolute
+ * error of 1e-2.  Use grad_fp32 = 1 where gradients must be within a fixed
+ * absolute error of the exact result at such lengths.  Ignored for fp32
+ * dtype (the gradients are fp32 already). */
 typedef struct {
   int B, H, L, d, block_size, r;
   int dtype;
@@ -106,6 +118,7 @@ typedef struct {
   float dropout;
   uint64_t dropout_seed;
   int mask_queries;
+  int grad_fp32;
 } bb_attn_desc;
 
 /* Random block table ([gitcode page] section "随机块掩码是如何生成的": per
@@ -176,7 +189,8 @@ BB_API int bb_attn_fwd(const bb_attn_desc* desc, const void* q, const void* k,
  * recomputing the probabilities from lse instead of storing them.
  *   q, k, v, out, lse, key_mask, rand_idx as produced / used by bb_attn_fwd
  *   dout      [B][H][L][d] dtype, device
- *   dq, dk, dv [B][H][L][d] dtype, device (written)
+ *   dq, dk, dv [B][H][L][d] dtype (fp32 when desc->grad_fp32 = 1), device
+ *             (written)
  *   workspace device, >= bb_attn_workspace_size(desc, 1) bytes; holds the
  *             transposed block adjacency (query blocks per key block) and
  *             the per-row D = <dO, O>. */
@@ -229,20 +243,34 @@ BB_API int bb_attn_bwd_events(const bb_attn_desc* desc, const void* q,
  * device that loads the library keeps until the process exits.  The caller
  * still provides q, k, v, key_mask, rand_idx, out and lse.
  *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating routine.
- *  - The first call on a device looks up the scratch's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *  - Every call looks up the scratch's device address (cudaGetSymbolAddress)
+ *    in the CUDA context current on the calling thread, so the call serves
+ *    whichever context is current (the runtime's primary context or a
+ *    caller's own driver-API context on the device).  The first call in a
+ *    context also loads the library's device code there; make that first
+ *    call before any stream capture.
  *  - Returns BB_ERR_WORKSPACE, without launching anything, when the problem
  *    needs more than 32 MiB of workspace (bb_attn_workspace_size(desc, 0)).
- *  - Every call shares the one scratch array, which keeps the last call's
- *    contents: calls that overlap on the GPU (other streams, other threads
- *    on the same device) race; order them on one stream.  The device status
- *    word lives in the scratch and is not reported by this call. */
+ *  - Every call shares the one scratch array of the context, which keeps the
+ *    last call's contents (the call clears its status word and writes
+ *    everything else before reading it): calls that overlap on the GPU
+ *    (other streams, other threads on the same device) race; order them on
+ *    one stream.  The device status word of the last call (a bounded wait
+ *    that ran out, a corrupt random table) is read with
+ *    bb_attn_noalloc_status. */
 BB_API int bb_attn_fwd_noalloc(const bb_attn_desc* desc, const void* q,
                                const void* k, const void* v,
                                const uint8_t* key_mask,
                                const int32_t* rand_idx, void* out, float* lse,
                                void* stream);
+
+/* Status word left in the built-in scratch by the last bb_attn_fwd_noalloc
+ * of the current context: waits for `stream`, then returns BB_OK,
+ * BB_ERR_TIMEOUT or BB_ERR_BAD_TABLE (as bb_attn_check_status does for a
+ * workspace), or BB_ERR_CUDA if the lookup or the copy failed.  Allocates
+ * nothing.  Like the forward it reports on, it has no counterpart in the
+ * pages. */
+BB_API int bb_attn_noalloc_status(void* stream);
 
 /* Waits for `stream`, then returns the status word the last call that used
  * `workspace` left there (BB_OK, BB_ERR_TIMEOUT or BB_ERR_BAD_TABLE), or

@@ -33,7 +33,7 @@ int main(void) {
   int32_t table[H * NB * R], table_ex[H * NB * R];
   int h, i, a;
   size_t ws = 0;
-  bb_attn_desc d = {2, H, NB * 64, 64, 64, R, BB_BF16, 0.f, 0.f, 0.f, 0, 0};
+  bb_attn_desc d = {2, H, NB * 64, 64, 64, R, BB_BF16, 0.f, 0.f, 0.f, 0, 0, 0};
   bb_attn_desc bad = d;
   const uintptr_t fake = (uintptr_t)1 << 20; /* never dereferenced */
   void* p = (void*)fake;

@@ -15,15 +15,17 @@ ATOL = {"f32": 2e-5, "bf16": 1e-2}
 
 def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
             scale=0.0, mask_value=0.0, table=None, dropout=0.0,
-            dropout_seed=0, mask_queries=0):
-    """Forward (and backward) through the C ABI; returns CPU tensors."""
+            dropout_seed=0, mask_queries=0, grad_fp32=0):
+    """Forward (and backward) through the C ABI; returns CPU tensors.
+    grad_fp32: the backward writes dq, dk, dv as fp32 (returned as such;
+    bf16 gradients come back widened to fp32 exactly)."""
     dev = torch.device("cuda")
     B, H, L = cfg["B"], cfg["H"], cfg["L"]
     att = bb.Attention(B, H, L, cfg["block_size"], cfg["r"],
                        synth.torch_dtype(cfg["dtype"]), d=cfg["d"],
                        seed=table_seed, scale=scale, mask_value=mask_value,
                        dropout=dropout, dropout_seed=dropout_seed,
-                       mask_queries=mask_queries)
+                       mask_queries=mask_queries, grad_fp32=grad_fp32)
     if table is not None:
         att.table_host = torch.as_tensor(table, dtype=torch.int32)
         att.table = att.table_host.to(dev)
@@ -72,3 +74,12 @@ def assert_close(gpu, ora, b, h, atol, names):
         err = np.abs(g - ora[n]).max()
         assert np.isfinite(g).all(), (n, b, h)
         assert err <= atol, f"{n}[{b},{h}] max-abs err {err:.3e} > {atol}"
+
+
+def assert_bf16_is_rounded_fp32(g16, g32, names=("dq", "dk", "dv")):
+    """bf16 gradients equal the fp32 gradients of the same kernels rounded
+    to nearest even, bit for bit (the kernels accumulate in fp32 and round
+    only when storing)."""
+    for n in names:
+        want = g32[n].to(torch.bfloat16).float()
+        assert torch.equal(g16[n], want), n

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
     assert "bb_attn_fwd" in names and "bb_attn_bwd" in names
     for name in names:
         assert hasattr(lib, name), name
-    assert bb.bb_abi_version() == 3
+    assert bb.bb_abi_version() == 4
 
 
 @pytest.mark.parametrize("seed,H,nb,r", [
@@ -124,6 +124,7 @@ def test_workspace_size_and_validation():
         (dict(dropout=1.0), -1), (dict(dropout=-0.1), -1),
         (dict(dropout=float("nan")), -1), (dict(dropout=255.6 / 256), -1),
         (dict(mask_queries=2), -1), (dict(mask_queries=-1), -1),
+        (dict(grad_fp32=2), -1), (dict(grad_fp32=-1), -1),
     ]
     lib = bb.lib()
     for kw, code in bad:
@@ -131,6 +132,8 @@ def test_workspace_size_and_validation():
         got = lib.bb_attn_workspace_size(ctypes.byref(_desc(**kw)), 0,
                                          ctypes.byref(n))
         assert got == code, (kw, got)
+    # fp32 gradient outputs change nothing in the workspace
+    assert bb.bb_attn_workspace_size(_desc(grad_fp32=1), 1) == n1
     for rate in (0.1, 0.5, 255.4 / 256):  # valid rates, any seed
         assert bb.bb_attn_workspace_size(
             _desc(dropout=rate, dropout_seed=2**64 - 1), 1) == n1

@@ -450,10 +450,38 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
   }
 }
 
+// One word of the forward's masked-tile bitmap (see Problem::tdead): warp w
+// of batch b writes word w (w = 0: the flag word, from the first 32 keys;
+// w >= 1: tiles 32 (w - 1) .. 32 (w - 1) + 31, lane i testing the 64 keys of
+// one tile).
+__device__ void dead_tile_word(const Problem& p, int nt, int b, int w, int lane) {
+  const uint8_t* km = p.key_mask + (size_t)b * p.L;
+  bool bit;
+  if (w == 0) {
+    bit = km[lane] != 0;  // keys 0..31 lie in block 0 for every block size
+  } else {
+    const int j = 32 * (w - 1) + lane;
+    bit = false;
+    if (j < nt) {
+      const uint4* m4 = reinterpret_cast<const uint4*>(km + (size_t)j * kTile);
+      uint32_t any = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint4 x = __ldg(m4 + c);
+        any |= x.x | x.y | x.z | x.w;
+      }
+      bit = any == 0;
+    }
+  }
+  const uint32_t word = __ballot_sync(0xffffffffu, bit);
+  if (lane == 0) p.tdead[(size_t)b * p.tdead_words + w] = w == 0 ? (word != 0 ? 1u : 0u) : word;
+}
+
 // Plans, one warp per item: query-side lists (do_q) and key-side walks
-// (do_k, after the CSR exists).
+// (do_k, after the CSR exists); with do_dead, then one warp per word of the
+// forward's masked-tile bitmap.
 __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do_q,
-                                                               int do_k) {
+                                                               int do_k, int do_dead) {
   __shared__ int cand[kPlanWarps][128];
   __shared__ int stage[kPlanWarps][kStageCap];
   const Geom g = make_geom(p.L, p.bs);
@@ -463,6 +491,12 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
   if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
   const int id = blockIdx.x * kPlanWarps + warp;
   const int nq = do_q ? nitems : 0;
+  const int nk = do_k ? nitems : 0;
+  if (do_dead && id >= nq + nk) {
+    const int x = id - nq - nk;
+    if (x < p.B * p.tdead_words) dead_tile_word(p, g.nt, x / p.tdead_words, x % p.tdead_words, lane);
+    return;
+  }
   if (id < nq) {
     plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], stage[warp], lane);
   } else if (do_k && id - nq < nitems) {
@@ -636,11 +670,15 @@ int tc_kplan_cap(const Problem& p) {
   return 2 * pair_cap(p.nb, p.r) + g.n_git * g.nt + 64;
 }
 
+int tc_tdead_words(const Problem& p) { return 1 + (make_geom(p.L, p.bs).nt + 31) / 32; }
+
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
   const int items = p.H * (int)tc_items_per_bh(p);
-  const int n = items * (key_side ? 2 : 1);
+  // The forward with a key mask also writes its masked-tile bitmap.
+  const int dead = (!key_side && p.key_mask && p.tdead) ? 1 : 0;
+  const int n = items * (key_side ? 2 : 1) + (dead ? p.B * p.tdead_words : 0);
   plan_kernel<<<(n + kPlanWarps - 1) / kPlanWarps, 32 * kPlanWarps, 0, s>>>(
-      p, 1, key_side ? 1 : 0);
+      p, 1, key_side ? 1 : 0, dead);
   return cudaGetLastError();
 }
 

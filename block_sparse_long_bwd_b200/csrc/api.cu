@@ -23,6 +23,8 @@ WsLayout ws_layout(const Problem& p, int pass) {
     off = align_up(off + tc_fwd_part_bytes(p), 256);
     w.qplan_off = off;
     off = align_up(off + tc_qplan_bytes(p), 256);
+    w.tdead_off = off;
+    off = align_up(off + (size_t)p.B * tc_tdead_words(p) * sizeof(uint32_t), 256);
     w.total = off;
     return w;
   }
@@ -133,6 +135,10 @@ int carve(Problem* p, int pass, void* ws, size_t ws_bytes) {
   p->part = (float*)(base + w.part_off);
   p->part_floats = (ws_bytes - w.part_off) / sizeof(float);
   if (w.qplan_off) p->qplan = base + w.qplan_off;
+  if (w.tdead_off) {
+    p->tdead = (uint32_t*)(base + w.tdead_off);
+    p->tdead_words = tc_tdead_words(*p);
+  }
   if (w.kof_off) {
     p->kof = (int*)(base + w.kof_off);
     p->kplan = (uint32_t*)(base + w.kplan_off);

@@ -58,6 +58,11 @@ struct Problem {
                      // then [H] allocation counters
   uint32_t* kplan;   // [H][kcap] key-side walk entries
   int kcap;
+  // forward, with a key mask: per batch b, word 0 = 1 when key tiles may be
+  // skipped (a key among the first 32 is valid), then one bit per 64-key
+  // tile whose keys are all masked; [B][tdead_words]
+  uint32_t* tdead;
+  int tdead_words;
 };
 
 // Upper bound of attended (query block, key block) pairs per head.
@@ -67,6 +72,7 @@ inline int pair_cap(int nb, int r) { return nb * (7 + r) + 8; }
 struct WsLayout {
   size_t status_off, D_off, offs_off, list_off, part_off;
   size_t qplan_off, kof_off, kplan_off;  // tensor-core plans (0: none)
+  size_t tdead_off;                      // masked-tile bitmap (0: none)
   size_t total;
 };
 WsLayout ws_layout(const Problem& p, int pass);
@@ -105,6 +111,9 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
 
 bool tc_bwd_supported(const Problem& p);
 size_t tc_qplan_bytes(const Problem& p);
+// Words per batch of the forward's masked-tile bitmap (a flag word, then one
+// bit per 64-key tile).
+int tc_tdead_words(const Problem& p);
 int tc_kplan_cap(const Problem& p);
 size_t tc_items_per_bh(const Problem& p);
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s);

@@ -81,6 +81,16 @@ __device__ __forceinline__ uint64_t keep_row64(const Problem& p, int b, int h, i
   return ((uint64_t)hi << 32) | lo;
 }
 
+// 32 keep bits of query token t over the keys of column half hc of key tile
+// kt (bit e is key 64 kt + 32 hc + e): the half of keep_row64 a warp that
+// owns one column half needs.
+__device__ __forceinline__ uint32_t keep_row32(const Problem& p, int b, int h, int t, int kt,
+                                               int hc) {
+  const uint32_t thr4 = keep_thr4(p);
+  return keep_group(p, b, h, t, 4 * kt + 2 * hc, thr4) |
+         (keep_group(p, b, h, t, 4 * kt + 2 * hc + 1, thr4) << 16);
+}
+
 // One element's decision (the CUDA-core kernels).
 __device__ __forceinline__ bool keep_one(const Problem& p, int b, int h, int t, int u) {
   return (keep_group(p, b, h, t, u >> 4, keep_thr4(p)) >> (u & 15)) & 1u;
@@ -100,6 +110,18 @@ __device__ __forceinline__ uint32_t transpose32(uint32_t x, int lane) {
     x = (lane & s) ? ((x & ~m) | ((y >> s) & m)) : ((x & m) | ((y & m) << s));
   }
   return x;
+}
+
+// dK/dV: keep bits of the warp's 32 key tokens u0 .. u0 + 31 (u0 a multiple
+// of 32) against the 32 query tokens t0 .. t0 + 31: bit j of the result is
+// this lane's key u0 + lane against query t0 + j.  All 32 lanes must call it.
+__device__ __forceinline__ uint32_t keep_cols32(const Problem& p, int b, int h, int u0, int t0,
+                                                int lane) {
+  const uint32_t thr4 = keep_thr4(p);
+  const int g = u0 >> 4;
+  const uint32_t r = keep_group(p, b, h, t0 + lane, g, thr4) |
+                     (keep_group(p, b, h, t0 + lane, g + 1, thr4) << 16);
+  return transpose32(r, lane);
 }
 
 // dK/dV: keep bits of the warp's 32 key tokens u0 .. u0 + 31 (u0 a multiple

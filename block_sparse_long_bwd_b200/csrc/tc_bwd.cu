@@ -14,12 +14,16 @@
 //   key tiles) and walk the planned query tiles that attend them (from the
 //   transposed adjacency), each with a group/half mask; the global key
 //   blocks, attended by every query block, are split into chunks of query
-//   tiles.  Per query tile: S^T = K_pair Q^T and dP^T = V_pair dO^T; P^T and
-//   dS^T (bf16) back over them in TMEM; dV += P^T dO and dK += dS^T Q
-//   accumulate in TMEM.  From kSplitMinL the global key blocks run in a
-//   launch of their own with a bf16 low part of P^T and dS^T.  Each key row
-//   is owned by exactly one item (or one chunk partial), so there are no
-//   atomics on data.
+//   tiles.  Per query tile: S^T = K_pair Q^T and dP^T = V_pair dO^T (issued
+//   by a warp of their own into double-buffered TMEM, so a tile's scores
+//   are computed while the softmax works on the one before); P^T and dS^T
+//   (bf16) into TMEM buffers of their own, formed by eight softmax warps,
+//   two per TMEM lane quarter on the two 32-column halves of the tile;
+//   dV += P^T dO and dK += dS^T Q (issued by the MMA warp) accumulate in
+//   TMEM.  One CTA per SM holds all 512 TMEM columns.  From kSplitMinL
+//   the global key blocks run in a launch of their own with a bf16 low part
+//   of P^T and dS^T.  Each key row is owned by exactly one item (or one
+//   chunk partial), so there are no atomics on data.
 // bwd_finish_kernel: sums the chunk partials of the global query rows (dQ)
 //   and of the global key blocks (dK, dV) in a fixed order.
 #include "dropout.cuh"
@@ -30,11 +34,22 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+// 1-CTA-per-SM kernels: warp 0 loads, warp 1 issues the gradient MMAs,
+// warp 2 issues S / dP (S^T / dP^T), warps 3-10 run the softmax, two per
+// SM sub-partition on the two column halves of each tile.  A tcgen05.mma
+// costs its issuing thread ~50 cycles, so the score MMAs get a thread of
+// their own and follow the loads as soon as data and TMEM buffer are ready.
+constexpr int kThreads1 = 352;
+// Per-tile information the loader passes to the score-MMA warp through the
+// stage barriers (written before the stage's expect_tx arrive).
+constexpr int kTinfo = 16;          // ring entries (> stages in flight)
+constexpr uint8_t kTinfoEnd = 0x80; // no more tiles
+// dQ kernel: two CTAs per SM, 192 threads (TMA warp, MMA warp, four
+// softmax warps), 256 TMEM columns each, three K / V stages.
+constexpr int kThreads2 = 192;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kKvStages = 3;
-constexpr int kQStages = 3;
-constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // Q, dO, NL, D
+constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // dK/dV: Q, dO, NL, D
 
 struct BwdArgs {
   PairArgs qa;       // items: query side (dq) and, mirrored, key side (dkdv)
@@ -87,6 +102,41 @@ __device__ __forceinline__ void store_grad_row(const Problem& p, void* base, siz
     w.w = pack_bf16(__uint_as_float(src[6]) * mul, __uint_as_float(src[7]) * mul);
     dst[v] = w;
   }
+}
+
+// Half a gradient row: 32 fp32 bit patterns (columns col0 .. col0 + 31)
+// times mul, stored as bf16 (rounded to nearest even) or fp32 as the call
+// asked.
+__device__ __forceinline__ void store_grad_half(const Problem& p, void* base, size_t row,
+                                                int col0, const uint32_t (&v)[32],
+                                                float mul) {
+  if (p.grad_f32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(base) + row * kHeadDim + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      dst[i] = make_float4(__uint_as_float(v[4 * i]) * mul, __uint_as_float(v[4 * i + 1]) * mul,
+                           __uint_as_float(v[4 * i + 2]) * mul,
+                           __uint_as_float(v[4 * i + 3]) * mul);
+    return;
+  }
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(base) + row * kHeadDim + col0);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t* x = v + 8 * i;
+    dst[i] = make_uint4(pack_bf16(__uint_as_float(x[0]) * mul, __uint_as_float(x[1]) * mul),
+                        pack_bf16(__uint_as_float(x[2]) * mul, __uint_as_float(x[3]) * mul),
+                        pack_bf16(__uint_as_float(x[4]) * mul, __uint_as_float(x[5]) * mul),
+                        pack_bf16(__uint_as_float(x[6]) * mul, __uint_as_float(x[7]) * mul));
+  }
+}
+
+// 32 fp32 values (bit patterns) to consecutive floats of a partial row.
+__device__ __forceinline__ void store_part32(float* dst, const uint32_t (&v)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
 }
 
 // ======================= dQ =======================
@@ -149,7 +199,7 @@ struct DqBars {
 };
 
 template <bool kDrop>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads2, 2)
     tc_dq_kernel(const __grid_constant__ BwdArgs ba,
                  const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK,
@@ -539,10 +589,30 @@ __device__ __forceinline__ void walk_range(const Problem& p, const Geom& g,
   e1 = max(e0, min(e0 + p.kof[2 * k + 1], p.kcap));
 }
 
+// The dK/dV kernel runs one CTA per SM with all 512 TMEM columns:
+//   acc (dK 0-63, dV 64-127), S^T[2] (128-255), dP^T[2] (256-383),
+//   P^T[2] (bf16 pairs, 384-447), dS^T[2] (bf16 pairs, 448-511).
+// Query tile g uses buffers g & 1.  P^T and dS^T have columns of their own,
+// so S^T / dP^T of tile g + 2 are computed as soon as the softmax has read
+// tile g's (and while it still works on it); the dV / dK MMAs of tile g
+// read P^T / dS^T, which the softmax of tile g + 2 overwrites only after
+// those MMAs completed.  With the hi/lo split (global key blocks at long
+// lengths) the low parts go over S^T / dP^T of the same tile, so there the
+// next S^T / dP^T of the buffer also waits for the dV / dK MMAs.
+constexpr int kKvQStages = 8;  // query-tile stages (Q, dO, NL, D)
+constexpr uint32_t kKvTmemCols = 512;
+constexpr uint32_t kKvDK = 0, kKvDV = 64, kKvS = 128, kKvDP = 256, kKvP = 384, kKvDS = 448;
+
 struct KvBars {
-  uint64_t kp_full, kp_empty;
-  uint64_t qt_full[kQStages], qt_empty[kQStages];
-  uint64_t s_full, p_full, acc_full, acc_empty;
+  // K / V pair of item k in slot k & 1: kp_full = landed (and kitem[] of the
+  // slot published); kp_empty = its last S^T / dP^T MMAs completed and the
+  // MMA warp and the four softmax warps have read kitem[].
+  uint64_t kp_full[2], kp_empty[2];
+  uint64_t qt_full[kKvQStages], qt_empty[kKvQStages];
+  // per tile buffer b: S^T / dP^T computed; read by the softmax; P^T / dS^T
+  // written; the dV / dK MMAs that read them completed
+  uint64_t s_full[2], s_free[2], p_full[2], g_done[2];
+  uint64_t acc_full, acc_empty;
 };
 
 // kSplit: bf16 hi/lo split of the global key blocks' P^T and dS^T, for
@@ -552,7 +622,7 @@ struct KvBars {
 // kDrop: seeded attention dropout (P^T kept times 1 / keep probability for
 // dV; dS^T = P^T (m dP^T - D)).
 template <bool kSplit, bool kDrop>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads1, 1)
     tc_dkdv_kernel(const __grid_constant__ BwdArgs ba,
                    const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
@@ -560,7 +630,10 @@ __global__ void __launch_bounds__(kThreads, 2)
                    const __grid_constant__ CUtensorMap tmG) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ KvBars bars;
-  __shared__ int4 kitem[2];  // (b, h, loc, 1) of item k in slot k & 1; w = 0: no more items
+  __shared__ int4 kitem[2];  // (b, h, loc, 1) of the item in pair slot s; w = 0: no more items
+  // flat tile g at g % kTinfo: pair slot | kp_full parity << 1 | last tile
+  // of its item << 2, or kTinfoEnd
+  __shared__ uint8_t tinfo[kTinfo];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -568,26 +641,31 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* base = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint8_t* Ks = base;                      // [128][64] K pair
-  uint8_t* Vs = base + 2 * kTileBytes;     // [128][64] V pair
-  uint8_t* QT = base + 4 * kTileBytes;     // [stage][Q | dO | NL[64] | D[64]]
+  // [2 slots][K pair (2 tiles) | V pair (2 tiles)], then the query stages
+  // [Q | dO | NL[64] | D[64]].
+  uint8_t* KV = base;
+  uint8_t* QT = base + 2 * 4 * kTileBytes;
 
   if (threadIdx.x == 0) {
     abort_flag = 0;
-    mbar_init(&bars.kp_full, 1);
-    mbar_init(&bars.kp_empty, 1);
-    for (int s = 0; s < kQStages; ++s) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars.kp_full[s], 1);
+      mbar_init(&bars.kp_empty[s], 10);  // last S^T commit + MMA warp + 8 softmax warps
+      mbar_init(&bars.s_full[s], 1);
+      mbar_init(&bars.s_free[s], 8);
+      mbar_init(&bars.p_full[s], 8);
+      mbar_init(&bars.g_done[s], 1);
+    }
+    for (int s = 0; s < kKvQStages; ++s) {
       mbar_init(&bars.qt_full[s], 1);
       mbar_init(&bars.qt_empty[s], 1);
     }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.p_full, 4);
     mbar_init(&bars.acc_full, 1);
-    mbar_init(&bars.acc_empty, 4);
+    mbar_init(&bars.acc_empty, 8);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_alloc(&tmem_base_sh, kKvTmemCols);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -600,50 +678,60 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t tDK = tmem, tDV = tmem + 64, tS = tmem + 128, tDP = tmem + 192;
 
   if (warp == 0) {
+    // ---------------- loads (one thread) ----------------
     if (lane == 0) {
-      uint32_t g = 0;
-      int kp_issued = 0;
-      uint32_t kp_par = 0;
+      uint32_t gq = 0;  // query stages loaded (flat tiles)
+      int kp_issued[2] = {0, 0};
+      uint32_t kp_par[2] = {0, 0};
+      bool ok = true;
       for (int k = 0;; ++k) {
-        if (!mbar_wait(&bars.kp_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
+        const int ps = k & 1;
+        // Pair slot ps held item k - 2: released once its last S^T / dP^T
+        // completed and every role has read kitem[].
+        if (!mbar_wait(&bars.kp_empty[ps], ((k >> 1) & 1) ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
         // Items are taken from the launch's counter (middle windows first);
         // the slot's (b, h, loc) is published by the kp_full arrive.
         int ib, ih, iloc;
         if (!next_work(ba.qa.geo, p.B, p.H, ba.kloc0, ba.kgeo.per_bh, ba.kctr, ib, ih,
                        iloc)) {
-          kitem[k & 1] = make_int4(0, 0, 0, 0);
-          mbar_arrive_release(&bars.kp_full);
+          kitem[ps] = make_int4(0, 0, 0, 0);
+          mbar_arrive_release(&bars.kp_full[ps]);
           break;
         }
-        kitem[k & 1] = make_int4(ib, ih, iloc, 1);
+        kitem[ps] = make_int4(ib, ih, iloc, 1);
         const ItemMeta it = item_meta_at(ba.qa.geo, ib, ih, p.H, iloc);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.qa.geo, it, e0, e1);
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
-        mbar_expect_tx(&bars.kp_full, 2u * nh * kTileBytes);
+        uint8_t* kv = KV + ps * 4 * kTileBytes;
+        mbar_expect_tx(&bars.kp_full[ps], 2u * nh * kTileBytes);
         for (int hh = 0; hh < nh; ++hh) {
           const int y = row0 + it.t[hh] * kTile;
-          tma_load_2d(Ks + hh * kTileBytes, &tmK, &bars.kp_full, 0, y);
-          tma_load_2d(Vs + hh * kTileBytes, &tmV, &bars.kp_full, 0, y);
+          tma_load_2d(kv + hh * kTileBytes, &tmK, &bars.kp_full[ps], 0, y);
+          tma_load_2d(kv + (2 + hh) * kTileBytes, &tmV, &bars.kp_full[ps], 0, y);
         }
-        kp_issued = 1;
-        kp_par = k & 1;
-        bool ok = true;
+        kp_issued[ps] = 1;
+        kp_par[ps] = (k >> 1) & 1;
+        if (e1 == e0) mma_commit(&bars.kp_empty[ps]);  // no MMA reads this pair
         uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
         for (int e = e0; e < e1; ++e) {
           const int i = (int)(nxt & 0xFFFFu);  // query tile
           if (e + 1 < e1) nxt = __ldg(walk + e + 1);
-          const int st = g % kQStages;
-          if (!mbar_wait(&bars.qt_empty[st], ((g / kQStages) & 1) ^ 1,
-                         &abort_flag, p.status)) {
+          const uint32_t g = gq;
+          const uint32_t st = g % kKvQStages;
+          if (!mbar_wait(&bars.qt_empty[st], ((g / kKvQStages) & 1) ^ 1, &abort_flag,
+                         p.status)) {
             ok = false;
             break;
           }
+          tinfo[g % kTinfo] = (uint8_t)(ps | (((k >> 1) & 1) << 1) | (e == e1 - 1 ? 4 : 0));
           uint8_t* q = QT + st * kQStageBytes;
           mbar_expect_tx(&bars.qt_full[st], 2 * kTileBytes + 512);
           const int y = row0 + i * kTile;
@@ -651,127 +739,154 @@ __global__ void __launch_bounds__(kThreads, 2)
           tma_load_2d(q + kTileBytes, &tmG, &bars.qt_full[st], 0, y);
           bulk_load(q + 2 * kTileBytes, ba.NL + y, 256, &bars.qt_full[st]);
           bulk_load(q + 2 * kTileBytes + 256, ba.D + y, 256, &bars.qt_full[st]);
-          ++g;
+          ++gq;
         }
         if (!ok) break;
       }
+      // No more tiles: tell the score-MMA warp through the next stage.
+      if (ok) {
+        const uint32_t st = gq % kKvQStages;
+        if (mbar_wait(&bars.qt_empty[st], ((gq / kKvQStages) & 1) ^ 1, &abort_flag, p.status)) {
+          tinfo[gq % kTinfo] = kTinfoEnd;
+          mbar_arrive_release(&bars.qt_full[st]);
+        }
+      }
       if (abort_flag) {
-        for (uint32_t s = 0; s < (uint32_t)kQStages; ++s) {
-          if (g < s + 1) continue;
-          const uint32_t last = g - 1 - ((g - 1 - s) % kQStages);
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(&bars.qt_full[s], (last / kQStages) & 1) &&
-                 globaltimer() - t0 < 100000000ull) {
+        for (uint32_t s = 0; s < (uint32_t)kKvQStages; ++s)
+          if (gq >= s + 1) {
+            const uint32_t last = gq - 1 - ((gq - 1 - s) % kKvQStages);
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&bars.qt_full[s], (last / kKvQStages) & 1) &&
+                   globaltimer() - t0 < 100000000ull) {
+            }
           }
-        }
-        if (kp_issued) {
-          const uint64_t t0 = globaltimer();
-          while (!mbar_try_wait(&bars.kp_full, kp_par) &&
-                 globaltimer() - t0 < 100000000ull) {
+        for (int s = 0; s < 2; ++s)
+          if (kp_issued[s]) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&bars.kp_full[s], kp_par[s]) &&
+                   globaltimer() - t0 < 100000000ull) {
+            }
           }
-        }
+      }
+    }
+  } else if (warp == 2) {
+    // -------- S^T = K Q^T, dP^T = V dO^T (one thread) --------
+    if (lane == 0) {
+      const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+      for (uint32_t g = 0;; ++g) {
+        const int b = g & 1;
+        const uint32_t st = g % kKvQStages;
+        if (!mbar_wait(&bars.qt_full[st], (g / kKvQStages) & 1, &abort_flag, p.status)) break;
+        const int ti = tinfo[g % kTinfo];
+        if (ti & kTinfoEnd) break;
+        const int ps = ti & 1;
+        if (!mbar_wait(&bars.kp_full[ps], (ti >> 1) & 1, &abort_flag, p.status) ||
+            !mbar_wait(&bars.s_free[b], ((g >> 1) & 1) ^ 1, &abort_flag, p.status) ||
+            (kSplit &&
+             !mbar_wait(&bars.g_done[b], ((g >> 1) & 1) ^ 1, &abort_flag, p.status)))
+          break;
+        tc_fence_after();
+        const uint32_t kaddr = smem_u32(KV + ps * 4 * kTileBytes);
+        const uint32_t vaddr = kaddr + 2 * kTileBytes;
+        const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
+        const uint32_t gaddr = qaddr + kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kKvS + b * 64, sdesc_sw128(kaddr + kk * 32, 16),
+                 sdesc_sw128(qaddr + kk * 32, 16), idS, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kKvDP + b * 64, sdesc_sw128(vaddr + kk * 32, 16),
+                 sdesc_sw128(gaddr + kk * 32, 16), idS, kk > 0);
+        mma_commit(&bars.s_full[b]);
+        if (ti & 4) mma_commit(&bars.kp_empty[ps]);  // the pair's last reader
       }
     }
   } else if (warp == 1) {
-    const uint32_t idS = idesc_bf16(128, 64, 0, 0);
+    // ---------- dV += P^T dO, dK += dS^T Q (one thread) ----------
     const uint32_t idAcc = idesc_bf16(128, 64, 0, 1);
-    const uint32_t kaddr = smem_u32(Ks), vaddr = smem_u32(Vs);
-    uint32_t g = 0, u = 0;
+    uint32_t u = 0, ai = 0;  // flat tile counter, items with tiles
     bool ok = true;
     for (int k = 0; ok; ++k) {
-      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
-      const int4 wi = kitem[k & 1];
+      const int ps = k & 1;
+      if (!mbar_wait(&bars.kp_full[ps], (k >> 1) & 1, &abort_flag, p.status)) break;
+      const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
       int w0, w1;
       walk_range(p, ba.qa.geo, it, w0, w1);
       const int nwalk = w1 - w0;
-      tc_fence_after();
-      for (int t = 0; t < nwalk;) {
-        const int st = g % kQStages;
-        // S^T and dP^T overwrite the buffers that hold the previous tile's
-        // P^T and dS^T; the dV / dK MMAs reading those were issued earlier by
-        // this thread and execute first (in-order), so no completion wait.
-        if (!mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
-                       p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
-        const uint32_t gaddr = qaddr + kTileBytes;
-        if (lane == 0) {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tS, sdesc_sw128(kaddr + kk * 32, 16),
-                   sdesc_sw128(qaddr + kk * 32, 16), idS, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tDP, sdesc_sw128(vaddr + kk * 32, 16),
-                   sdesc_sw128(gaddr + kk * 32, 16), idS, kk > 0);
-          mma_commit(&bars.s_full);
-        }
-        __syncwarp();
-        if (!mbar_wait(&bars.p_full, u & 1, &abort_flag, p.status) ||
-            (t == 0 &&
-             !mbar_wait(&bars.acc_empty, (k & 1) ^ 1, &abort_flag, p.status))) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
+      for (int t = 0; t < nwalk; ++t) {
+        const uint32_t g = u;
+        const int b = g & 1;
+        const uint32_t st = g % kKvQStages;
+        if (!mbar_wait(&bars.p_full[b], (g >> 1) & 1, &abort_flag, p.status) ||
+            (t == 0 && !mbar_wait(&bars.acc_empty, (ai & 1) ^ 1, &abort_flag, p.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
         if (lane == 0) {
-          // P^T / dS^T columns: K step kk (16 query rows) at kk * 8, plus 16
-          // for the second query half; low parts 16 columns further.
+          const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
+          const uint32_t gaddr = qaddr + kTileBytes;
+          // A operands: 16 query rows per K step = 8 TMEM columns of bf16
+          // pairs; the low parts of a split tile sit in the S^T / dP^T
+          // columns of the same buffer, query half hc at columns 32 hc ..
+          // 32 hc + 15.
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tDV, tS + kk * 8 + (kk >> 1) * 16, sdesc_sw128(gaddr + kk * 2048, 8192),
-                   idAcc, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + kKvDV, tmem + kKvP + b * 32 + kk * 8,
+                   sdesc_sw128(gaddr + kk * 2048, 8192), idAcc, (t > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16, sdesc_sw128(qaddr + kk * 2048, 8192),
-                   idAcc, (t > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem + kKvDK, tmem + kKvDS + b * 32 + kk * 8,
+                   sdesc_sw128(qaddr + kk * 2048, 8192), idAcc, (t > 0 || kk > 0) ? 1u : 0u);
           if (kSplit && it.global) {
             // Global key blocks sum over every query row: at long lengths
             // their P^T and dS^T also carry a bf16 low part, so the products
             // keep ~16 bits instead of 8.
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ts(tDV, tS + kk * 8 + (kk >> 1) * 16 + 16,
+              mma_ts(tmem + kKvDV, tmem + kKvS + b * 64 + kk * 8 + (kk >> 1) * 16,
                      sdesc_sw128(gaddr + kk * 2048, 8192), idAcc, 1u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ts(tDK, tDP + kk * 8 + (kk >> 1) * 16 + 16,
+              mma_ts(tmem + kKvDK, tmem + kKvDP + b * 64 + kk * 8 + (kk >> 1) * 16,
                      sdesc_sw128(qaddr + kk * 2048, 8192), idAcc, 1u);
           }
+          mma_commit(&bars.g_done[b]);
           mma_commit(&bars.qt_empty[st]);
+          if (t == nwalk - 1) mma_commit(&bars.acc_full);
         }
         __syncwarp();
-        ++g;
         ++u;
-        ++t;
       }
-      if (!ok) break;
-      if (lane == 0) {
-        mma_commit(&bars.acc_full);
-        mma_commit(&bars.kp_empty);
-      }
-      __syncwarp();
+      if (nwalk > 0) ++ai;
     }
   } else {
+    // Softmax warps 3-10: two per TMEM lane quarter (one per SM sub-
+    // partition), each owning one 32-column half (query columns) of the
+    // tile: P^T comes from the stored lse, so no reduction between them.
     const int quarter = warp & 3;
+    const int hc = (warp - 3) >> 2;  // query-column half
     const int row = quarter * 32 + lane;
     const int half = row >> 6, r64 = row & 63;
     const int gshift = 2 * quarter;  // this warp's key-row group = its quarter
     const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
-    uint32_t g = 0, u = 0;
+    uint32_t u = 0, ai = 0;
     for (int k = 0;; ++k) {
+      const int ps = k & 1;
       // The item of this round: published with its K / V pair (kp_full).
-      if (!mbar_wait(&bars.kp_full, k & 1, &abort_flag, p.status)) break;
-      const int4 wi = kitem[k & 1];
+      if (!mbar_wait(&bars.kp_full[ps], (k >> 1) & 1, &abort_flag, p.status)) break;
+      const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
       int e0, e1;
       walk_range(p, ba.qa.geo, it, e0, e1);
@@ -781,143 +896,153 @@ __global__ void __launch_bounds__(kThreads, 2)
       float off = 0.f;
       if (rvalid && p.key_mask)
         off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
+      const bool split = kSplit && it.global;  // bf16 low parts too
       bool ok = true;
       uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
       for (int e = e0; e < e1; ++e) {
         const int mask = (int)(nxt >> 16);
         const int qtile = (int)(nxt & 0xFFFFu);
         if (e + 1 < e1) nxt = __ldg(walk + e + 1);
-        const int st = g % kQStages;
-        if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
+        const uint32_t g = u;
+        const int b = g & 1;
+        const uint32_t st = g % kKvQStages;
+        if (!mbar_wait(&bars.s_full[b], (g >> 1) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int m2 = (mask >> gshift) & 3;  // attending query-column halves
-        const bool split = kSplit && it.global;  // bf16 low parts too
+        // Do query rows of this warp's column half attend this key group?
+        const bool att = (mask >> (gshift + hc)) & 1;
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
-        if (m2 && !mbar_wait(&bars.qt_full[st], (g / kQStages) & 1, &abort_flag,
-                             p.status)) {
+        if (att && !mbar_wait(&bars.qt_full[st], (g / kKvQStages) & 1, &abort_flag,
+                              p.status)) {
           ok = false;
           break;
         }
         const float* NLs =
             reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
         const float* Ds = NLs + 64;
-        // Dropout keep bits of this lane's key against the tile's 64 query
-        // tokens (m2 is uniform over the warp, as the shuffles need).
-        uint32_t keep[2] = {0u, 0u};
-        if (kDrop && m2)
-          keep_cols64(p, it.b, it.h, (int)(ktok & ~(size_t)31), qtile * kTile, lane, keep[0],
-                      keep[1]);
-        // Per query-column half hc (32 columns): read S^T and dP^T, then
-        // write P^T and dS^T (bf16 pairs, 16 columns) over the columns just
-        // read: high parts at 32 hc, low parts (global items) at 32 hc + 16.
+        uint32_t sv[32], dp[32];
+        if (att) {
+          tmem_ld32(tmem + kKvS + b * 64 + hc * 32 + lane_off, sv);
+          tmem_ld32(tmem + kKvDP + b * 64 + hc * 32 + lane_off, dp);
+          tmem_ld_wait();
+        }
+        if (!split) {
+          // S^T / dP^T of this buffer are in registers (with the split the
+          // low parts go back over them, and the score MMAs of the buffer's
+          // next tile wait for the gradient MMAs instead).
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars.s_free[b]);
+        }
+        // Dropout keep bits of this lane's key against the half's 32 query
+        // tokens (att is uniform over the warp, as the shuffles need).
+        const uint32_t keep =
+            (kDrop && att)
+                ? keep_cols32(p, it.b, it.h, (int)(ktok & ~(size_t)31), qtile * kTile + hc * 32,
+                              lane)
+                : 0u;
+        // P^T and dS^T of the half (bf16 pairs, 16 columns each): high parts
+        // to the P^T / dS^T buffers, low parts (split tiles) over the S^T /
+        // dP^T columns just read.
+        uint32_t ph[16], dh[16], pl[16], dl[16];
+        if (att) {
 #pragma unroll
-        for (int hc = 0; hc < 2; ++hc) {
-          uint32_t ph[16], dh[16], pl[16], dl[16];
-          if ((m2 >> hc) & 1) {
-            uint32_t sv[32], dp[32];
-            tmem_ld32(tS + hc * 32 + lane_off, sv);
-            tmem_ld32(tDP + hc * 32 + lane_off, dp);
-            tmem_ld_wait();
+          for (int e = 0; e < 32; e += 4) {
+            const int col = hc * 32 + e;
+            const float4 nl = *reinterpret_cast<const float4*>(NLs + col);
+            const float4 dd = *reinterpret_cast<const float4*>(Ds + col);
+            const float nls[4] = {nl.x, nl.y, nl.z, nl.w};
+            const float dds[4] = {dd.x, dd.y, dd.z, dd.w};
+            float pv[4], dv[4];
+            const float2 c2 = make_float2(c, c), off2 = make_float2(off, off);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const int col = hc * 32 + e;
-              const float4 nl = *reinterpret_cast<const float4*>(NLs + col);
-              const float4 dd = *reinterpret_cast<const float4*>(Ds + col);
-              const float nls[4] = {nl.x, nl.y, nl.z, nl.w};
-              const float dds[4] = {dd.x, dd.y, dd.z, dd.w};
-              float pv[4], dv[4];
-              const float2 c2 = make_float2(c, c), off2 = make_float2(off, off);
-#pragma unroll
-              for (int x = 0; x < 4; x += 2) {
-                // Paired (f32x2) arithmetic, each element rounded as before.
-                const float2 a = fma2(
-                    make_float2(__uint_as_float(sv[e + x]), __uint_as_float(sv[e + x + 1])), c2,
-                    add2(make_float2(nls[x], nls[x + 1]), off2));
-                pv[x] = ex2(a.x);
-                pv[x + 1] = ex2(a.y);
-                if (kDrop) {
-                  // m = 1 / keep probability where kept, 0 where dropped:
-                  // dS = P (m dP - D), and m P enters dV.
-                  const float m0 = ((keep[hc] >> (e + x)) & 1u) ? p.drop_scale : 0.f;
-                  const float m1 = ((keep[hc] >> (e + x + 1)) & 1u) ? p.drop_scale : 0.f;
-                  dv[x] = pv[x] * fmaf(m0, __uint_as_float(dp[e + x]), -dds[x]);
-                  dv[x + 1] = pv[x + 1] * fmaf(m1, __uint_as_float(dp[e + x + 1]), -dds[x + 1]);
-                  pv[x] *= m0;
-                  pv[x + 1] *= m1;
-                } else {
-                  const float2 d = mul2(
-                      make_float2(pv[x], pv[x + 1]),
-                      sub2(make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
-                           make_float2(dds[x], dds[x + 1])));
-                  dv[x] = d.x;
-                  dv[x + 1] = d.y;
-                }
-              }
-#pragma unroll
-              for (int x = 0; x < 2; ++x) {
-                const int o = (e >> 1) + x;
-                ph[o] = pack_bf16(pv[2 * x], pv[2 * x + 1]);
-                dh[o] = pack_bf16(dv[2 * x], dv[2 * x + 1]);
-                if (split) {
-                  pl[o] = pack_bf16(pv[2 * x] - __uint_as_float(ph[o] << 16),
-                                    pv[2 * x + 1] - __uint_as_float(ph[o] & 0xFFFF0000u));
-                  dl[o] = pack_bf16(dv[2 * x] - __uint_as_float(dh[o] << 16),
-                                    dv[2 * x + 1] - __uint_as_float(dh[o] & 0xFFFF0000u));
-                }
+            for (int x = 0; x < 4; x += 2) {
+              // Paired (f32x2) arithmetic, each element rounded as before.
+              const float2 a = fma2(
+                  make_float2(__uint_as_float(sv[e + x]), __uint_as_float(sv[e + x + 1])), c2,
+                  add2(make_float2(nls[x], nls[x + 1]), off2));
+              pv[x] = ex2(a.x);
+              pv[x + 1] = ex2(a.y);
+              if (kDrop) {
+                // m = 1 / keep probability where kept, 0 where dropped:
+                // dS = P (m dP - D), and m P enters dV.
+                const float m0 = ((keep >> (e + x)) & 1u) ? p.drop_scale : 0.f;
+                const float m1 = ((keep >> (e + x + 1)) & 1u) ? p.drop_scale : 0.f;
+                dv[x] = pv[x] * fmaf(m0, __uint_as_float(dp[e + x]), -dds[x]);
+                dv[x + 1] = pv[x + 1] * fmaf(m1, __uint_as_float(dp[e + x + 1]), -dds[x + 1]);
+                pv[x] *= m0;
+                pv[x + 1] *= m1;
+              } else {
+                const float2 d = mul2(
+                    make_float2(pv[x], pv[x + 1]),
+                    sub2(make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
+                         make_float2(dds[x], dds[x + 1])));
+                dv[x] = d.x;
+                dv[x + 1] = d.y;
               }
             }
-          } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ph[e] = dh[e] = pl[e] = dl[e] = 0u;
+            for (int x = 0; x < 2; ++x) {
+              const int o = (e >> 1) + x;
+              ph[o] = pack_bf16(pv[2 * x], pv[2 * x + 1]);
+              dh[o] = pack_bf16(dv[2 * x], dv[2 * x + 1]);
+              if (split) {
+                pl[o] = pack_bf16(pv[2 * x] - __uint_as_float(ph[o] << 16),
+                                  pv[2 * x + 1] - __uint_as_float(ph[o] & 0xFFFF0000u));
+                dl[o] = pack_bf16(dv[2 * x] - __uint_as_float(dh[o] << 16),
+                                  dv[2 * x + 1] - __uint_as_float(dh[o] & 0xFFFF0000u));
+              }
+            }
           }
-          tmem_st16(tS + hc * 32 + lane_off, ph);
-          tmem_st16(tDP + hc * 32 + lane_off, dh);
-          if (split) {
-            tmem_st16(tS + hc * 32 + 16 + lane_off, pl);
-            tmem_st16(tDP + hc * 32 + 16 + lane_off, dl);
-          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) ph[e] = dh[e] = pl[e] = dl[e] = 0u;
+        }
+        // P^T / dS^T buffer b is free once the dV / dK MMAs of tile g - 2
+        // completed.
+        if (!mbar_wait(&bars.g_done[b], ((g >> 1) & 1) ^ 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tmem + kKvP + b * 32 + hc * 16 + lane_off, ph);
+        tmem_st16(tmem + kKvDS + b * 32 + hc * 16 + lane_off, dh);
+        if (split) {
+          tmem_st16(tmem + kKvS + b * 64 + hc * 32 + lane_off, pl);
+          tmem_st16(tmem + kKvDP + b * 64 + hc * 32 + lane_off, dl);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full);
-        ++g;
+        if (lane == 0) {
+          if (split) mbar_arrive(&bars.s_free[b]);
+          mbar_arrive(&bars.p_full[b]);
+        }
         ++u;
       }
       if (!ok) break;
-      if (!mbar_wait(&bars.acc_full, k & 1, &abort_flag, p.status)) break;
+      if (e1 == e0) continue;  // nothing accumulated (not planned)
+      if (!mbar_wait(&bars.acc_full, ai & 1, &abort_flag, p.status)) break;
+      ++ai;
       tc_fence_after();
-      uint32_t k0[32], k1[32], v0[32], v1[32];
-      tmem_ld32(tDK + lane_off, k0);
-      tmem_ld32(tDK + 32 + lane_off, k1);
-      tmem_ld32(tDV + lane_off, v0);
-      tmem_ld32(tDV + 32 + lane_off, v1);
+      uint32_t kx[32], vx[32];
+      tmem_ld32(tmem + kKvDK + hc * 32 + lane_off, kx);
+      tmem_ld32(tmem + kKvDV + hc * 32 + lane_off, vx);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty);
       if (rvalid) {
         if (!it.global) {
-          store_grad_row(p, p.dk, krow, k0, k1, p.scale);
-          store_grad_row(p, p.dv, krow, v0, v1, 1.0f);
+          store_grad_half(p, p.dk, krow, hc * 32, kx, p.scale);
+          store_grad_half(p, p.dv, krow, hc * 32, vx, 1.0f);
         } else {
-          float4* dst = reinterpret_cast<float4*>(
-              ba.kvpart + ((((size_t)it.bh * ba.qa.geo.n_git + it.gi) * ba.qa.geo.nchunks +
-                            it.chunk) * 128 + row) * 128);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            dst[v] = make_float4(__uint_as_float(k0[4 * v]), __uint_as_float(k0[4 * v + 1]),
-                                 __uint_as_float(k0[4 * v + 2]), __uint_as_float(k0[4 * v + 3]));
-            dst[8 + v] = make_float4(__uint_as_float(k1[4 * v]), __uint_as_float(k1[4 * v + 1]),
-                                     __uint_as_float(k1[4 * v + 2]), __uint_as_float(k1[4 * v + 3]));
-            dst[16 + v] = make_float4(__uint_as_float(v0[4 * v]), __uint_as_float(v0[4 * v + 1]),
-                                      __uint_as_float(v0[4 * v + 2]), __uint_as_float(v0[4 * v + 3]));
-            dst[24 + v] = make_float4(__uint_as_float(v1[4 * v]), __uint_as_float(v1[4 * v + 1]),
-                                      __uint_as_float(v1[4 * v + 2]), __uint_as_float(v1[4 * v + 3]));
-          }
+          float* dst = ba.kvpart + ((((size_t)it.bh * ba.qa.geo.n_git + it.gi) *
+                                     ba.qa.geo.nchunks + it.chunk) * 128 + row) * 128;
+          store_part32(dst + hc * 32, kx);
+          store_part32(dst + 64 + hc * 32, vx);
         }
       }
     }
@@ -927,7 +1052,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, kKvTmemCols);
   }
 }
 
@@ -1033,14 +1158,14 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   cudaError_t e = cudaFuncSetAttribute(
       dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
   if (e != cudaSuccess) return e;
-  dq_kernel<<<min(ba.qa.items, 2 * sms), kThreads, smem_dq, s>>>(
+  dq_kernel<<<min(ba.qa.items, 2 * sms), kThreads2, smem_dq, s>>>(
       ba, tm.q, tm.k, tm.v, tm.dout);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = marks->mark(s);
   if (e != cudaSuccess) return e;
 
-  const size_t smem_kv = 1024 + 4 * kTileBytes + kQStages * kQStageBytes;
+  const size_t smem_kv = 1024 + 2 * 4 * kTileBytes + kKvQStages * kQStageBytes;
   // From kSplitMinL the global key blocks' items (the only ones with the
   // hi/lo split) run in a launch of their own, the middle windows without.
   const Geom& g = ba.qa.geo;
@@ -1071,7 +1196,7 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);
     if (e != cudaSuccess) return e;
-    kv_kernel<<<min(bk.kitems, 2 * sms), kThreads, smem_kv, s>>>(
+    kv_kernel<<<min(bk.kitems, sms), kThreads1, smem_kv, s>>>(
         bk, tm.q, tm.k, tm.v, tm.dout);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

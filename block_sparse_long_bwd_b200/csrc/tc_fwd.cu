@@ -41,7 +41,10 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr uint32_t kColS = 0, kColP = 128, kColO = 192;
 
 struct Bars {
-  uint64_t list_full[2], list_empty[2], q_full[2], q_empty[2];
+  // list_full: the tile list's bulk copy landed (producer only);
+  // list_ready: the producer has dropped the item's fully masked key tiles
+  // and publishes the list to the other roles.
+  uint64_t list_full[2], list_ready[2], list_empty[2], q_full[2], q_empty[2];
   uint64_t kv_full[kNST], kv_empty[kNST];
   uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
   // One P V completion barrier per P buffer: P V(u) commits to
@@ -91,6 +94,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.list_full[s], 1);
+      mbar_init(&bars.list_ready[s], 1);
       mbar_init(&bars.list_empty[s], 5);
       mbar_init(&bars.q_full[s], 1);
       mbar_init(&bars.q_empty[s], 1);
@@ -136,11 +140,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         // The item's key-tile list was planned before this kernel: one bulk
         // copy into the slot (the producer waits for it like the others).
         // Items are taken from the launch's counter (middle windows first);
-        // the slot's (b, h, loc) is published by the list_full arrive.
+        // the slot's (b, h, loc) is published by the list_ready arrive.
         int ib, ih, iloc;
         if (!next_work(a.geo, p.B, p.H, 0, a.geo.per_bh, p.sched, ib, ih, iloc)) {
           item_sh[slot] = make_int4(0, 0, 0, 0);
-          mbar_arrive_release(&bars.list_full[slot]);
+          mbar_arrive_release(&bars.list_ready[slot]);
           break;
         }
         item_sh[slot] = make_int4(ib, ih, iloc, 1);
@@ -150,9 +154,29 @@ __global__ void __launch_bounds__(kThreads, 2)
         bulk_load(&lists[slot],
                   static_cast<const TileList*>(p.qplan) + (size_t)m.h * a.geo.per_bh + m.loc,
                   sizeof(TileList), &bars.list_full[slot]);
-        if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status) ||
-            !mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status))
-          break;
+        if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+        if (p.key_mask && p.tdead) {
+          // Drop key tiles whose 64 keys are all masked.  Exact when every
+          // row has a valid attended key (the flag word: a valid key among
+          // the first 32, which lie in block 0, attended by every row): a
+          // masked key's probability is then exp(-10000 + ...) = 0.
+          const uint32_t* dw = p.tdead + (size_t)m.b * p.tdead_words;
+          if (__ldg(dw) & 1u) {
+            TileList& Lw = lists[slot];
+            int n2 = 0;
+            for (int t = 0; t < Lw.n; ++t) {
+              const int j = Lw.tile[t];
+              if ((__ldg(dw + 1 + (j >> 5)) >> (j & 31)) & 1u) continue;
+              Lw.tile[n2] = Lw.tile[t];
+              Lw.mask[n2] = Lw.mask[t];
+              ++n2;
+            }
+            Lw.n = n2;
+            fence_proxy_async_smem();  // before the slot's next bulk copy
+          }
+        }
+        mbar_arrive_release(&bars.list_ready[slot]);
+        if (!mbar_wait(&bars.q_empty[slot], ph ^ 1, &abort_flag, p.status)) break;
         const int row0 = m.bh * p.L;
         const uint32_t qbytes = (m.t[1] >= 0 ? 2u : 1u) * kTileBytes;
         mbar_expect_tx(&bars.q_full[slot], qbytes);
@@ -205,11 +229,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t idS = idesc_bf16(128, 64, 0, 0);   // Q (K-major) x K^T (K-major)
     const uint32_t idPV = idesc_bf16(128, 64, 0, 1);  // P (TMEM) x V (MN-major)
     uint32_t g = 0, u = 0;  // K/V stage counter, tile counter
+    uint32_t oi = 0;        // items with at least one tile (O handed over)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
-      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      if (!mbar_wait(&bars.list_ready[slot], ph, &abort_flag, p.status)) break;
       if (!item_sh[slot].w) break;
       const int n = lists[slot].n;
       if (!mbar_wait(&bars.q_full[slot], ph, &abort_flag, p.status)) break;
@@ -222,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int st = (g + t) % kNST;
         if (!mbar_wait(&bars.p_full[b2], (uu >> 1) & 1, &abort_flag, p.status))
           return false;
-        if (t == 0 && !mbar_wait(&bars.o_empty, (k & 1) ^ 1, &abort_flag, p.status))
+        if (t == 0 && !mbar_wait(&bars.o_empty, (oi & 1) ^ 1, &abort_flag, p.status))
           return false;
         tc_fence_after();
         if (lane == 0) {
@@ -267,6 +292,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
       if (ok && n > 0 && !issue_pv(n - 1)) ok = false;
+      if (n == 0 && lane == 0) mma_commit(&bars.q_empty[slot]);  // nothing read Q
+      __syncwarp();
+      if (n > 0) ++oi;
       g += n;
       u += n;
       if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
@@ -285,12 +313,28 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int k = 0;; ++k) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
-      if (!mbar_wait(&bars.list_full[slot], ph, &abort_flag, p.status)) break;
+      if (!mbar_wait(&bars.list_ready[slot], ph, &abort_flag, p.status)) break;
       const int4 wi = item_sh[slot];
       if (!wi.w) break;
       const TileList& L = lists[slot];
       const ItemMeta im = item_meta_at(a.geo, wi.x, wi.y, p.H, wi.z);
       const int n = L.n;
+      if (n == 0) {
+        // Every key tile of this chunk was masked (only global items can
+        // lose all their tiles: middle items keep tile 0): an empty partial.
+        if (im.global && ((im.gvalid >> quarter) & 1)) {
+          float* part = p.part + ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks +
+                                   im.chunk) * 128 + row) * kPartStride;
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            reinterpret_cast<float4*>(part)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+          part[64] = -INFINITY;
+          part[65] = 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
+        continue;
+      }
       float m = -INFINITY, l = 0.f;
       // Query token of this row (dropout counters; any row when invalid).
       const int tq = (((im.gvalid >> quarter) & 1) ? im.t[half] : 0) * kTile + (row & 63);

@@ -46,9 +46,10 @@ struct Bars {
   // and publishes the list to the other roles.
   uint64_t list_full[2], list_ready[2], list_empty[2], q_full[2], q_empty[2];
   uint64_t kv_full[kNST], kv_empty[kNST];
-  uint64_t s_full[2], s_empty[2], p_full[2], p_empty[2];
-  // One P V completion barrier per P buffer: P V(u) commits to
-  // pv_done[u & 1], so a wait for P V(u) by parity is never confused with
+  uint64_t s_full[2], s_empty[2], p_full[2];
+  // One P V completion barrier per P buffer (it also frees the buffer):
+  // P V(u) commits to pv_done[u & 1], so a wait for P V(u) by parity is
+  // never confused with
   // P V(u - 1), which may still be in flight.
   uint64_t pv_done[2], o_empty;
 };
@@ -101,7 +102,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(&bars.s_full[s], 1);
       mbar_init(&bars.s_empty[s], 4);
       mbar_init(&bars.p_full[s], 4);
-      mbar_init(&bars.p_empty[s], 1);
       mbar_init(&bars.pv_done[s], 1);
     }
     mbar_init(&bars.o_empty, 4);
@@ -258,7 +258,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                    sdesc_sw128(vaddr + kk * 2048, 8192), idPV,
                    (t > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&bars.pv_done[b2]);
-          mma_commit(&bars.p_empty[b2]);
           mma_commit(&bars.kv_empty[st]);
         }
         __syncwarp();
@@ -310,6 +309,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     const float c = p.scale * kLog2e;
     const float mvl = p.mask_value * kLog2e;
     uint32_t u = 0;  // tile counter (same sequence as the MMA warp)
+    // Slot whose output store is in flight (lane 0): the slot is released
+    // (list_empty) once the store has read the staged rows, which is
+    // checked one tile into the next item instead of waiting right away.
+    int pend = -1;
+    auto release_pending = [&]() {
+      if (lane == 0 && pend >= 0) {
+        bulk_wait_read_all();
+        mbar_arrive(&bars.list_empty[pend]);
+      }
+      pend = -1;
+    };
     for (int k = 0;; ++k) {
       const int slot = k & 1;
       const uint32_t ph = (k >> 1) & 1;
@@ -332,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           part[65] = 0.f;
         }
         __syncwarp();
+        release_pending();
         if (lane == 0) mbar_arrive(&bars.list_empty[slot]);
         continue;
       }
@@ -367,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_empty[b2]);
         // P buffer b2 is free once the P V two tiles back has completed.
-        if (!mbar_wait(&bars.p_empty[b2], par ^ 1, &abort_flag, p.status)) {
+        if (!mbar_wait(&bars.pv_done[b2], par ^ 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
@@ -461,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.p_full[b2]);
+        if (t == 0) release_pending();
       }
       if (!ok) break;
       u += n;
@@ -526,10 +538,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                        (int)((size_t)im.bh * p.L + (size_t)im.t[half] * kTile +
                              (quarter & 1) * 32));
           bulk_commit_group();
-          bulk_wait_read_all();  // the slot may be refilled after list_empty
+        } else {
+          mbar_arrive(&bars.list_empty[slot]);
         }
-        mbar_arrive(&bars.list_empty[slot]);
       }
+      if (tma_out) pend = slot;  // released after the store has read the rows
       if (write) {
         if (!im.global) {
           p.lse_out[grow] = (m + __log2f(l)) * (1.0f / kLog2e);

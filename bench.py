@@ -868,13 +868,69 @@ def time_workload(name, steps, dev, flush):
     return rec
 
 
+def time_projections(name, B, L, hidden, H, steps, dev, flush, peaks):
+    """The fused Q/K/V projection and the output projection of a layer
+    (x [B, L, hidden] -> q, k, v [B, H, L, 64]; o -> out [B, L, hidden]),
+    device-timed with CUDA events, L2 flushed between steps; beside them the
+    plain torch (cuBLAS) matmul of the same shapes, without the layout
+    change, for context."""
+    from block_sparse_long_bwd_b200 import binding as bb
+
+    inp = synth.make_proj_inputs(B, L, hidden, H, seed=41)
+    t = {k_: v_.to(dev) for k_, v_ in inp.items()}
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    D = 64 * H
+    q = torch.empty((B, H, L, 64), dtype=torch.bfloat16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    out = torch.empty((B, L, hidden), dtype=torch.bfloat16, device=dev)
+    x2 = t["x"].view(B * L, hidden)
+    o2 = q.permute(0, 2, 1, 3).reshape(B * L, D).contiguous()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        tot = 0.0
+        for s_ in range(steps):
+            flush.fill_(s_ & 0xFF)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        return tot / steps
+
+    ms_qkv = timed(lambda: bb.bb_qkv_proj(t["x"], t["w_qkv"], t["b_qkv"], H, ws, q, k, v,
+                                          stream=stream))
+    ms_out = timed(lambda: bb.bb_out_proj(q, t["w_o"], t["b_o"], ws, out, stream=stream))
+    ms_qkv_ref = timed(lambda: torch.addmm(t["b_qkv"].to(torch.bfloat16), x2, t["w_qkv"].t()))
+    ms_out_ref = timed(lambda: torch.addmm(t["b_o"].to(torch.bfloat16), o2, t["w_o"].t()))
+    st = bb.bb_attn_check_status(ws)
+    fl_qkv = 2.0 * B * L * 3 * D * hidden
+    fl_out = 2.0 * B * L * hidden * D
+    tf = lambda fl, ms: round(fl / (ms / 1e3) / 1e12, 2)
+    return {"workload": name, "B": B, "L": L, "hidden": hidden, "H": H, "status": st,
+            "qkv_ms": round(ms_qkv, 5), "qkv_tflops": tf(fl_qkv, ms_qkv),
+            "qkv_frac_of_peak": round(fl_qkv / (ms_qkv / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "out_ms": round(ms_out, 5), "out_tflops": tf(fl_out, ms_out),
+            "out_frac_of_peak": round(fl_out / (ms_out / 1e3) / 1e12 / peaks["bf16_tflops"], 4),
+            "torch_matmul_same_shapes_ms": {"qkv": round(ms_qkv_ref, 5),
+                                            "out": round(ms_out_ref, 5)}}
+
+
 def sub_records(dev, peaks, sweep_steps=5):
     """The other workloads and the sweep, timed in the same run after the
     headline: the BigBird-base forward (its padded batch), the 16K pattern
-    (fwd+bwd), and every sweep point with the linear-in-L verdict."""
+    (fwd+bwd), the layer's projections at the BigBird-large and -base
+    widths, and every sweep point with the linear-in-L verdict."""
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     subs = {n: time_workload(n, 10, dev, flush)
             for n in ("base_fwd_l4096", "long_l16384")}
+    subs["projections"] = [
+        time_projections("bigbird_large_layer_l4096", 4, 4096, 1024, 16, 10, dev, flush, peaks),
+        time_projections("bigbird_base_layer_l4096", 8, 4096, 768, 12, 10, dev, flush, peaks)]
     rows = []
     for bs in synth.SWEEP_BS:
         for r in synth.SWEEP_R:

@@ -92,6 +92,10 @@ def lib():
         L.bb_attn_fwd_noalloc.argtypes = [ctypes.POINTER(bb_attn_desc)] + [
             _P] * 8
         L.bb_attn_fwd_noalloc.restype = ctypes.c_int
+        L.bb_qkv_proj.argtypes = [ctypes.c_int] * 4 + [_P] * 7 + [ctypes.c_size_t, _P]
+        L.bb_qkv_proj.restype = ctypes.c_int
+        L.bb_out_proj.argtypes = [ctypes.c_int] * 4 + [_P] * 5 + [ctypes.c_size_t, _P]
+        L.bb_out_proj.restype = ctypes.c_int
         L.bb_attn_noalloc_status.argtypes = [_P]
         L.bb_attn_noalloc_status.restype = ctypes.c_int
         L.bb_attn_check_status.argtypes = [_P, _P]
@@ -271,6 +275,49 @@ def bb_attn_bwd(desc, q, k, v, out, lse, dout, key_mask, rand_idx, dq, dk, dv,
     else:
         arr, n = _event_array(events)
         _check(lib().bb_attn_bwd_events(*args, arr, n), "bb_attn_bwd_events")
+
+
+def bb_qkv_proj(x, w_qkv, b_qkv, H, workspace, q=None, k=None, v=None, stream=None):
+    """Fused Q/K/V projection (see include/bb_attn.h): x [B, L, hidden] bf16,
+    w_qkv [3*H*64, hidden] bf16, b_qkv [3*H*64] fp32 or None; returns q, k, v
+    [B, H, L, 64] bf16."""
+    B, L, hidden = x.shape
+    _cuda_tensor(x, "x", torch.bfloat16)
+    _cuda_tensor(w_qkv, "w_qkv", torch.bfloat16)
+    if b_qkv is not None:
+        _cuda_tensor(b_qkv, "b_qkv", torch.float32)
+    _cuda_tensor(workspace, "workspace")
+    out = []
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t is None:
+            t = torch.empty((B, H, L, 64), dtype=torch.bfloat16, device=x.device)
+        _cuda_tensor(t, name, torch.bfloat16)
+        out.append(t)
+    _check(lib().bb_qkv_proj(B, L, hidden, H, _ptr(x), _ptr(w_qkv), _ptr(b_qkv),
+                             _ptr(out[0]), _ptr(out[1]), _ptr(out[2]), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(),
+                             _stream_ptr(stream)), "bb_qkv_proj")
+    return tuple(out)
+
+
+def bb_out_proj(o, w_o, b_o, workspace, out=None, stream=None):
+    """Output projection (see include/bb_attn.h): o [B, H, L, 64] bf16,
+    w_o [hidden, H*64] bf16, b_o [hidden] fp32 or None; returns out
+    [B, L, hidden] bf16."""
+    B, H, L, d = o.shape
+    hidden = w_o.shape[0]
+    _cuda_tensor(o, "o", torch.bfloat16)
+    _cuda_tensor(w_o, "w_o", torch.bfloat16)
+    if b_o is not None:
+        _cuda_tensor(b_o, "b_o", torch.float32)
+    _cuda_tensor(workspace, "workspace")
+    if out is None:
+        out = torch.empty((B, L, hidden), dtype=torch.bfloat16, device=o.device)
+    _cuda_tensor(out, "out", torch.bfloat16)
+    _check(lib().bb_out_proj(B, L, H, hidden, _ptr(o), _ptr(w_o), _ptr(b_o), _ptr(out),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream_ptr(stream)), "bb_out_proj")
+    return out
 
 
 def bb_attn_noalloc_status(stream=None):

@@ -102,6 +102,10 @@ struct TensorMaps {
 // Encodes the maps a pass needs; false if the driver entry point or the
 // encode call fails.
 bool encode_tensor_maps(const Problem& p, int pass, TensorMaps* tm);
+// 2-D bf16 map over [rows][inner] (row stride in elements, a multiple of 8),
+// box box_inner x box_rows, 128-byte swizzle (box_inner = 64).
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride, uint32_t box_inner, uint32_t box_rows);
 
 // Tensor-core path (bf16, block 64, d 64).
 bool tc_fwd_supported(const Problem& p);

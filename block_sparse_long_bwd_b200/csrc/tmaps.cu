@@ -45,6 +45,20 @@ bool encode_rows(CUtensorMap* m, const void* base, uint64_t rows,
 
 }  // namespace
 
+bool encode_bf16_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                    uint64_t row_stride, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool encode_tensor_maps(const Problem& p, int pass, TensorMaps* tm) {
   const uint64_t rows = (uint64_t)p.B * p.H * p.L;
   bool ok = encode_rows(&tm->q, p.q, rows) && encode_rows(&tm->k, p.k, rows) &&

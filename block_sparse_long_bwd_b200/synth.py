@@ -105,3 +105,23 @@ def make_inputs(cfg, with_grad=True, batch_slice=None):
         assert bool((km[:, :bs].sum(dim=1) > 0).all())
     out["key_mask"] = km
     return out
+
+
+def make_proj_inputs(B, L, hidden, H, seed, d=64, bias=True):
+    """Seeded inputs of the projections either side of the attention:
+    drawn in the order x, w_qkv, b_qkv, w_o, b_o from
+    ``torch.Generator().manual_seed(seed)``; x ~ N(0, 1) [B, L, hidden],
+    weights ~ N(0, 1/in_features) (so outputs have unit scale) in the
+    linear-layer layout [out, in], biases ~ N(0, 0.01) fp32 (None when
+    bias=False).  x and the weights are cast to bf16 (round to nearest
+    even); the oracle reads the same values."""
+    g = torch.Generator().manual_seed(seed)
+    D = H * d
+    x = torch.randn((B, L, hidden), generator=g).to(torch.bfloat16)
+    w_qkv = (torch.randn((3 * D, hidden), generator=g) / hidden ** 0.5).to(torch.bfloat16)
+    b_qkv = torch.randn((3 * D,), generator=g) * 0.1
+    w_o = (torch.randn((hidden, D), generator=g) / D ** 0.5).to(torch.bfloat16)
+    b_o = torch.randn((hidden,), generator=g) * 0.1
+    if not bias:
+        b_qkv = b_o = None
+    return {"x": x, "w_qkv": w_qkv, "b_qkv": b_qkv, "w_o": w_o, "b_o": b_o}

@@ -200,6 +200,40 @@ BB_API int bb_attn_bwd(const bb_attn_desc* desc, const void* q, const void* k,
                 const int32_t* rand_idx, void* dq, void* dk, void* dv,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* The projections on either side of the attention in the pages' encoder
+ * layer ([gitcode page] section "两条构建路径：EncoderScaffold 与
+ * BigBirdEncoder": the layer is a transformer block around BigBirdAttention
+ * with key_dim = hidden / heads), on tcgen05 tensor cores.  Head dim 64.
+ * Weights follow the linear-layer convention W[out_features][in_features];
+ * bias is fp32 [out_features] or NULL (no bias).  Accumulation is fp32; the
+ * bf16 results are rounded to nearest even once.
+ *
+ * Fused Q/K/V projection: with D = H * 64,
+ *   q[b][h][l][j] = b_qkv[h*64 + j]       + sum_c x[b][l][c] w_qkv[h*64 + j][c]
+ *   k[b][h][l][j] = b_qkv[D + h*64 + j]   + sum_c x[b][l][c] w_qkv[D + h*64 + j][c]
+ *   v[b][h][l][j] = b_qkv[2D + h*64 + j]  + sum_c x[b][l][c] w_qkv[2D + h*64 + j][c]
+ *   x      [B][L][hidden] bf16, device
+ *   w_qkv  [3 * H * 64][hidden] bf16, device;  b_qkv [3 * H * 64] fp32 or NULL
+ *   q, k, v [B][H][L][64] bf16, device (written): the layout bb_attn_fwd reads
+ * Requires L % 128 == 0, hidden % 64 == 0 and H % 4 == 0 (BigBird-base and
+ * -large: hidden 768 / 1024, H 12 / 16), else BB_ERR_UNSUPPORTED.
+ * workspace: device, >= 256 bytes, 16-byte aligned; holds the status word
+ * (bb_attn_check_status).  Asynchronous on `stream`. */
+BB_API int bb_qkv_proj(int B, int L, int hidden, int H, const void* x, const void* w_qkv,
+                       const float* b_qkv, void* q, void* k, void* v, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/* Output projection of the attention output o [B][H][L][64] (as bb_attn_fwd
+ * writes it):
+ *   out[b][l][n] = b_o[n] + sum_{h, j} o[b][h][l][j] w_o[n][h*64 + j]
+ *   w_o [hidden][H * 64] bf16, device;  b_o [hidden] fp32 or NULL
+ *   out [B][L][hidden] bf16, device (written)
+ * Requires L % 128 == 0 and hidden % 256 == 0, else BB_ERR_UNSUPPORTED.
+ * workspace as for bb_qkv_proj. */
+BB_API int bb_out_proj(int B, int L, int H, int hidden, const void* o, const void* w_o,
+                       const float* b_o, void* out, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
 /* Number of kernel launches bb_attn_fwd (pass 0) or bb_attn_bwd (pass 1)
  * makes for `desc`, written to *launches.  Host only. */
 BB_API int bb_attn_launch_count(const bb_attn_desc* desc, int pass,

@@ -11,8 +11,10 @@ from .bigbird_oracle import (  # noqa: F401
     dropout_scale,
     dropout_threshold,
     forward,
+    output_projection,
     pair_count,
     philox4x32_10,
+    qkv_projection,
     rand_table,
     random_candidates,
 )

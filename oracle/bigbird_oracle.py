@@ -80,7 +80,8 @@ properties; tests/test_dropout_oracle.py checks the dropout generator
 against the published Philox4x32-10 known-answer vectors and the dropped
 forward and backward against dense torch fp64 with autograd and finite
 differences; tests/test_query_mask_oracle.py does the same for the query
-mask.
+mask; tests/test_proj_oracle.py checks the projections against explicit
+element-by-element sums and identity-weight read-outs.
 """
 
 import math
@@ -407,3 +408,49 @@ def pair_count(num_blocks, table_h):
     """Number of attended (query block, key block) pairs for one head."""
     return sum(len(attended_blocks(i, num_blocks, table_h[i]))
                for i in range(num_blocks))
+
+
+# ---------------------------------------------------------------------------
+# The projections on either side of the attention.
+#
+# [GC] section "两条构建路径：EncoderScaffold 与 BigBirdEncoder": the encoder
+# layer is a transformer block whose attention is BigBirdAttention, with
+# key_dim = hidden / num_heads; its query, key and value are dense layers of
+# the layer input, split into heads, and its output is a dense layer of the
+# concatenated heads.  Written here as plain fp64 matrix products with the
+# linear-layer weight convention W[out_features][in_features].
+# ---------------------------------------------------------------------------
+
+
+def qkv_projection(x, w_qkv, b_qkv, heads, head_dim=64):
+    """q, k, v [B, H, L, head_dim] of x [B, L, hidden].
+
+    w_qkv [3 * H * head_dim, hidden]: rows 0 .. D-1 produce the query
+    features (D = H * head_dim; feature h * head_dim + j is component j of
+    head h), rows D .. 2D-1 the key features, rows 2D .. 3D-1 the value
+    features; b_qkv [3D] or None."""
+    x = _prep(x)
+    w = _prep(w_qkv)
+    B, L, _ = x.shape
+    D = heads * head_dim
+    y = x @ w.T
+    if b_qkv is not None:
+        y = y + _prep(b_qkv)
+    out = []
+    for part in range(3):
+        z = y[:, :, part * D:(part + 1) * D].reshape(B, L, heads, head_dim)
+        out.append(np.ascontiguousarray(z.transpose(0, 2, 1, 3)))
+    return tuple(out)
+
+
+def output_projection(o, w_o, b_o):
+    """out [B, L, hidden] of the attention output o [B, H, L, head_dim]:
+    the heads concatenated per token (feature h * head_dim + j), times
+    w_o [hidden, H * head_dim] transposed, plus b_o [hidden] or None."""
+    o = _prep(o)
+    B, H, L, d = o.shape
+    cat = o.transpose(0, 2, 1, 3).reshape(B, L, H * d)
+    y = cat @ _prep(w_o).T
+    if b_o is not None:
+        y = y + _prep(b_o)
+    return y

@@ -253,3 +253,25 @@ def test_host_calls_are_reentrant_across_threads():
     for t in threads:
         t.join()
     assert not errors, errors
+
+
+def test_projection_argument_checks_without_a_gpu():
+    """The projection entry points validate before touching any pointer or
+    calling CUDA: NULL or misaligned pointers, sizes the tiles do not cover,
+    a missing or short workspace."""
+    lib = bb.lib()
+    P = 1 << 20  # a fake 16-byte aligned address, never dereferenced
+    ws = P
+    # NULL input / misaligned pointer
+    assert lib.bb_qkv_proj(1, 128, 768, 12, None, P, None, P, P, P, ws, 256, None) == -1
+    assert lib.bb_qkv_proj(1, 128, 768, 12, P + 2, P, None, P, P, P, ws, 256, None) == -1
+    assert lib.bb_out_proj(1, 128, 12, 768, None, P, None, P, ws, 256, None) == -1
+    # shapes: L % 128, hidden % 64, H % 4 (QKV); hidden % 256 (output)
+    assert lib.bb_qkv_proj(1, 100, 768, 12, P, P, None, P, P, P, ws, 256, None) == -2
+    assert lib.bb_qkv_proj(1, 128, 770, 12, P, P, None, P, P, P, ws, 256, None) == -2
+    assert lib.bb_qkv_proj(1, 128, 768, 6, P, P, None, P, P, P, ws, 256, None) == -2
+    assert lib.bb_out_proj(1, 128, 12, 640, P, P, None, P, ws, 256, None) == -2
+    assert lib.bb_qkv_proj(0, 128, 768, 12, P, P, None, P, P, P, ws, 256, None) == -1
+    # workspace
+    assert lib.bb_qkv_proj(1, 128, 768, 12, P, P, None, P, P, P, None, 256, None) == -4
+    assert lib.bb_out_proj(1, 128, 12, 768, P, P, None, P, ws, 64, None) == -4

@@ -84,6 +84,8 @@ def parse():
     # Leave out the sub-records (the other workloads and the sweep, timed
     # after the headline on rank 0).
     ap.add_argument("--skip-sub", action="store_true")
+    # Time only the layer's projections (BigBird-large widths); for profiling.
+    ap.add_argument("--proj-only", action="store_true")
     # Sweep mode: one line per (L, block, r) point of the length / block /
     # random-count sweep (B*L = 32768 tokens, H = 12), then the linear-in-L
     # check; not the headline line.
@@ -951,6 +953,14 @@ def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.proj_only:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        peaks, _ = load_peaks()
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        print(json.dumps(time_projections("bigbird_large_layer_l4096", 4, 4096, 1024, 16,
+                                          max(1, args.steps), dev, flush, peaks)), flush=True)
         return
     world, rank, local = init_dist(args)
     try:

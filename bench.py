@@ -50,15 +50,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 # captured, that file, the workload captured).  Another workload or a
 # changed source reports null.
 NCU_TRAFFIC = {
-    # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, 1 launch;
-    # hashes of the sources the counters were taken on: they no longer match
-    # since the dropout and query-mask variants, so the figure reads null
-    # until a new capture)
-    "tc_fwd": (147637504 + 31209472, "0f41c4d9c5be114a", "tc_fwd.cu",
+    # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, one
+    # launch each, captured on the sources these hashes describe)
+    "tc_fwd": (148775424 + 31886336, "3821985e8dd14902", "tc_fwd.cu",
                "large_train_l4096"),
-    "tc_dq": (224994560 + 33675264, "44becb5d0e98a1ed", "tc_bwd.cu",
+    "tc_dq": (225114624 + 33682688, "9db64f7eace72bc5", "tc_bwd.cu",
               "large_train_l4096"),
-    "tc_dkdv": (200701696 + 64869376, "44becb5d0e98a1ed", "tc_bwd.cu",
+    "tc_dkdv": (202466560 + 65625856, "9db64f7eace72bc5", "tc_bwd.cu",
                 "large_train_l4096"),
 }
 

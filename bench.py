@@ -73,6 +73,9 @@ def parse():
     # 0, the default, is the plain operation the headline line times).
     ap.add_argument("--dropout", type=float, default=0.0)
     ap.add_argument("--dropout-seed", type=int, default=0)
+    # With dropout: draw the keep decisions in every pass instead of having
+    # the forward store them for the backward (the default).
+    ap.add_argument("--redraw-dropout", action="store_true")
     # With a masked workload: the key mask also zeroes the output rows of
     # padding tokens (off by default).
     ap.add_argument("--mask-queries", action="store_true")
@@ -263,19 +266,22 @@ def aggregate_tokens_per_s(tokens_per_rank, steps, max_total_ms, world):
     return tokens_per_rank * world * steps / (max_total_ms / 1e3)
 
 
-def algorithmic(cfg, pairs_total):
-    """Algorithmic FLOPs and bytes per launch of each kernel kind."""
+def algorithmic(cfg, pairs_total, keep_bits=False):
+    """Algorithmic FLOPs and bytes per launch of each kernel kind.
+    keep_bits: the forward stores one dropout keep bit per attended element
+    and the two backward passes read them."""
     B, H, L, d, bs = cfg["B"], cfg["H"], cfg["L"], cfg["d"], cfg["block_size"]
     e = 2 if cfg["dtype"] == "bf16" else 4
     rows = B * H * L
     elems = rows * d
     unit = pairs_total * bs * bs * d  # one bs x bs x d contraction per pair
+    kb = pairs_total * bs * bs // 8 if keep_bits else 0
     return {
-        "fwd": (4 * unit, 4 * elems * e + 4 * rows),
+        "fwd": (4 * unit, 4 * elems * e + 4 * rows + kb),
         "bwd_pre": (0, 2 * elems * e + 4 * rows),
         "csr_build": (0, 0),
-        "dq": (6 * unit, 5 * elems * e + 8 * rows),
-        "dkdv": (8 * unit, 6 * elems * e + 8 * rows),
+        "dq": (6 * unit, 5 * elems * e + 8 * rows + kb),
+        "dkdv": (8 * unit, 6 * elems * e + 8 * rows + kb),
     }
 
 
@@ -313,7 +319,8 @@ def run_ours(args, world, rank, local):
     att = bb.Attention(B, H, L, bs, r, dt, d=cfg["d"], seed=synth.TABLE_SEED,
                        device=dev, dropout=args.dropout,
                        dropout_seed=args.dropout_seed,
-                       mask_queries=int(args.mask_queries))
+                       mask_queries=int(args.mask_queries),
+                       keep_dropout_bits=not args.redraw_dropout)
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     g = inp["dout"].to(dev) if backward else None
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
@@ -397,7 +404,8 @@ def run_ours(args, world, rank, local):
     # Attended FLOPs over the pattern's pairs (masked keys included).
     pairs = sum(pairs_per_head(nb, att.table_host[h].numpy())
                 for h in range(H)) * B
-    alg = algorithmic(cfg, pairs)
+    alg = algorithmic(cfg, pairs, keep_bits=att.dropout_bits is not None
+                      and cfg["dtype"] == "bf16")
     vkf = valid_key_fraction(nb, bs, att.table_host.numpy(), inp["key_mask"])
     fwd_flops = 4 * pairs * bs * bs * cfg["d"]
     bwd_flops = 10 * pairs * bs * bs * cfg["d"] if backward else 0
@@ -461,6 +469,10 @@ def run_ours(args, world, rank, local):
                    "block_size": bs, "d": cfg["d"], "r": r,
                    "mask": cfg["mask"], "passes": cfg["passes"],
                    "dropout": args.dropout,
+                   "dropout_keep_bits": ("stored by the forward"
+                                         if att.dropout_bits is not None
+                                         else "drawn in every pass")
+                   if args.dropout else None,
                    "mask_queries": bool(args.mask_queries),
                    "global_batch": B * world, "seq_len": L,
                    "parallelism": f"replicas x{world} (independent batches)",

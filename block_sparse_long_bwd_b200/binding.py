@@ -39,7 +39,8 @@ class bb_attn_desc(ctypes.Structure):
                 ("r", ctypes.c_int), ("dtype", ctypes.c_int),
                 ("scale", ctypes.c_float), ("mask_value", ctypes.c_float),
                 ("dropout", ctypes.c_float), ("dropout_seed", ctypes.c_uint64),
-                ("mask_queries", ctypes.c_int), ("grad_fp32", ctypes.c_int)]
+                ("mask_queries", ctypes.c_int), ("grad_fp32", ctypes.c_int),
+                ("dropout_bits", ctypes.c_void_p)]
 
 
 _lib = None
@@ -67,6 +68,9 @@ def lib():
             ctypes.POINTER(bb_attn_desc), ctypes.c_int,
             ctypes.POINTER(ctypes.c_size_t)]
         L.bb_attn_workspace_size.restype = ctypes.c_int
+        L.bb_attn_dropout_bits_size.argtypes = [
+            ctypes.POINTER(bb_attn_desc), ctypes.POINTER(ctypes.c_size_t)]
+        L.bb_attn_dropout_bits_size.restype = ctypes.c_int
         L.bb_attn_fwd.argtypes = [ctypes.POINTER(bb_attn_desc)] + [_P] * 8 + [
             ctypes.c_size_t, _P]
         L.bb_attn_fwd.restype = ctypes.c_int
@@ -116,12 +120,26 @@ def bb_abi_version():
 
 
 def make_desc(B, H, L, d, block_size, r, dtype, scale=0.0, mask_value=0.0,
-              dropout=0.0, dropout_seed=0, mask_queries=0, grad_fp32=0):
+              dropout=0.0, dropout_seed=0, mask_queries=0, grad_fp32=0,
+              dropout_bits=None):
+    """dropout_bits: None or a contiguous CUDA uint8 tensor of
+    bb_attn_dropout_bits_size bytes (the forward's keep decisions for the
+    backward); the descriptor holds its address, not a reference."""
     if isinstance(dtype, torch.dtype):
         dtype = {torch.float32: BB_F32, torch.bfloat16: BB_BF16}[dtype]
+    if dropout_bits is not None:
+        _cuda_tensor(dropout_bits, "dropout_bits", torch.uint8)
     return bb_attn_desc(B, H, L, d, block_size, r, dtype, scale, mask_value,
                         dropout, dropout_seed & ((1 << 64) - 1),
-                        int(mask_queries), int(grad_fp32))
+                        int(mask_queries), int(grad_fp32), _ptr(dropout_bits))
+
+
+def bb_attn_dropout_bits_size(desc):
+    n = ctypes.c_size_t(0)
+    _check(lib().bb_attn_dropout_bits_size(ctypes.byref(desc),
+                                           ctypes.byref(n)),
+           "bb_attn_dropout_bits_size")
+    return n.value
 
 
 def grad_dtype(desc):
@@ -363,14 +381,23 @@ class Attention:
     def __init__(self, B, H, L, block_size, r, dtype, d=64, seed=0,
                  device="cuda", scale=0.0, mask_value=0.0, dropout=0.0,
                  dropout_seed=0, max_rand_mask_length=0, last_idx=0,
-                 mask_queries=0, grad_fp32=0):
+                 mask_queries=0, grad_fp32=0, keep_dropout_bits=True):
         """max_rand_mask_length, last_idx (tokens; 0 = off): the pages'
         layer options for the random table (drawn for the maximum length,
         random blocks before token last_idx); seed: the layer index there.
-        grad_fp32: the backward writes dq, dk, dv as fp32."""
+        grad_fp32: the backward writes dq, dk, dv as fp32.
+        keep_dropout_bits: with dropout, hold a keep-bit buffer that the
+        forward fills and the backward reads (same results, fewer draws);
+        False makes every pass draw its decisions."""
         self.desc = make_desc(B, H, L, d, block_size, r, dtype, scale,
                               mask_value, dropout, dropout_seed, mask_queries,
                               grad_fp32)
+        self.dropout_bits = None
+        nbits = bb_attn_dropout_bits_size(self.desc) if keep_dropout_bits else 0
+        if nbits:
+            self.dropout_bits = torch.empty(nbits, dtype=torch.uint8,
+                                            device=device)
+            self.desc.dropout_bits = _ptr(self.dropout_bits)
         self.dtype = dtype
         self.table_host = make_table(seed, H, L, block_size, r,
                                      max_rand_mask_length, last_idx)

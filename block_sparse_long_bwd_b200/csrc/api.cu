@@ -115,6 +115,13 @@ int make_problem(const bb_attn_desc* desc, Problem* p) {
   p->mask_q = desc->mask_queries;  // cleared at the call when key_mask is NULL
   if (desc->grad_fp32 != 0 && desc->grad_fp32 != 1) return BB_ERR_INVALID;
   p->grad_f32 = (p->dtype == BB_F32) ? 1 : desc->grad_fp32;
+  // Stored keep decisions: only with dropout on, and only where both passes
+  // run the tensor-core kernels (the one place they are written and read).
+  if (desc->dropout_bits && !aligned16(desc->dropout_bits)) return BB_ERR_INVALID;
+  if (desc->dropout_bits && p->drop_thr && tc_fwd_supported(*p) && tc_bwd_supported(*p)) {
+    p->keep_bits = static_cast<uint32_t*>(desc->dropout_bits);
+    p->keep_slots = keep_slots_per_bh(p->nb, p->r);
+  }
   return BB_OK;
 }
 
@@ -211,6 +218,17 @@ int bb_rand_attn_build_ex(uint64_t seed, int heads, int num_blocks, int r,
 int bb_rand_attn_build(uint64_t seed, int heads, int num_blocks, int r,
                        int32_t* out_host) {
   return bb_rand_attn_build_ex(seed, heads, num_blocks, r, 0, 0, out_host);
+}
+
+int bb_attn_dropout_bits_size(const bb_attn_desc* desc, size_t* bytes) {
+  if (!bytes) return BB_ERR_INVALID;
+  Problem p;
+  int st = make_problem(desc, &p);
+  if (st != BB_OK) return st;
+  *bytes = p.drop_thr ? (size_t)p.B * p.H * keep_slots_per_bh(p.nb, p.r) *
+                            ((size_t)p.bs * p.bs / 8)
+                      : 0;
+  return BB_OK;
 }
 
 int bb_attn_workspace_size(const bb_attn_desc* desc, int pass, size_t* bytes) {

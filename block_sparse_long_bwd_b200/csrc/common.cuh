@@ -63,7 +63,18 @@ struct Problem {
   // tile whose keys are all masked; [B][tdead_words]
   uint32_t* tdead;
   int tdead_words;
+  // dropout keep decisions carried from the forward to the backward
+  // (caller buffer, tensor-core path only; nullptr: drawn in every pass):
+  // keep_slots slots of bs x bs bits per (b, h), see keep_slot()
+  uint32_t* keep_bits;
+  int keep_slots;
 };
+
+// Slots of the stored keep bits per (b, h): one per attended (query block,
+// key block) pair, with a fixed stride of 5 + r for the middle blocks.
+inline int keep_slots_per_bh(int nb, int r) {
+  return nb == 1 ? 1 : 2 * nb + (nb - 2) * (5 + r);
+}
 
 // Upper bound of attended (query block, key block) pairs per head.
 inline int pair_cap(int nb, int r) { return nb * (7 + r) + 8; }

@@ -16,6 +16,11 @@
 // tile.  The dK/dV threads own key rows; a warp there draws, per 64-query
 // tile, the rows of its 32 keys (four calls a lane) and transposes the
 // 32 x 32 bit blocks with shuffles.
+//
+// Optionally (Problem::keep_bits, a caller buffer) the forward also stores
+// the decisions it draws, one bit per attended element, and the two
+// backward passes load them instead of drawing them again: the same bits,
+// so the same results, for a word load where three Philox calls were.
 #pragma once
 
 #include <stdint.h>
@@ -138,6 +143,136 @@ __device__ __forceinline__ void keep_cols64(const Problem& p, int b, int h, int 
                       (keep_group(p, b, h, t0 + 32 + lane, g + 1, thr4) << 16);
   lo = transpose32(ra, lane);
   hi = transpose32(rb, lane);
+}
+
+// ---- stored keep decisions ------------------------------------------------
+
+// Slot of the attended pair (query block i, key block u) among the
+// keep_slots slots of one (b, h).  Query blocks 0 and nb - 1 attend every
+// key block: slots u and nb + u.  A middle block i has 5 + r slots from
+// 2 nb + (i - 1)(5 + r); its pair takes the count of members of
+// {0, i - 1 (if >= 2), i, i + 1 (if <= nb - 2)} and of table entries of row i
+// in [0, nb) below u.  Every attended block below u is counted, so distinct
+// attended blocks get distinct slots, and the count is at most 4 + r, so
+// it stays inside the row's stride (for any table, corrupt ones included).
+__device__ __forceinline__ int keep_slot(const Problem& p, int h, int i, int u) {
+  const int nb = p.nb;
+  if (i == 0) return u;
+  if (i == nb - 1) return nb + u;
+  int c = (u > 0) + (i >= 2 && i - 1 < u) + (i < u) + (i + 1 <= nb - 2 && i + 1 < u);
+  const int32_t* row = p.rand_idx + ((size_t)h * nb + i) * p.r;
+  // Four independent loads per round, so their latencies overlap.
+  for (int a = 0; a < p.r; a += 4) {
+    int j[4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) j[x] = a + x < p.r ? __ldg(row + a + x) : -1;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) c += (j[x] >= 0 && j[x] < u);
+  }
+  return 2 * nb + (i - 1) * (5 + p.r) + c;
+}
+
+__device__ __forceinline__ int keep_log2_bs(const Problem& p) {
+  return p.bs == 32 ? 5 : (p.bs == 64 ? 6 : 7);
+}
+
+// Slot of query token tq against the block of key token k0.
+__device__ __forceinline__ int keep_slot_of(const Problem& p, int h, int tq, int k0) {
+  const int sh = keep_log2_bs(p);
+  return keep_slot(p, h, tq >> sh, k0 >> sh);
+}
+
+// Word of the stored bits holding query token tq against the 32 key tokens
+// k0 .. k0 + 31 (k0 a multiple of 32) in slot `slot` of (b, h) = bh: a slot
+// is bs x bs bits, query row major, bs / 32 words per row.
+__device__ __forceinline__ uint32_t* keep_at(const Problem& p, int bh, int slot, int tq, int k0) {
+  const int wpr = p.bs >> 5;  // words per row
+  const int q = tq & (p.bs - 1), w = (k0 & (p.bs - 1)) >> 5;
+  return p.keep_bits + ((size_t)bh * p.keep_slots + slot) * (size_t)(wpr * p.bs) + q * wpr + w;
+}
+
+__device__ __forceinline__ uint32_t* keep_ptr(const Problem& p, int bh, int h, int tq, int k0) {
+  return keep_at(p, bh, keep_slot_of(p, h, tq, k0), tq, k0);
+}
+
+// The table row of one query block held in registers (up to four random
+// blocks per row, the common case), so that the slots of a row's tiles cost
+// no loads: a softmax thread's query block is the same on every tile of an
+// item.  With r > 4 the slots are looked up in the table.
+struct KeepRow {
+  int i;       // query block
+  int id[4];   // table row i (-1 past r, or for the global blocks)
+};
+
+__device__ __forceinline__ KeepRow keep_row(const Problem& p, int h, int tq) {
+  KeepRow kr;
+  kr.i = tq >> keep_log2_bs(p);
+  const bool mid = kr.i > 0 && kr.i < p.nb - 1 && p.r <= 4;
+  const int32_t* row = p.rand_idx + ((size_t)h * p.nb + (mid ? kr.i : 0)) * p.r;
+#pragma unroll
+  for (int x = 0; x < 4; ++x) kr.id[x] = (mid && x < p.r) ? __ldg(row + x) : -1;
+  return kr;
+}
+
+// keep_slot(p, h, kr.i, u).
+__device__ __forceinline__ int keep_slot_row(const Problem& p, int h, const KeepRow& kr,
+                                             int u) {
+  const int nb = p.nb, i = kr.i;
+  if (i == 0) return u;
+  if (i == nb - 1) return nb + u;
+  if (p.r > 4) return keep_slot(p, h, i, u);
+  int c = (u > 0) + (i >= 2 && i - 1 < u) + (i < u) + (i + 1 <= nb - 2 && i + 1 < u);
+#pragma unroll
+  for (int x = 0; x < 4; ++x) c += (unsigned)kr.id[x] < (unsigned)u;  // -1 never counts
+  return 2 * nb + (i - 1) * (5 + p.r) + c;
+}
+
+// The slots of a row's attended column halves m2 of key tile kt (one block
+// for both halves when the block size is 64 or more; -1 for an unattended
+// half).
+__device__ __forceinline__ void keep_slots64(const Problem& p, int h, const KeepRow& kr, int kt,
+                                             int m2, int& s0, int& s1) {
+  const int sh = keep_log2_bs(p);
+  s0 = (m2 & 1) ? keep_slot_row(p, h, kr, (kt * 64) >> sh) : -1;
+  s1 = (m2 & 2) ? ((p.bs >= 64 && (m2 & 1)) ? s0 : keep_slot_row(p, h, kr, (kt * 64 + 32) >> sh))
+                : -1;
+}
+
+// Forward: store the decisions of query token tq over key tile kt (bit e of
+// bits: key 64 kt + e) into the slots keep_slots64 gave.  With both halves
+// in one block the two words are adjacent: one 8-byte store.
+__device__ __forceinline__ void keep_store64(const Problem& p, int bh, int tq, int kt, int s0,
+                                             int s1, uint64_t bits) {
+  const int k0 = kt * 64;
+  if (s0 >= 0 && s1 >= 0 && p.bs >= 64) {
+    *reinterpret_cast<uint2*>(keep_at(p, bh, s0, tq, k0)) =
+        make_uint2((uint32_t)bits, (uint32_t)(bits >> 32));
+  } else {
+    if (s0 >= 0) *keep_at(p, bh, s0, tq, k0) = (uint32_t)bits;
+    if (s1 >= 0) *keep_at(p, bh, s1, tq, k0 + 32) = (uint32_t)(bits >> 32);
+  }
+}
+
+// Multiplier of a probability under the keep bit e of `keep`: 1 / keep
+// probability (sc) where kept, 0 where dropped.
+__device__ __forceinline__ float keep_factor(uint32_t keep, int e, float sc) {
+  return ((keep >> e) & 1u) ? sc : 0.f;
+}
+
+// dQ: the stored counterpart of keep_row64 for the attended halves m2
+// (unattended halves read as 0).
+__device__ __forceinline__ uint64_t keep_load64(const Problem& p, int bh, int h,
+                                                const KeepRow& kr, int tq, int kt, int m2) {
+  int s0, s1;
+  keep_slots64(p, h, kr, kt, m2, s0, s1);
+  const int k0 = kt * 64;
+  if (s0 >= 0 && s1 >= 0 && p.bs >= 64) {
+    const uint2 w = __ldg(reinterpret_cast<const uint2*>(keep_at(p, bh, s0, tq, k0)));
+    return ((uint64_t)w.y << 32) | w.x;
+  }
+  const uint32_t lo = s0 >= 0 ? __ldg(keep_at(p, bh, s0, tq, k0)) : 0u;
+  const uint32_t hi = s1 >= 0 ? __ldg(keep_at(p, bh, s1, tq, k0 + 32)) : 0u;
+  return ((uint64_t)hi << 32) | lo;
 }
 
 }  // namespace bb

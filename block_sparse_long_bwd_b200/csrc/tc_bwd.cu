@@ -181,13 +181,15 @@ __device__ __forceinline__ void dq_ds_half(const uint32_t (&pv)[32], const uint3
 __device__ __forceinline__ void dq_ds_half_drop(const uint32_t (&pv)[32],
                                                 const uint32_t (&dp)[32], float Dr, float sc,
                                                 uint32_t keep, uint32_t* out) {
+  const float2 nD2 = make_float2(-Dr, -Dr);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    const float m0 = ((keep >> e) & 1u) ? sc : 0.f;
-    const float m1 = ((keep >> (e + 1)) & 1u) ? sc : 0.f;
-    const float d0 = __uint_as_float(pv[e]) * fmaf(m0, __uint_as_float(dp[e]), -Dr);
-    const float d1 = __uint_as_float(pv[e + 1]) * fmaf(m1, __uint_as_float(dp[e + 1]), -Dr);
-    out[e >> 1] = pack_bf16(d0, d1);
+    // Paired (f32x2): m dP - D, then times P, each element rounded once.
+    const float2 m = make_float2(keep_factor(keep, e, sc), keep_factor(keep, e + 1, sc));
+    const float2 t =
+        fma2(m, make_float2(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])), nD2);
+    const float2 d = mul2(make_float2(__uint_as_float(pv[e]), __uint_as_float(pv[e + 1])), t);
+    out[e >> 1] = pack_bf16(d.x, d.y);
   }
 }
 
@@ -466,13 +468,24 @@ __global__ void __launch_bounds__(kThreads2, 2)
         }
       }
       bool ok = true;
+      // Stored dropout decisions: this row's table row, and the words of
+      // each tile loaded one tile ahead.
+      KeepRow kr;
+      if (kDrop && p.keep_bits) kr = keep_row(p, im.h, tq);
+      auto keep_words = [&](int tt) -> uint64_t {
+        const int mm = (L.mask[tt] >> gshift) & 3;
+        return mm ? keep_load64(p, im.bh, im.h, kr, tq, L.tile[tt], mm) : 0ull;
+      };
+      uint64_t dbn = (kDrop && p.keep_bits && n > 0) ? keep_words(0) : 0ull;
       for (int t = 0; t < n; ++t, ++u) {
+        const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
+        const uint64_t dbs = dbn;
+        if (kDrop && p.keep_bits && t + 1 < n) dbn = keep_words(t + 1);
         if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
         // S of the attended halves into registers: once every warp has it
         // (s_free) the MMA warp computes the next tile's S; P is formed in
         // place.  dP follows half by half; after the second half (dp_free)
@@ -485,8 +498,9 @@ __global__ void __launch_bounds__(kThreads2, 2)
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free);
         const uint64_t kb = (m2 && p.key_mask) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
-        const uint64_t db =
-            (kDrop && m2) ? keep_row64(p, im.b, im.h, tq, L.tile[t]) : 0ull;
+        const uint64_t db = (kDrop && m2)
+                                ? (p.keep_bits ? dbs : keep_row64(p, im.b, im.h, tq, L.tile[t]))
+                                : 0ull;
         if (m2 & 1) dq_p_half(s0, kb, 0, c, nl2, mvl);
         if (m2 & 2) dq_p_half(s1, kb, 32, c, nl2, mvl);
         uint32_t dS[32];
@@ -898,21 +912,35 @@ __global__ void __launch_bounds__(kThreads1, 1)
         off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
       const bool split = kSplit && it.global;  // bf16 low parts too
       bool ok = true;
-      uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
+      // Walk entries are loaded two tiles ahead; with stored dropout
+      // decisions, lane l loads the word of query token t0 + l against the
+      // warp's 32 keys one tile ahead (transposed below).
+      auto keep_word = [&](uint32_t ent) -> uint32_t {
+        if (!(((int)(ent >> 16) >> (gshift + hc)) & 1)) return 0u;
+        return __ldg(keep_ptr(p, it.bh, it.h, (int)(ent & 0xFFFFu) * kTile + hc * 32 + lane,
+                              (int)(ktok & ~(size_t)31)));
+      };
+      uint32_t cur = e0 < e1 ? __ldg(walk + e0) : 0u;
+      uint32_t nxt = e0 + 1 < e1 ? __ldg(walk + e0 + 1) : 0u;
+      uint32_t kwn = (kDrop && p.keep_bits && e0 < e1) ? keep_word(cur) : 0u;
       for (int e = e0; e < e1; ++e) {
-        const int mask = (int)(nxt >> 16);
-        const int qtile = (int)(nxt & 0xFFFFu);
-        if (e + 1 < e1) nxt = __ldg(walk + e + 1);
+        const uint32_t ent = cur;
+        cur = nxt;
+        if (e + 2 < e1) nxt = __ldg(walk + e + 2);
+        const int mask = (int)(ent >> 16);
+        const int qtile = (int)(ent & 0xFFFFu);
+        const uint32_t kw = kwn;
+        if (kDrop && p.keep_bits && e + 1 < e1) kwn = keep_word(cur);
         const uint32_t g = u;
         const int b = g & 1;
         const uint32_t st = g % kKvQStages;
+        // Do query rows of this warp's column half attend this key group?
+        const bool att = (mask >> (gshift + hc)) & 1;
         if (!mbar_wait(&bars.s_full[b], (g >> 1) & 1, &abort_flag, p.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // Do query rows of this warp's column half attend this key group?
-        const bool att = (mask >> (gshift + hc)) & 1;
         // The stage's NL / D arrived by bulk copy: observe its barrier too.
         if (att && !mbar_wait(&bars.qt_full[st], (g / kKvQStages) & 1, &abort_flag,
                               p.status)) {
@@ -940,8 +968,9 @@ __global__ void __launch_bounds__(kThreads1, 1)
         // tokens (att is uniform over the warp, as the shuffles need).
         const uint32_t keep =
             (kDrop && att)
-                ? keep_cols32(p, it.b, it.h, (int)(ktok & ~(size_t)31), qtile * kTile + hc * 32,
-                              lane)
+                ? (p.keep_bits ? transpose32(kw, lane)
+                               : keep_cols32(p, it.b, it.h, (int)(ktok & ~(size_t)31),
+                                             qtile * kTile + hc * 32, lane))
                 : 0u;
         // P^T and dS^T of the half (bf16 pairs, 16 columns each): high parts
         // to the P^T / dS^T buffers, low parts (split tiles) over the S^T /
@@ -967,13 +996,20 @@ __global__ void __launch_bounds__(kThreads1, 1)
               pv[x + 1] = ex2(a.y);
               if (kDrop) {
                 // m = 1 / keep probability where kept, 0 where dropped:
-                // dS = P (m dP - D), and m P enters dV.
-                const float m0 = ((keep >> (e + x)) & 1u) ? p.drop_scale : 0.f;
-                const float m1 = ((keep >> (e + x + 1)) & 1u) ? p.drop_scale : 0.f;
-                dv[x] = pv[x] * fmaf(m0, __uint_as_float(dp[e + x]), -dds[x]);
-                dv[x + 1] = pv[x + 1] * fmaf(m1, __uint_as_float(dp[e + x + 1]), -dds[x + 1]);
-                pv[x] *= m0;
-                pv[x + 1] *= m1;
+                // dS = P (m dP - D), and m P enters dV (paired, each element
+                // rounded once).
+                const float2 m = make_float2(keep_factor(keep, e + x, p.drop_scale),
+                                             keep_factor(keep, e + x + 1, p.drop_scale));
+                const float2 pp = make_float2(pv[x], pv[x + 1]);
+                const float2 t = fma2(
+                    m, make_float2(__uint_as_float(dp[e + x]), __uint_as_float(dp[e + x + 1])),
+                    make_float2(-dds[x], -dds[x + 1]));
+                const float2 d = mul2(pp, t);
+                const float2 pk = mul2(pp, m);
+                dv[x] = d.x;
+                dv[x + 1] = d.y;
+                pv[x] = pk.x;
+                pv[x + 1] = pk.y;
               } else {
                 const float2 d = mul2(
                     make_float2(pv[x], pv[x + 1]),

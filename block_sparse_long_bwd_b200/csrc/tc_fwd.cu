@@ -349,6 +349,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       float m = -INFINITY, l = 0.f;
       // Query token of this row (dropout counters; any row when invalid).
       const int tq = (((im.gvalid >> quarter) & 1) ? im.t[half] : 0) * kTile + (row & 63);
+      // Stored dropout decisions: this row's query block and its table row.
+      const bool keep_out = kDrop && p.keep_bits && ((im.gvalid >> quarter) & 1);
+      KeepRow kr;
+      if (keep_out) kr = keep_row(p, im.h, tq);
       bool ok = true;
       for (int t = 0; t < n; ++t) {
         const uint32_t uu = u + t;
@@ -356,6 +360,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t par = (uu >> 1) & 1;
         const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
         const bool att = m2 != 0;
+        // Where this row's dropout decisions go when the caller keeps them
+        // (worked out while the scores are still being computed).
+        int ks0 = -1, ks1 = -1;
+        if (keep_out && att) keep_slots64(p, im.h, kr, L.tile[t], m2, ks0, ks1);
         if (!mbar_wait(&bars.s_full[b2], par, &abort_flag, p.status)) {
           ok = false;
           break;
@@ -439,6 +447,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           const float cc = scaled ? 1.f : c;
           const float2 cc2 = make_float2(cc, cc), nm2 = make_float2(-m, -m);
           const uint64_t db = kDrop ? keep_row64(p, im.b, im.h, tq, L.tile[t]) : 0ull;
+          // Hand the decisions to the backward when the caller keeps them.
+          if (kDrop && p.keep_bits && (ks0 >= 0 || ks1 >= 0))
+            keep_store64(p, im.bh, tq, L.tile[t], ks0, ks1, db);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t Ph[16];
@@ -449,9 +460,11 @@ __global__ void __launch_bounds__(kThreads, 2)
               sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pp);
               if (kDrop) {
                 // Kept probabilities times 1 / keep probability, dropped 0.
-                const int col = 32 * hh + e;
-                Ph[e >> 1] = pack_bf16(((db >> col) & 1ull) ? pp.x * p.drop_scale : 0.f,
-                                       ((db >> (col + 1)) & 1ull) ? pp.y * p.drop_scale : 0.f);
+                const uint32_t dw = (uint32_t)(db >> (32 * hh));
+                const float2 mk = make_float2(keep_factor(dw, e, p.drop_scale),
+                                              keep_factor(dw, e + 1, p.drop_scale));
+                const float2 pk = mul2(pp, mk);
+                Ph[e >> 1] = pack_bf16(pk.x, pk.y);
               } else {
                 Ph[e >> 1] = pack_bf16(pp.x, pp.y);
               }

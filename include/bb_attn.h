@@ -46,7 +46,7 @@
 extern "C" {
 #endif
 
-#define BB_ABI_VERSION 4
+#define BB_ABI_VERSION 5
 
 #if defined(__GNUC__)
 #define BB_API __attribute__((visibility("default")))
@@ -109,7 +109,32 @@ typedef enum { BB_F32 = 0, BB_BF16 = 1 } bb_dtype;
  * bf16's own spacing (1/32, then 1/16 above 8) alone exceeds an absolute
  * error of 1e-2.  Use grad_fp32 = 1 where gradients must be within a fixed
  * absolute error of the exact result at such lengths.  Ignored for fp32
- * dtype (the gradients are fp32 already). */
+ * dtype (the gradients are fp32 already).
+ *
+ * dropout_bits (optional; NULL = off): a device buffer of
+ * bb_attn_dropout_bits_size(desc) bytes, 16-byte aligned, owned by the
+ * caller, that carries the dropout keep decisions from the forward to the
+ * backward.  With a nonzero dropout rate, bb_attn_fwd writes there the
+ * decisions it draws, and bb_attn_bwd reads them instead of drawing them
+ * again (a Philox4x32-10 call per 16 elements in each of its two passes).
+ * The decisions are the same either way, so the results are bit for bit
+ * those of a call with dropout_bits = NULL; only the time differs.  The
+ * buffer must hold what a forward with the same descriptor (dropout_seed
+ * included), rand_idx and key_mask wrote, and must not be written between
+ * that forward and the backward.  Entries of key tiles whose keys are all
+ * masked may be left unwritten (their probabilities are 0, so their
+ * decisions change nothing).  Used by the tensor-core kernels (bf16, the shapes listed for
+ * them); the CUDA-core kernels neither write nor read it.  Ignored when the
+ * rate rounds to 0.  Layout (a pure function of the descriptor and the
+ * table): per (b, h), slots of block_size x block_size bits, one per
+ * attended (query block i, key block u) pair, query row major with 32 keys
+ * per uint32 word (bit j of word w of row q: key u * block_size + 32 w + j,
+ * bit set = kept).  Slots of (b, h) start at word
+ * (b * H + h) * S * block_size^2 / 32 with S = 2 nb + (nb - 2)(5 + r)
+ * (S = 1 for nb = 1); query block 0 uses slot u, block nb - 1 slot nb + u,
+ * and a middle block i slot 2 nb + (i - 1)(5 + r) + c(i, u), where c(i, u)
+ * counts the members of {0, i - 1 if >= 2, i, i + 1 if <= nb - 2} and the
+ * entries of table row i in [0, nb) that are below u. */
 typedef struct {
   int B, H, L, d, block_size, r;
   int dtype;
@@ -119,6 +144,7 @@ typedef struct {
   uint64_t dropout_seed;
   int mask_queries;
   int grad_fp32;
+  void* dropout_bits;
 } bb_attn_desc;
 
 /* Random block table ([gitcode page] section "随机块掩码是如何生成的": per
@@ -165,6 +191,12 @@ BB_API int bb_rand_attn_build_ex(uint64_t seed, int heads, int num_blocks, int r
 /* Bytes of device workspace bb_attn_fwd (pass 0) or bb_attn_bwd (pass 1)
  * needs for `desc`; written to *bytes.  Host only. */
 BB_API int bb_attn_workspace_size(const bb_attn_desc* desc, int pass, size_t* bytes);
+
+/* Bytes of the optional dropout keep-bit buffer (bb_attn_desc.dropout_bits)
+ * for `desc`: B * H * S * block_size^2 / 8 with S as given there (about 1
+ * bit per attended probability); 0 when the dropout rate rounds to 0.
+ * Written to *bytes.  Host only. */
+BB_API int bb_attn_dropout_bits_size(const bb_attn_desc* desc, size_t* bytes);
 
 /* Forward ([gitcode page] section "BigBird：从二次方注意力到线性稀疏注意力":
  * five segments first / second / middle / second_last / last, masked keys

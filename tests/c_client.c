@@ -33,7 +33,7 @@ int main(void) {
   int32_t table[H * NB * R], table_ex[H * NB * R];
   int h, i, a;
   size_t ws = 0;
-  bb_attn_desc d = {2, H, NB * 64, 64, 64, R, BB_BF16, 0.f, 0.f, 0.f, 0, 0, 0};
+  bb_attn_desc d = {2, H, NB * 64, 64, 64, R, BB_BF16, 0.f, 0.f, 0.f, 0, 0, 0, NULL};
   bb_attn_desc bad = d;
   const uintptr_t fake = (uintptr_t)1 << 20; /* never dereferenced */
   void* p = (void*)fake;
@@ -70,6 +70,14 @@ int main(void) {
   bad = d;
   bad.dropout = 1.0f;
   CHECK(bb_attn_workspace_size(&bad, 0, &ws) == BB_ERR_INVALID);
+  /* dropout keep-bit buffer: 1 bit per attended probability slot */
+  CHECK(bb_attn_dropout_bits_size(&d, &ws) == BB_OK && ws == 0);
+  bad = d;
+  bad.dropout = 0.1f;
+  CHECK(bb_attn_dropout_bits_size(&bad, &ws) == BB_OK &&
+        ws == (size_t)2 * H * (2 * NB + (NB - 2) * (5 + R)) * 64 * 64 / 8);
+  bad.dropout_bits = (void*)(fake + 4); /* misaligned */
+  CHECK(bb_attn_dropout_bits_size(&bad, &ws) == BB_ERR_INVALID);
 
   /* Compute calls: refused on the host before any CUDA call. */
   CHECK(bb_attn_workspace_size(&d, 0, &ws) == BB_OK);

@@ -15,17 +15,24 @@ ATOL = {"f32": 2e-5, "bf16": 1e-2}
 
 def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
             scale=0.0, mask_value=0.0, table=None, dropout=0.0,
-            dropout_seed=0, mask_queries=0, grad_fp32=0):
+            dropout_seed=0, mask_queries=0, grad_fp32=0,
+            keep_dropout_bits=True, bits_fill=None):
     """Forward (and backward) through the C ABI; returns CPU tensors.
     grad_fp32: the backward writes dq, dk, dv as fp32 (returned as such;
-    bf16 gradients come back widened to fp32 exactly)."""
+    bf16 gradients come back widened to fp32 exactly).
+    keep_dropout_bits: with dropout, the forward stores its keep decisions
+    for the backward (returned as "dropout_bits", uint8); bits_fill: byte
+    written over that buffer before the forward."""
     dev = torch.device("cuda")
     B, H, L = cfg["B"], cfg["H"], cfg["L"]
     att = bb.Attention(B, H, L, cfg["block_size"], cfg["r"],
                        synth.torch_dtype(cfg["dtype"]), d=cfg["d"],
                        seed=table_seed, scale=scale, mask_value=mask_value,
                        dropout=dropout, dropout_seed=dropout_seed,
-                       mask_queries=mask_queries, grad_fp32=grad_fp32)
+                       mask_queries=mask_queries, grad_fp32=grad_fp32,
+                       keep_dropout_bits=keep_dropout_bits)
+    if att.dropout_bits is not None and bits_fill is not None:
+        att.dropout_bits.fill_(bits_fill)
     if table is not None:
         att.table_host = torch.as_tensor(table, dtype=torch.int32)
         att.table = att.table_host.to(dev)
@@ -40,8 +47,11 @@ def run_gpu(cfg, inp, table_seed=synth.TABLE_SEED, backward=True,
         res.update(dq=dq, dk=dk, dv=dv,
                    status_bwd=bb.bb_attn_check_status(att.ws_bwd))
     torch.cuda.synchronize()
-    return {k_: (v_.float().cpu() if torch.is_tensor(v_) and v_.is_cuda
-                 else v_) for k_, v_ in res.items()}
+    out = {k_: (v_.float().cpu() if torch.is_tensor(v_) and v_.is_cuda
+                else v_) for k_, v_ in res.items()}
+    if att.dropout_bits is not None:
+        out["dropout_bits"] = att.dropout_bits.cpu()
+    return out
 
 
 def oracle_slice(cfg, inp, table, b, h, backward=True, scale=None,

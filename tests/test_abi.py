@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
     assert "bb_attn_fwd" in names and "bb_attn_bwd" in names
     for name in names:
         assert hasattr(lib, name), name
-    assert bb.bb_abi_version() == 4
+    assert bb.bb_abi_version() == 5
 
 
 @pytest.mark.parametrize("seed,H,nb,r", [
@@ -141,6 +141,45 @@ def test_workspace_size_and_validation():
     assert lib.bb_attn_workspace_size(None, 0, ctypes.byref(n)) == -1
     assert lib.bb_attn_workspace_size(ctypes.byref(_desc()), 2,
                                       ctypes.byref(n)) == -1
+
+
+def _keep_slots(nb, r):
+    # One slot per attended (query block, key block) pair: nb for each
+    # global query block, 5 + r for each middle one.
+    return 1 if nb == 1 else 2 * nb + (nb - 2) * (5 + r)
+
+
+@pytest.mark.parametrize("L,bs,r", [
+    (512, 64, 3), (4096, 64, 3), (1024, 32, 6), (2048, 128, 0), (64, 64, 3),
+    (128, 64, 2), (4096 * 4, 64, 3),
+])
+def test_dropout_bits_size(L, bs, r):
+    nb = L // bs
+    d = _desc(L=L, block_size=bs, r=r, dropout=0.1)
+    want = 2 * 3 * _keep_slots(nb, r) * bs * bs // 8
+    assert bb.bb_attn_dropout_bits_size(d) == want
+    # room for every attended pair of a drawn table
+    table = oracle.rand_table(0, 3, nb, r)
+    for h in range(3):
+        assert oracle.pair_count(nb, table[h]) <= _keep_slots(nb, r)
+    # no dropout (or a rate that rounds to 0): no buffer
+    assert bb.bb_attn_dropout_bits_size(_desc(L=L, block_size=bs, r=r)) == 0
+    assert bb.bb_attn_dropout_bits_size(
+        _desc(L=L, block_size=bs, r=r, dropout=0.001)) == 0
+
+
+def test_dropout_bits_pointer_validation():
+    lib = bb.lib()
+    d = _desc(dropout=0.1)
+    d.dropout_bits = 8  # misaligned (never dereferenced)
+    n = ctypes.c_size_t(0)
+    assert lib.bb_attn_dropout_bits_size(ctypes.byref(d), ctypes.byref(n)) == -1
+    assert lib.bb_attn_workspace_size(ctypes.byref(d), 0, ctypes.byref(n)) == -1
+    d.dropout_bits = 1 << 20  # aligned: accepted, sizes unchanged
+    assert bb.bb_attn_workspace_size(d, 0) == bb.bb_attn_workspace_size(
+        _desc(dropout=0.1), 0)
+    assert lib.bb_attn_dropout_bits_size(None, ctypes.byref(n)) == -1
+    assert lib.bb_attn_dropout_bits_size(ctypes.byref(d), None) == -1
 
 
 def test_compute_calls_reject_bad_arguments_on_host():

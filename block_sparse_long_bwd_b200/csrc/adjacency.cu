@@ -226,10 +226,10 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
   TileList& L = static_cast<TileList*>(p.qplan)[(size_t)h * g.per_bh + loc];
   if (m.global) {
     const int bits = expand_groups(m.gvalid, 3);
-    const int j0 = m.chunk * kChunk, j1 = min(g.nt, j0 + kChunk);
-    if (lane < j1 - j0) {
-      L.tile[lane] = (int16_t)(j0 + lane);
-      L.mask[lane] = (uint8_t)bits;
+    const int j0 = m.chunk * g.chunk, j1 = min(g.nt, j0 + g.chunk);
+    for (int x = lane; x < j1 - j0; x += 32) {
+      L.tile[x] = (int16_t)(j0 + x);
+      L.mask[x] = (uint8_t)bits;
     }
     if (lane == 0) L.n = j1 - j0;
     return;
@@ -345,7 +345,7 @@ __device__ void plan_q_item(const Problem& p, const Geom& g, int h, int loc,
 // area, so no allocator is needed: a middle window's walk has at most T x
 // (the CSR list lengths of its key blocks) entries (T = 2 query tiles per
 // query block at block size 128, else 1), so its region starts at T times
-// the CSR offset of its first key block; global chunks (kChunk query tiles
+// the CSR offset of its first key block; global chunks (g.chunk query tiles
 // each) follow T x (all CSR entries).
 // offs / list: the head's CSR (global memory, or shared memory when
 // stage is null: the lists are then read in place).
@@ -360,8 +360,8 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
   const int T = g.bs == 128 ? 2 : 1;
   int base, cap;
   if (w.global) {
-    base = T * offs[g.nb] + (w.gi * g.nchunks + w.chunk) * kChunk;
-    cap = kChunk;
+    base = T * offs[g.nb] + (w.gi * g.nchunks + w.chunk) * g.chunk;
+    cap = g.chunk;
   } else {
     const int row0 = w.t[0] * kTile;  // window rows [row0, row0 + 128)
     const int jf = block_of(g, row0);
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
                                                                int do_k, int do_dead) {
   __shared__ int cand[kPlanWarps][128];
   __shared__ int stage[kPlanWarps][kStageCap];
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nitems = p.H * g.per_bh;
   // The work counters of the tensor-core launches that follow.
@@ -606,7 +606,7 @@ __global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, i
   extern __shared__ int csr_sm[];
   __shared__ int cand[kFusedWarps][128];
   __shared__ int merged[kFusedWarps][128];
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
   if ((int)blockIdx.x < qctas) {
@@ -632,7 +632,7 @@ size_t fused_plan_smem(const Problem& p) {
 bool tc_bwd_plan_fused(const Problem& p) { return fused_plan_smem(p) <= 160u * 1024u; }
 
 cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s) {
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   const int nitems = p.H * g.per_bh;
   const int qctas = (nitems + kFusedWarps - 1) / kFusedWarps;
   // One key-side item per warp (each CTA rebuilds its head's small
@@ -656,7 +656,7 @@ cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-size_t tc_items_per_bh(const Problem& p) { return make_geom(p.L, p.bs).per_bh; }
+size_t tc_items_per_bh(const Problem& p) { return make_geom(p).per_bh; }
 
 size_t tc_qplan_bytes(const Problem& p) {
   return (size_t)p.H * tc_items_per_bh(p) * sizeof(TileList);
@@ -666,11 +666,11 @@ size_t tc_qplan_bytes(const Problem& p) {
 // window stands for at least one attended (query block, key block) pair
 // (two tiles per block at block size 128); global items visit all tiles.
 int tc_kplan_cap(const Problem& p) {
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   return 2 * pair_cap(p.nb, p.r) + g.n_git * g.nt + 64;
 }
 
-int tc_tdead_words(const Problem& p) { return 1 + (make_geom(p.L, p.bs).nt + 31) / 32; }
+int tc_tdead_words(const Problem& p) { return 1 + (make_geom(p).nt + 31) / 32; }
 
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
   const int items = p.H * (int)tc_items_per_bh(p);

@@ -347,7 +347,9 @@ static const char* const kBwdSimt[] = {"bwd_pre", "csr_build", "simt_dq",
 // built in shared memory, one launch) or, when a head's adjacency does not
 // fit there, csr_build + plan; then dQ, dK/dV (two launches at long lengths:
 // the global key blocks with the hi/lo split on their own,
-// tc_dkdv_launches), and the merge of the global rows' partials.
+// tc_dkdv_launches), and the merge of the global rows' partials when those
+// rows are split into chunks (tc_global_rows_chunked; the forward's
+// fwd_combine likewise).
 static const char* const kBwdTcTail1[] = {"tc_dq", "tc_dkdv", "bwd_finish"};
 static const char* const kBwdTcTail2[] = {"tc_dq", "tc_dkdv", "tc_dkdv", "bwd_finish"};
 
@@ -360,7 +362,7 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
   if (pass == 0) {
     const bool tc = tc_fwd_supported(p);
     *names = tc ? kFwdTc : kFwdSimt;
-    *n = tc ? 3 : 1;
+    *n = tc ? (tc_global_rows_chunked(p) ? 3 : 2) : 1;
   } else {
     if (!tc_bwd_supported(p)) {
       *names = kBwdSimt;
@@ -374,7 +376,8 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     buf[c++] = "plan";
     const bool two = tc_dkdv_launches(p) == 2;
     const char* const* tail = two ? kBwdTcTail2 : kBwdTcTail1;
-    const int nt = two ? 4 : 3;
+    // The merge launch only when global rows are chunked.
+    const int nt = (two ? 4 : 3) - (tc_global_rows_chunked(p) ? 0 : 1);
     for (int i = 0; i < nt; ++i) buf[c++] = tail[i];
     *names = buf;
     *n = c;

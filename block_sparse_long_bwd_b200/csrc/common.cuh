@@ -136,6 +136,9 @@ size_t tc_bwd_extra_bytes(const Problem& p);
 // Number of dK/dV launches of the tensor-core backward (1, or 2 at lengths
 // where the global key blocks run with the hi/lo split on their own).
 int tc_dkdv_launches(const Problem& p);
+// True when global rows are split into chunks whose partials a merge launch
+// (fwd_combine / bwd_finish) combines; false when they run whole.
+bool tc_global_rows_chunked(const Problem& p);
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);
 

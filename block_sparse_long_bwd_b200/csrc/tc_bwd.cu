@@ -561,7 +561,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.dq_empty);
       if (rvalid) {
-        if (!im.global) {
+        if (!im.global || a.geo.nchunks == 1) {  // final rows (no chunk partials)
           store_grad_row(p, p.dq, grow, q0, q1, p.scale);
         } else {
           float4* dst = reinterpret_cast<float4*>(
@@ -1071,7 +1071,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty);
       if (rvalid) {
-        if (!it.global) {
+        if (!it.global || ba.qa.geo.nchunks == 1) {  // final rows (no chunk partials)
           store_grad_half(p, p.dk, krow, hc * 32, kx, p.scale);
           store_grad_half(p, p.dv, krow, hc * 32, vx, 1.0f);
         } else {
@@ -1160,12 +1160,14 @@ bool tc_bwd_supported(const Problem& p) { return tc_shape_ok(p); }
 
 // D, NL: rows floats each; dq partials; dK/dV partials.
 int tc_dkdv_launches(const Problem& p) {
-  return (p.L >= kSplitMinL && make_geom(p.L, p.bs).n_mid > 0) ? 2 : 1;
+  return (p.L >= kSplitMinL && make_geom(p).n_mid > 0) ? 2 : 1;
 }
+
+bool tc_global_rows_chunked(const Problem& p) { return make_geom(p).nchunks > 1; }
 
 size_t tc_bwd_extra_bytes(const Problem& p) {
   const size_t rows = (size_t)p.B * p.H * p.L;
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   const size_t units = (size_t)p.B * p.H * g.n_git * g.nchunks * 128;
   return rows * 4 /* NL */ + units * 64 * 4 + units * 128 * 4 + 3 * 256;
 }
@@ -1232,14 +1234,20 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);
     if (e != cudaSuccess) return e;
+    if (i > 0) {
+      e = marks->mark(s);
+      if (e != cudaSuccess) return e;
+    }
     kv_kernel<<<min(bk.kitems, sms), kThreads1, smem_kv, s>>>(
         bk, tm.q, tm.k, tm.v, tm.dout);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    e = marks->mark(s);
-    if (e != cudaSuccess) return e;
   }
 
+  // Global rows written whole: no chunk partials to merge.
+  if (g.nchunks == 1) return cudaSuccess;
+  e = marks->mark(s);
+  if (e != cudaSuccess) return e;
   const size_t frows = (size_t)p.B * p.H * ba.qa.geo.n_git * 128;
   bwd_finish_kernel<<<(unsigned)((frows + 7) / 8), 256, 0, s>>>(ba);
   return cudaGetLastError();

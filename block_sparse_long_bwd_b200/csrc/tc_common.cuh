@@ -33,7 +33,9 @@ constexpr int kTile = 64;                             // tokens per tile
 // low part in the dK/dV pass (they sum over every query row).
 constexpr int kSplitMinL = 16384;
 constexpr int kMaxT = 64;                             // tiles per item
-constexpr int kChunk = 8;                             // tiles per chunk
+constexpr int kChunk = 8;                             // tiles per chunk (split rows)
+// CTAs the balance rule below plans for: two per SM of a B200 (148 SMs).
+constexpr int kBalanceCtas = 2 * 148;
 constexpr uint32_t kTileBytes = kTile * kHeadDim * 2; // one 64 x 64 bf16 tile
 constexpr int kPartStride = 68;                       // floats per fwd partial row
 
@@ -45,11 +47,14 @@ struct Geom {
   int ngt;              // tiles holding global blocks (ascending in gt)
   int gt[4];
   int n_git;            // global items = ceil(ngt / 2)
+  int chunk;            // tiles per chunk of a global item
   int nchunks;          // chunks of the tile range [0, nt)
   int per_bh;           // items per (b, h): n_mid + n_git * nchunks
 };
 
-__host__ __device__ inline Geom make_geom(int L, int bs) {
+// Geometry for L tokens in blocks of bs; chunk = tiles per chunk of a global
+// item (0: kChunk).
+__host__ __device__ inline Geom make_geom(int L, int bs, int chunk = 0) {
   Geom g;
   g.bs = bs;
   g.bs_shift = bs == 32 ? 5 : bs == 64 ? 6 : 7;
@@ -74,9 +79,29 @@ __host__ __device__ inline Geom make_geom(int L, int bs) {
     if (!dup && t >= 0) g.gt[g.ngt++] = t;
   }
   g.n_git = (g.ngt + 1) / 2;
-  g.nchunks = (g.nt + kChunk - 1) / kChunk;
+  g.chunk = chunk > 0 ? chunk : kChunk;
+  g.nchunks = (g.nt + g.chunk - 1) / g.chunk;
   g.per_bh = g.n_mid + g.n_git * g.nchunks;
   return g;
+}
+
+// Tiles per chunk of a global item for problem p.  A global row visits every
+// key tile (a global key block every query tile).  When one tile list holds
+// them all (nt <= kMaxT) and the rest of the problem gives the launch's CTAs
+// more work each than one such item (middle windows estimated at 8 + r
+// tiles), the item runs whole: it writes its rows directly and no partials
+// are merged.  Otherwise rows are split into chunks of kChunk tiles whose
+// partials are merged in a fixed order by a launch of their own.
+__host__ __device__ inline int global_chunk_tiles(const Problem& p) {
+  const Geom g = make_geom(p.L, p.bs);
+  if (g.nt > kMaxT) return kChunk;
+  const long long work = (long long)p.B * p.H *
+                         ((long long)g.n_mid * (8 + p.r) + (long long)g.n_git * g.nt);
+  return work >= (long long)kBalanceCtas * g.nt ? g.nt : kChunk;
+}
+
+__host__ __device__ inline Geom make_geom(const Problem& p) {
+  return make_geom(p.L, p.bs, global_chunk_tiles(p));
 }
 
 // Block of token row `tok`.
@@ -127,7 +152,7 @@ struct PairArgs {
 inline PairArgs make_pair_args(const Problem& p) {
   PairArgs a;
   a.p = p;
-  a.geo = make_geom(p.L, p.bs);
+  a.geo = make_geom(p);
   a.items = p.B * p.H * a.geo.per_bh;
   return a;
 }
@@ -203,9 +228,10 @@ __host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int
 }
 
 // Next work item of a launch, taken from its counter: the locs [loc0, loc0 +
-// nloc) of every (b, h), middle windows first (longer tile lists), then the
-// global chunks, so the short items fill the end of the launch.  False when
-// none is left.
+// nloc) of every (b, h), longest items first so the short ones fill the end
+// of the launch: middle windows, then the global chunks; whole (unchunked)
+// global items, which are longer than a window, before the windows.  False
+// when none is left.
 __device__ __forceinline__ bool next_work(const Geom& g, int B, int H, int loc0, int nloc,
                                           int* ctr, int& b, int& h, int& loc) {
   const int nglob = g.n_git * g.nchunks;
@@ -214,16 +240,18 @@ __device__ __forceinline__ bool next_work(const Geom& g, int B, int H, int loc0,
   const int ngl = nloc - nmid;
   const int BH = B * H;
   const int w = atomicAdd(ctr, 1);
+  if (w >= BH * nloc) return false;
   int bh;
-  if (w < BH * nmid) {
-    bh = w / nmid;
-    loc = mlo + w % nmid;
-  } else if (w < BH * nloc) {
-    const int w2 = w - BH * nmid;
-    bh = w2 / ngl;
-    loc = loc0 + w2 % ngl;
+  const bool glob_first = g.nchunks == 1;
+  const int nfirst = glob_first ? ngl : nmid;
+  if (w < BH * nfirst) {
+    bh = w / nfirst;
+    loc = (glob_first ? loc0 : mlo) + w % nfirst;
   } else {
-    return false;
+    const int w2 = w - BH * nfirst;
+    const int nsecond = glob_first ? nmid : ngl;
+    bh = w2 / nsecond;
+    loc = (glob_first ? mlo : loc0) + w2 % nsecond;
   }
   b = bh / H;
   h = bh % H;
@@ -239,8 +267,8 @@ __host__ __device__ inline bool build_tile_list(const Problem& p, const Geom& g,
   bool table_ok = true;
   if (m.global) {
     const int bits = expand_groups(m.gvalid, 3);
-    const int j1 = g.nt < (m.chunk + 1) * kChunk ? g.nt : (m.chunk + 1) * kChunk;
-    for (int j = m.chunk * kChunk; j < j1; ++j) {
+    const int j1 = g.nt < (m.chunk + 1) * g.chunk ? g.nt : (m.chunk + 1) * g.chunk;
+    for (int j = m.chunk * g.chunk; j < j1; ++j) {
       L.tile[L.n] = (int16_t)j;
       L.mask[L.n] = (uint8_t)bits;
       ++L.n;
@@ -322,8 +350,8 @@ struct KeyWalk {
     gvalid = m.gvalid;
     if (global) {
       gmask = expand_groups(gvalid, 3);
-      cur = chunk * kChunk;
-      end = g.nt < cur + kChunk ? g.nt : cur + kChunk;
+      cur = chunk * g.chunk;
+      end = g.nt < cur + g.chunk ? g.nt : cur + g.chunk;
       return;
     }
     for (int gr = 0; gr < 4; ++gr) {

@@ -496,10 +496,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_after();
       const int r64 = row & 63;
       const bool write = (im.gvalid >> quarter) & 1;
-      float inv = im.global ? 1.f : 1.f / l;
-      // Query-side mask: the output row of a padding token is 0 (global
-      // rows are zeroed when their chunks are combined).
-      if (p.mask_q && write && !im.global && !p.key_mask[(size_t)im.b * p.L + tq]) inv = 0.f;
+      // Rows of a middle window or of an unchunked global item are final
+      // here; a global chunk leaves an unnormalised partial (m, l, O).
+      const bool whole = !im.global || a.geo.nchunks == 1;
+      float inv = whole ? 1.f / l : 1.f;
+      // Query-side mask: the output row of a padding token is 0 (chunked
+      // global rows are zeroed when their chunks are combined).
+      if (p.mask_q && write && whole && !p.key_mask[(size_t)im.b * p.L + tq]) inv = 0.f;
       const size_t grow = (size_t)im.bh * p.L + (size_t)(write ? im.t[half] : 0) * kTile + r64;
       float* part = p.part +
                     ((((size_t)im.bh * a.geo.n_git + im.gi) * a.geo.nchunks + im.chunk) * 128 +
@@ -510,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // S MMA that read it has completed (they precede the last P V), and the
       // producer refills the slot only after this item's list_empty.
       uint8_t* stage = Qs + slot * 2 * kTileBytes + quarter * 4096;
-      const bool tma_out = write && !im.global;
+      const bool tma_out = write && whole;
       // Not unrolled: runs once per item, so a small loop body costs less
       // instruction fetch than four copies.
 #pragma unroll 1
@@ -522,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           float v[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(o[e]) * inv;
-          if (!im.global) {
+          if (whole) {
             // 16-byte chunks 2 q16 and 2 q16 + 1 of this row, 128-byte swizzle
             // (chunk index XOR row mod 8), as the store's tensor map expects.
             uint8_t* rowp = stage + lane * 128;
@@ -557,7 +560,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (tma_out) pend = slot;  // released after the store has read the rows
       if (write) {
-        if (!im.global) {
+        if (whole) {
           p.lse_out[grow] = (m + __log2f(l)) * (1.0f / kLog2e);
         } else {
           part[64] = m;
@@ -622,7 +625,7 @@ __global__ void __launch_bounds__(256) fwd_combine_kernel(const PairArgs a) {
 // ---- host side ----------------------------------------------------------
 
 size_t tc_fwd_part_bytes(const Problem& p) {
-  const Geom g = make_geom(p.L, p.bs);
+  const Geom g = make_geom(p);
   return (size_t)p.B * p.H * g.n_git * g.nchunks * 128 * kPartStride * sizeof(float);
 }
 
@@ -643,6 +646,7 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
   kernel<<<grid, kThreads, smem, s>>>(a, tm.q, tm.k, tm.v, tm.out32);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.geo.nchunks == 1) return cudaSuccess;  // global rows written whole
   e = marks->mark(s);
   if (e != cudaSuccess) return e;
   const size_t rows = (size_t)p.B * p.H * a.geo.n_git * 128;

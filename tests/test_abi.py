@@ -226,7 +226,8 @@ def test_launch_lists_follow_the_dispatch():
     tensor-core path for bf16 shapes (backward plans in one launch while a
     head's transposed adjacency fits in shared memory), one dK/dV launch
     below 16384 tokens and two from there (global key blocks with the hi/lo
-    split on their own), the CUDA-core path for fp32."""
+    split on their own), merge launches only where global rows are split
+    into chunks, the CUDA-core path for fp32."""
     import torch
     short = bb.make_desc(2, 4, 4096, 64, 64, 3, torch.bfloat16)
     assert _names(short, 0) == ["plan", "tc_fwd", "fwd_combine"]
@@ -238,7 +239,15 @@ def test_launch_lists_follow_the_dispatch():
     assert _names(opt, 1) == _names(short, 1)
     for bs in (32, 64, 128):
         long_ = bb.make_desc(1, 2, 16384, 64, bs, 3, torch.bfloat16)
+        assert _names(long_, 0) == ["plan", "tc_fwd", "fwd_combine"], bs
         assert _names(long_, 1) == ["plan", "tc_dq", "tc_dkdv", "tc_dkdv", "bwd_finish"], bs
+    # Enough work that a global row's 64 tiles run as one item: no chunk
+    # partials, so no merge launches (the BigBird-large and -base shapes).
+    for B, H in ((4, 16), (8, 12)):
+        for bs in (32, 64, 128):
+            whole = bb.make_desc(B, H, 4096, 64, bs, 3, torch.bfloat16)
+            assert _names(whole, 0) == ["plan", "tc_fwd"], (B, H, bs)
+            assert _names(whole, 1) == ["plan", "tc_dq", "tc_dkdv"], (B, H, bs)
     f32 = bb.make_desc(1, 2, 1024, 64, 64, 3, torch.float32)
     assert _names(f32, 0) == ["simt_fwd"]
     assert _names(f32, 1) == ["bwd_pre", "csr_build", "simt_dq", "simt_dkdv"]

@@ -86,18 +86,24 @@ __host__ __device__ inline Geom make_geom(int L, int bs, int chunk = 0) {
 }
 
 // Tiles per chunk of a global item for problem p.  A global row visits every
-// key tile (a global key block every query tile).  When one tile list holds
-// them all (nt <= kMaxT) and the rest of the problem gives the launch's CTAs
-// more work each than one such item (middle windows estimated at 8 + r
-// tiles), the item runs whole: it writes its rows directly and no partials
-// are merged.  Otherwise rows are split into chunks of kChunk tiles whose
-// partials are merged in a fixed order by a launch of their own.
+// key tile (a global key block every query tile).  Long chunks mean fewer
+// partials to write and merge, but an item must stay shorter than the work
+// each CTA of the launch gets (middle windows estimated at 8 + r tiles).
+//  - One tile list holds the whole row (nt <= kMaxT) and it balances: the
+//    item runs whole, writes its rows directly, and nothing is merged.
+//  - Below the length where the global key blocks get a dK/dV launch of
+//    their own, chunks of kMaxT tiles when they balance.
+//  - Otherwise chunks of kChunk tiles (the global key blocks' own launch
+//    needs many items to fill the GPU).
+// Chunk partials are merged in a fixed order by a launch of their own.
 __host__ __device__ inline int global_chunk_tiles(const Problem& p) {
   const Geom g = make_geom(p.L, p.bs);
-  if (g.nt > kMaxT) return kChunk;
   const long long work = (long long)p.B * p.H *
                          ((long long)g.n_mid * (8 + p.r) + (long long)g.n_git * g.nt);
-  return work >= (long long)kBalanceCtas * g.nt ? g.nt : kChunk;
+  if (g.nt <= kMaxT && work >= (long long)kBalanceCtas * g.nt) return g.nt;
+  if (g.nt > kMaxT && p.L < kSplitMinL && work >= (long long)kBalanceCtas * kMaxT)
+    return kMaxT;
+  return kChunk;
 }
 
 __host__ __device__ inline Geom make_geom(const Problem& p) {
@@ -229,9 +235,9 @@ __host__ __device__ __forceinline__ ItemMeta item_meta(const Geom& g, int H, int
 
 // Next work item of a launch, taken from its counter: the locs [loc0, loc0 +
 // nloc) of every (b, h), longest items first so the short ones fill the end
-// of the launch: middle windows, then the global chunks; whole (unchunked)
-// global items, which are longer than a window, before the windows.  False
-// when none is left.
+// of the launch: middle windows, then short global chunks; global items of
+// more than kChunk tiles, which are longer than a window, before the
+// windows.  False when none is left.
 __device__ __forceinline__ bool next_work(const Geom& g, int B, int H, int loc0, int nloc,
                                           int* ctr, int& b, int& h, int& loc) {
   const int nglob = g.n_git * g.nchunks;
@@ -242,7 +248,7 @@ __device__ __forceinline__ bool next_work(const Geom& g, int B, int H, int loc0,
   const int w = atomicAdd(ctr, 1);
   if (w >= BH * nloc) return false;
   int bh;
-  const bool glob_first = g.nchunks == 1;
+  const bool glob_first = g.chunk > kChunk;
   const int nfirst = glob_first ? ngl : nmid;
   if (w < BH * nfirst) {
     bh = w / nfirst;

@@ -610,12 +610,16 @@ __device__ __forceinline__ void walk_range(const Problem& p, const Geom& g,
 // so S^T / dP^T of tile g + 2 are computed as soon as the softmax has read
 // tile g's (and while it still works on it); the dV / dK MMAs of tile g
 // read P^T / dS^T, which the softmax of tile g + 2 overwrites only after
-// those MMAs completed.  With the hi/lo split (global key blocks at long
-// lengths) the low parts go over S^T / dP^T of the same tile, so there the
-// next S^T / dP^T of the buffer also waits for the dV / dK MMAs.
+// those MMAs completed.  The launch of the global key blocks at long
+// lengths (hi/lo split) keeps one S^T / dP^T buffer (128-191, 256-319) and
+// puts the double-buffered low parts of P^T / dS^T in the other halves
+// (192-255, 320-383): there S^T / dP^T of tile g + 1 are computed as soon
+// as the softmax has read tile g's.
 constexpr int kKvQStages = 8;  // query-tile stages (Q, dO, NL, D)
 constexpr uint32_t kKvTmemCols = 512;
 constexpr uint32_t kKvDK = 0, kKvDV = 64, kKvS = 128, kKvDP = 256, kKvP = 384, kKvDS = 448;
+// hi/lo split launch: low parts of P^T / dS^T, buffer b at + 32 b
+constexpr uint32_t kKvPL = kKvS + 64, kKvDSL = kKvDP + 64;
 
 struct KvBars {
   // K / V pair of item k in slot k & 1: kp_full = landed (and kitem[] of the
@@ -794,10 +798,12 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const int ti = tinfo[g % kTinfo];
         if (ti & kTinfoEnd) break;
         const int ps = ti & 1;
+        // S^T / dP^T buffer: g & 1, or the one buffer of the split launch
+        // (then used by every tile).
+        const int sb = kSplit ? 0 : b;
+        const uint32_t spar = kSplit ? (g & 1) : ((g >> 1) & 1);
         if (!mbar_wait(&bars.kp_full[ps], (ti >> 1) & 1, &abort_flag, p.status) ||
-            !mbar_wait(&bars.s_free[b], ((g >> 1) & 1) ^ 1, &abort_flag, p.status) ||
-            (kSplit &&
-             !mbar_wait(&bars.g_done[b], ((g >> 1) & 1) ^ 1, &abort_flag, p.status)))
+            !mbar_wait(&bars.s_free[sb], spar ^ 1, &abort_flag, p.status))
           break;
         tc_fence_after();
         const uint32_t kaddr = smem_u32(KV + ps * 4 * kTileBytes);
@@ -806,13 +812,13 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const uint32_t gaddr = qaddr + kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kKvS + b * 64, sdesc_sw128(kaddr + kk * 32, 16),
+          mma_ss(tmem + kKvS + sb * 64, sdesc_sw128(kaddr + kk * 32, 16),
                  sdesc_sw128(qaddr + kk * 32, 16), idS, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tmem + kKvDP + b * 64, sdesc_sw128(vaddr + kk * 32, 16),
+          mma_ss(tmem + kKvDP + sb * 64, sdesc_sw128(vaddr + kk * 32, 16),
                  sdesc_sw128(gaddr + kk * 32, 16), idS, kk > 0);
-        mma_commit(&bars.s_full[b]);
+        mma_commit(&bars.s_full[sb]);
         if (ti & 4) mma_commit(&bars.kp_empty[ps]);  // the pair's last reader
       }
     }
@@ -846,9 +852,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
           const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
           const uint32_t gaddr = qaddr + kTileBytes;
           // A operands: 16 query rows per K step = 8 TMEM columns of bf16
-          // pairs; the low parts of a split tile sit in the S^T / dP^T
-          // columns of the same buffer, query half hc at columns 32 hc ..
-          // 32 hc + 15.
+          // pairs (high and low parts alike).
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(tmem + kKvDV, tmem + kKvP + b * 32 + kk * 8,
@@ -863,11 +867,11 @@ __global__ void __launch_bounds__(kThreads1, 1)
             // keep ~16 bits instead of 8.
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ts(tmem + kKvDV, tmem + kKvS + b * 64 + kk * 8 + (kk >> 1) * 16,
+              mma_ts(tmem + kKvDV, tmem + kKvPL + b * 32 + kk * 8,
                      sdesc_sw128(gaddr + kk * 2048, 8192), idAcc, 1u);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_ts(tmem + kKvDK, tmem + kKvDP + b * 64 + kk * 8 + (kk >> 1) * 16,
+              mma_ts(tmem + kKvDK, tmem + kKvDSL + b * 32 + kk * 8,
                      sdesc_sw128(qaddr + kk * 2048, 8192), idAcc, 1u);
           }
           mma_commit(&bars.g_done[b]);
@@ -933,10 +937,12 @@ __global__ void __launch_bounds__(kThreads1, 1)
         if (kDrop && p.keep_bits && e + 1 < e1) kwn = keep_word(cur);
         const uint32_t g = u;
         const int b = g & 1;
+        const int sb = kSplit ? 0 : b;  // S^T / dP^T buffer (as the score warp)
         const uint32_t st = g % kKvQStages;
         // Do query rows of this warp's column half attend this key group?
         const bool att = (mask >> (gshift + hc)) & 1;
-        if (!mbar_wait(&bars.s_full[b], (g >> 1) & 1, &abort_flag, p.status)) {
+        if (!mbar_wait(&bars.s_full[sb], kSplit ? (g & 1) : ((g >> 1) & 1), &abort_flag,
+                       p.status)) {
           ok = false;
           break;
         }
@@ -952,18 +958,15 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const float* Ds = NLs + 64;
         uint32_t sv[32], dp[32];
         if (att) {
-          tmem_ld32(tmem + kKvS + b * 64 + hc * 32 + lane_off, sv);
-          tmem_ld32(tmem + kKvDP + b * 64 + hc * 32 + lane_off, dp);
+          tmem_ld32(tmem + kKvS + sb * 64 + hc * 32 + lane_off, sv);
+          tmem_ld32(tmem + kKvDP + sb * 64 + hc * 32 + lane_off, dp);
           tmem_ld_wait();
         }
-        if (!split) {
-          // S^T / dP^T of this buffer are in registers (with the split the
-          // low parts go back over them, and the score MMAs of the buffer's
-          // next tile wait for the gradient MMAs instead).
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bars.s_free[b]);
-        }
+        // S^T / dP^T of this buffer are in registers: the score MMAs may
+        // refill it.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_free[sb]);
         // Dropout keep bits of this lane's key against the half's 32 query
         // tokens (att is uniform over the warp, as the shuffles need).
         const uint32_t keep =
@@ -973,8 +976,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
                                              qtile * kTile + hc * 32, lane))
                 : 0u;
         // P^T and dS^T of the half (bf16 pairs, 16 columns each): high parts
-        // to the P^T / dS^T buffers, low parts (split tiles) over the S^T /
-        // dP^T columns just read.
+        // to the P^T / dS^T buffers, low parts (split tiles) to theirs.
         uint32_t ph[16], dh[16], pl[16], dl[16];
         if (att) {
 #pragma unroll
@@ -1046,16 +1048,13 @@ __global__ void __launch_bounds__(kThreads1, 1)
         tmem_st16(tmem + kKvP + b * 32 + hc * 16 + lane_off, ph);
         tmem_st16(tmem + kKvDS + b * 32 + hc * 16 + lane_off, dh);
         if (split) {
-          tmem_st16(tmem + kKvS + b * 64 + hc * 32 + lane_off, pl);
-          tmem_st16(tmem + kKvDP + b * 64 + hc * 32 + lane_off, dl);
+          tmem_st16(tmem + kKvPL + b * 32 + hc * 16 + lane_off, pl);
+          tmem_st16(tmem + kKvDSL + b * 32 + hc * 16 + lane_off, dl);
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if (split) mbar_arrive(&bars.s_free[b]);
-          mbar_arrive(&bars.p_full[b]);
-        }
+        if (lane == 0) mbar_arrive(&bars.p_full[b]);
         ++u;
       }
       if (!ok) break;

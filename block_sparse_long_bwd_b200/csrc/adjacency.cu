@@ -484,14 +484,14 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
                                                                int do_k, int do_dead) {
   __shared__ int cand[kPlanWarps][128];
   __shared__ int stage[kPlanWarps][kStageCap];
-  const Geom g = make_geom(p);
+  const Geom g = make_geom(p);    // query side
+  const Geom kg = make_kgeom(p);  // key side
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nitems = p.H * g.per_bh;
   // The work counters of the tensor-core launches that follow.
   if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
   const int id = blockIdx.x * kPlanWarps + warp;
-  const int nq = do_q ? nitems : 0;
-  const int nk = do_k ? nitems : 0;
+  const int nq = do_q ? p.H * g.per_bh : 0;
+  const int nk = do_k ? p.H * kg.per_bh : 0;
   if (do_dead && id >= nq + nk) {
     const int x = id - nq - nk;
     if (x < p.B * p.tdead_words) dead_tile_word(p, g.nt, x / p.tdead_words, x % p.tdead_words, lane);
@@ -499,10 +499,10 @@ __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do
   }
   if (id < nq) {
     plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], stage[warp], lane);
-  } else if (do_k && id - nq < nitems) {
+  } else if (id - nq < nk) {
     const int k = id - nq;
-    const int h = k / g.per_bh;
-    plan_k_item(p, g, h, k % g.per_bh, p.csr_offs + (size_t)h * (g.nb + 1),
+    const int h = k / kg.per_bh;
+    plan_k_item(p, kg, h, k % kg.per_bh, p.csr_offs + (size_t)h * (kg.nb + 1),
                 p.csr_list + (size_t)h * p.csr_cap, stage[warp], cand[warp], lane);
   }
 }
@@ -606,7 +606,8 @@ __global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, i
   extern __shared__ int csr_sm[];
   __shared__ int cand[kFusedWarps][128];
   __shared__ int merged[kFusedWarps][128];
-  const Geom g = make_geom(p);
+  const Geom g = make_geom(p);    // query side
+  const Geom kg = make_kgeom(p);  // key side
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (blockIdx.x == 0 && threadIdx.x < 4) p.sched[threadIdx.x] = 0;
   if ((int)blockIdx.x < qctas) {
@@ -619,8 +620,8 @@ __global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, i
   const int h = kb / kslices, slice = kb % kslices;
   int* offs;
   const int* list = build_head_csr(p, h, csr_sm, offs);
-  for (int loc = slice * kFusedWarps + warp; loc < g.per_bh; loc += kslices * kFusedWarps)
-    plan_k_item(p, g, h, loc, offs, list, nullptr, cand[warp], lane);
+  for (int loc = slice * kFusedWarps + warp; loc < kg.per_bh; loc += kslices * kFusedWarps)
+    plan_k_item(p, kg, h, loc, offs, list, nullptr, cand[warp], lane);
 }
 
 size_t fused_plan_smem(const Problem& p) {
@@ -637,7 +638,7 @@ cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s) {
   const int qctas = (nitems + kFusedWarps - 1) / kFusedWarps;
   // One key-side item per warp (each CTA rebuilds its head's small
   // adjacency, so more CTAs per head cost only parallel work).
-  const int kslices = max(1, (g.per_bh + kFusedWarps - 1) / kFusedWarps);
+  const int kslices = max(1, (make_kgeom(p).per_bh + kFusedWarps - 1) / kFusedWarps);
   const size_t smem = fused_plan_smem(p);
   cudaError_t e = cudaFuncSetAttribute(
       plan_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -658,6 +659,8 @@ cudaError_t launch_bwd_pre(const Problem& p, cudaStream_t s) {
 
 size_t tc_items_per_bh(const Problem& p) { return make_geom(p).per_bh; }
 
+size_t tc_key_items_per_bh(const Problem& p) { return make_kgeom(p).per_bh; }
+
 size_t tc_qplan_bytes(const Problem& p) {
   return (size_t)p.H * tc_items_per_bh(p) * sizeof(TileList);
 }
@@ -674,9 +677,10 @@ int tc_tdead_words(const Problem& p) { return 1 + (make_geom(p).nt + 31) / 32; }
 
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
   const int items = p.H * (int)tc_items_per_bh(p);
+  const int kitems = key_side ? p.H * (int)tc_key_items_per_bh(p) : 0;
   // The forward with a key mask also writes its masked-tile bitmap.
   const int dead = (!key_side && p.key_mask && p.tdead) ? 1 : 0;
-  const int n = items * (key_side ? 2 : 1) + (dead ? p.B * p.tdead_words : 0);
+  const int n = items + kitems + (dead ? p.B * p.tdead_words : 0);
   plan_kernel<<<(n + kPlanWarps - 1) / kPlanWarps, 32 * kPlanWarps, 0, s>>>(
       p, 1, key_side ? 1 : 0, dead);
   return cudaGetLastError();

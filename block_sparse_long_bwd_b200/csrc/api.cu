@@ -41,7 +41,7 @@ WsLayout ws_layout(const Problem& p, int pass) {
       w.qplan_off = off;
       off = align_up(off + tc_qplan_bytes(p), 256);
       w.kof_off = off;
-      off = align_up(off + ((size_t)p.H * tc_items_per_bh(p) * 2 + p.H) * sizeof(int), 256);
+      off = align_up(off + ((size_t)p.H * tc_key_items_per_bh(p) * 2 + p.H) * sizeof(int), 256);
       w.kplan_off = off;
       off = align_up(off + (size_t)p.H * tc_kplan_cap(p) * sizeof(uint32_t), 256);
       w.total = off;
@@ -362,7 +362,7 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
   if (pass == 0) {
     const bool tc = tc_fwd_supported(p);
     *names = tc ? kFwdTc : kFwdSimt;
-    *n = tc ? (tc_global_rows_chunked(p) ? 3 : 2) : 1;
+    *n = tc ? (tc_global_rows_chunked(p, 0) ? 3 : 2) : 1;
   } else {
     if (!tc_bwd_supported(p)) {
       *names = kBwdSimt;
@@ -377,7 +377,7 @@ static int launch_plan(const bb_attn_desc* desc, int pass,
     const bool two = tc_dkdv_launches(p) == 2;
     const char* const* tail = two ? kBwdTcTail2 : kBwdTcTail1;
     // The merge launch only when global rows are chunked.
-    const int nt = (two ? 4 : 3) - (tc_global_rows_chunked(p) ? 0 : 1);
+    const int nt = (two ? 4 : 3) - (tc_global_rows_chunked(p, 1) ? 0 : 1);
     for (int i = 0; i < nt; ++i) buf[c++] = tail[i];
     *names = buf;
     *n = c;

@@ -130,15 +130,17 @@ size_t tc_qplan_bytes(const Problem& p);
 // bit per 64-key tile).
 int tc_tdead_words(const Problem& p);
 int tc_kplan_cap(const Problem& p);
-size_t tc_items_per_bh(const Problem& p);
+size_t tc_items_per_bh(const Problem& p);      // query side
+size_t tc_key_items_per_bh(const Problem& p);  // key side
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s);
 size_t tc_bwd_extra_bytes(const Problem& p);
 // Number of dK/dV launches of the tensor-core backward (1, or 2 at lengths
 // where the global key blocks run with the hi/lo split on their own).
 int tc_dkdv_launches(const Problem& p);
-// True when global rows are split into chunks whose partials a merge launch
-// (fwd_combine / bwd_finish) combines; false when they run whole.
-bool tc_global_rows_chunked(const Problem& p);
+// True when the forward's (pass 0) or the backward's (pass 1) global rows
+// are split into chunks whose partials a merge launch (fwd_combine /
+// bwd_finish) combines; false when they run whole.
+bool tc_global_rows_chunked(const Problem& p, int pass);
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks);
 

@@ -52,11 +52,12 @@ constexpr int kKvStages = 3;
 constexpr uint32_t kQStageBytes = 2 * kTileBytes + 1024;  // dK/dV: Q, dO, NL, D
 
 struct BwdArgs {
-  PairArgs qa;       // items: query side (dq) and, mirrored, key side (dkdv)
-  // Key-side items this dK/dV launch takes: per (b, h) the locs
-  // [kloc0, kloc0 + kgeo.per_bh) (kgeo is qa.geo with per_bh narrowed).
+  PairArgs qa;       // query side (dq): problem, geometry, items
+  // Key side (dkdv): its geometry (the query side's items, with its own
+  // chunking of the global key blocks) and the items this launch takes:
+  // per (b, h) the locs [kloc0, kloc0 + knloc).
   Geom kgeo;
-  int kitems, kloc0;
+  int kitems, kloc0, knloc;
   int* kctr;  // this launch's work counter
   float* D;          // [B*H*L]
   float* NL;         // [B*H*L]: -lse * log2(e)
@@ -715,17 +716,16 @@ __global__ void __launch_bounds__(kThreads1, 1)
         // Items are taken from the launch's counter (middle windows first);
         // the slot's (b, h, loc) is published by the kp_full arrive.
         int ib, ih, iloc;
-        if (!next_work(ba.qa.geo, p.B, p.H, ba.kloc0, ba.kgeo.per_bh, ba.kctr, ib, ih,
-                       iloc)) {
+        if (!next_work(ba.kgeo, p.B, p.H, ba.kloc0, ba.knloc, ba.kctr, ib, ih, iloc)) {
           kitem[ps] = make_int4(0, 0, 0, 0);
           mbar_arrive_release(&bars.kp_full[ps]);
           break;
         }
         kitem[ps] = make_int4(ib, ih, iloc, 1);
-        const ItemMeta it = item_meta_at(ba.qa.geo, ib, ih, p.H, iloc);
+        const ItemMeta it = item_meta_at(ba.kgeo, ib, ih, p.H, iloc);
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
-        walk_range(p, ba.qa.geo, it, e0, e1);
+        walk_range(p, ba.kgeo, it, e0, e1);
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
         uint8_t* kv = KV + ps * 4 * kTileBytes;
@@ -832,9 +832,9 @@ __global__ void __launch_bounds__(kThreads1, 1)
       if (!mbar_wait(&bars.kp_full[ps], (k >> 1) & 1, &abort_flag, p.status)) break;
       const int4 wi = kitem[ps];
       if (!wi.w) break;
-      const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
+      const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
       int w0, w1;
-      walk_range(p, ba.qa.geo, it, w0, w1);
+      walk_range(p, ba.kgeo, it, w0, w1);
       const int nwalk = w1 - w0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
@@ -902,12 +902,12 @@ __global__ void __launch_bounds__(kThreads1, 1)
       if (!mbar_wait(&bars.kp_full[ps], (k >> 1) & 1, &abort_flag, p.status)) break;
       const int4 wi = kitem[ps];
       if (!wi.w) break;
-      const ItemMeta it = item_meta_at(ba.qa.geo, wi.x, wi.y, p.H, wi.z);
+      const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
       int e0, e1;
-      walk_range(p, ba.qa.geo, it, e0, e1);
+      walk_range(p, ba.kgeo, it, e0, e1);
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;
@@ -1070,12 +1070,12 @@ __global__ void __launch_bounds__(kThreads1, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty);
       if (rvalid) {
-        if (!it.global || ba.qa.geo.nchunks == 1) {  // final rows (no chunk partials)
+        if (!it.global || ba.kgeo.nchunks == 1) {  // final rows (no chunk partials)
           store_grad_half(p, p.dk, krow, hc * 32, kx, p.scale);
           store_grad_half(p, p.dv, krow, hc * 32, vx, 1.0f);
         } else {
-          float* dst = ba.kvpart + ((((size_t)it.bh * ba.qa.geo.n_git + it.gi) *
-                                     ba.qa.geo.nchunks + it.chunk) * 128 + row) * 128;
+          float* dst = ba.kvpart + ((((size_t)it.bh * ba.kgeo.n_git + it.gi) *
+                                     ba.kgeo.nchunks + it.chunk) * 128 + row) * 128;
           store_part32(dst + hc * 32, kx);
           store_part32(dst + 64 + hc * 32, vx);
         }
@@ -1091,12 +1091,26 @@ __global__ void __launch_bounds__(kThreads1, 1)
   }
 }
 
+// Element pair 2 lane, 2 lane + 1 of gradient row `grow` (fp32 or the I/O
+// type, rounded once).
+__device__ __forceinline__ void store_grad_pair(const Problem& p, void* base, size_t grow,
+                                                int lane, float x, float y) {
+  if (p.grad_f32)
+    reinterpret_cast<float2*>(static_cast<float*>(base) + grow * kHeadDim)[lane] =
+        make_float2(x, y);
+  else
+    reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(base) + grow * kHeadDim)[lane] =
+        pack_bf16(x, y);
+}
+
 // One warp per row of a global item (query rows for dQ, key rows for
 // dK / dV: both sides use the same tiles); lanes over d.  Chunks are summed
-// in a fixed order; rows outside the global blocks are skipped.
+// in a fixed order; rows outside the global blocks are skipped.  Each side
+// is merged only when its global rows were split into chunks.
 __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
   const Problem& p = ba.qa.p;
-  const Geom& g = ba.qa.geo;
+  const Geom& g = ba.qa.geo;  // query side
+  const Geom& kg = ba.kgeo;   // key side (same rows, its own chunks)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const size_t id = (size_t)blockIdx.x * 8 + warp;  // over bh x gi x 128
   const size_t total = (size_t)p.B * p.H * g.n_git * 128;
@@ -1108,47 +1122,45 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(const BwdArgs ba) {
   item_rows(g, true, gi, t, gvalid);
   if (!((gvalid >> (row >> 5)) & 1)) return;
   const size_t grow = bh * p.L + (size_t)t[row >> 6] * kTile + (row & 63);
-  const size_t ib = (bh * g.n_git + gi) * g.nchunks;
-  float q0 = 0.f, q1 = 0.f, k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
   // Unrolled so that several chunks' loads are in flight at once (the sums
   // keep the chunk order).
+  if (g.nchunks > 1) {
+    const size_t ib = (bh * g.n_git + gi) * g.nchunks;
+    float q0 = 0.f, q1 = 0.f;
 #pragma unroll 8
-  for (int c = 0; c < g.nchunks; ++c) {
-    const float2 x = reinterpret_cast<const float2*>(
-        ba.dqpart + ((ib + c) * 128 + row) * 64)[lane];
-    q0 += x.x;
-    q1 += x.y;
-    const float* src = ba.kvpart + ((ib + c) * 128 + row) * 128;
-    const float2 xk = reinterpret_cast<const float2*>(src)[lane];
-    const float2 xv = reinterpret_cast<const float2*>(src + 64)[lane];
-    k0 += xk.x;
-    k1 += xk.y;
-    v0 += xv.x;
-    v1 += xv.y;
+    for (int c = 0; c < g.nchunks; ++c) {
+      const float2 x = reinterpret_cast<const float2*>(
+          ba.dqpart + ((ib + c) * 128 + row) * 64)[lane];
+      q0 += x.x;
+      q1 += x.y;
+    }
+    store_grad_pair(p, p.dq, grow, lane, q0 * p.scale, q1 * p.scale);
   }
-  if (p.grad_f32) {
-    reinterpret_cast<float2*>(static_cast<float*>(p.dq) + grow * kHeadDim)[lane] =
-        make_float2(q0 * p.scale, q1 * p.scale);
-    reinterpret_cast<float2*>(static_cast<float*>(p.dk) + grow * kHeadDim)[lane] =
-        make_float2(k0 * p.scale, k1 * p.scale);
-    reinterpret_cast<float2*>(static_cast<float*>(p.dv) + grow * kHeadDim)[lane] =
-        make_float2(v0, v1);
-    return;
+  if (kg.nchunks > 1) {
+    const size_t ib = (bh * kg.n_git + gi) * kg.nchunks;
+    float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+#pragma unroll 8
+    for (int c = 0; c < kg.nchunks; ++c) {
+      const float* src = ba.kvpart + ((ib + c) * 128 + row) * 128;
+      const float2 xk = reinterpret_cast<const float2*>(src)[lane];
+      const float2 xv = reinterpret_cast<const float2*>(src + 64)[lane];
+      k0 += xk.x;
+      k1 += xk.y;
+      v0 += xv.x;
+      v1 += xv.y;
+    }
+    store_grad_pair(p, p.dk, grow, lane, k0 * p.scale, k1 * p.scale);
+    store_grad_pair(p, p.dv, grow, lane, v0, v1);
   }
-  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dq) + grow * kHeadDim)[lane] =
-      pack_bf16(q0 * p.scale, q1 * p.scale);
-  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dk) + grow * kHeadDim)[lane] =
-      pack_bf16(k0 * p.scale, k1 * p.scale);
-  reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.dv) + grow * kHeadDim)[lane] =
-      pack_bf16(v0, v1);
 }
 
 BwdArgs make_bwd_args(const Problem& p) {
   BwdArgs ba;
   ba.qa = make_pair_args(p);
-  ba.kgeo = ba.qa.geo;
-  ba.kitems = ba.qa.items;
+  ba.kgeo = make_kgeom(p);
+  ba.kitems = p.B * p.H * ba.kgeo.per_bh;
   ba.kloc0 = 0;
+  ba.knloc = ba.kgeo.per_bh;
   ba.kctr = p.sched + 1;
   return ba;
 }
@@ -1162,27 +1174,30 @@ int tc_dkdv_launches(const Problem& p) {
   return (p.L >= kSplitMinL && make_geom(p).n_mid > 0) ? 2 : 1;
 }
 
-bool tc_global_rows_chunked(const Problem& p) { return make_geom(p).nchunks > 1; }
+bool tc_global_rows_chunked(const Problem& p, int pass) {
+  return make_geom(p).nchunks > 1 || (pass == 1 && make_kgeom(p).nchunks > 1);
+}
 
 size_t tc_bwd_extra_bytes(const Problem& p) {
   const size_t rows = (size_t)p.B * p.H * p.L;
-  const Geom g = make_geom(p);
-  const size_t units = (size_t)p.B * p.H * g.n_git * g.nchunks * 128;
-  return rows * 4 /* NL */ + units * 64 * 4 + units * 128 * 4 + 3 * 256;
+  const Geom g = make_geom(p), kg = make_kgeom(p);
+  const size_t uq = (size_t)p.B * p.H * g.n_git * g.nchunks * 128;
+  const size_t uk = (size_t)p.B * p.H * kg.n_git * kg.nchunks * 128;
+  return rows * 4 /* NL */ + uq * 64 * 4 + uk * 128 * 4 + 3 * 256;
 }
 
 cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
   BwdArgs ba = make_bwd_args(p);
   const size_t rows = (size_t)p.B * p.H * p.L;
-  const size_t units = (size_t)p.B * p.H * ba.qa.geo.n_git * ba.qa.geo.nchunks * 128;
+  const size_t uq = (size_t)p.B * p.H * ba.qa.geo.n_git * ba.qa.geo.nchunks * 128;
   auto al = [](size_t x) { return (x + 255) / 256 * 256; };
   uint8_t* x = reinterpret_cast<uint8_t*>(p.part);
   ba.D = p.D;
   ba.NL = reinterpret_cast<float*>(x);
   x += al(rows * 4);
   ba.dqpart = reinterpret_cast<float*>(x);
-  x += al(units * 64 * 4);
+  x += al(uq * 64 * 4);
   ba.kvpart = reinterpret_cast<float*>(x);
 
   int dev = 0, sms = 148;
@@ -1205,7 +1220,7 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   const size_t smem_kv = 1024 + 2 * 4 * kTileBytes + kKvQStages * kQStageBytes;
   // From kSplitMinL the global key blocks' items (the only ones with the
   // hi/lo split) run in a launch of their own, the middle windows without.
-  const Geom& g = ba.qa.geo;
+  const Geom& g = ba.kgeo;
   const int nglob = g.n_git * g.nchunks;
   struct Part {
     bool split;
@@ -1221,9 +1236,8 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   }
   for (int i = 0; i < nparts; ++i) {
     BwdArgs bk = ba;
-    bk.kgeo = g;
-    bk.kgeo.per_bh = parts[i].per_bh;
     bk.kloc0 = parts[i].loc0;
+    bk.knloc = parts[i].per_bh;
     bk.kitems = p.B * p.H * parts[i].per_bh;
     bk.kctr = p.sched + 1 + i;  // sched[0]: dQ
     auto* kv_kernel = parts[i].split ? (drop ? tc_dkdv_kernel<true, true>
@@ -1243,8 +1257,8 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     if (e != cudaSuccess) return e;
   }
 
-  // Global rows written whole: no chunk partials to merge.
-  if (g.nchunks == 1) return cudaSuccess;
+  // Global rows written whole on both sides: no chunk partials to merge.
+  if (ba.qa.geo.nchunks == 1 && g.nchunks == 1) return cudaSuccess;
   e = marks->mark(s);
   if (e != cudaSuccess) return e;
   const size_t frows = (size_t)p.B * p.H * ba.qa.geo.n_git * 128;

@@ -91,23 +91,27 @@ __host__ __device__ inline Geom make_geom(int L, int bs, int chunk = 0) {
 // each CTA of the launch gets (middle windows estimated at 8 + r tiles).
 //  - One tile list holds the whole row (nt <= kMaxT) and it balances: the
 //    item runs whole, writes its rows directly, and nothing is merged.
-//  - Below the length where the global key blocks get a dK/dV launch of
-//    their own, chunks of kMaxT tiles when they balance.
-//  - Otherwise chunks of kChunk tiles (the global key blocks' own launch
-//    needs many items to fill the GPU).
+//  - Else chunks of kMaxT tiles when they balance, of kChunk otherwise.
 // Chunk partials are merged in a fixed order by a launch of their own.
 __host__ __device__ inline int global_chunk_tiles(const Problem& p) {
   const Geom g = make_geom(p.L, p.bs);
   const long long work = (long long)p.B * p.H *
                          ((long long)g.n_mid * (8 + p.r) + (long long)g.n_git * g.nt);
   if (g.nt <= kMaxT && work >= (long long)kBalanceCtas * g.nt) return g.nt;
-  if (g.nt > kMaxT && p.L < kSplitMinL && work >= (long long)kBalanceCtas * kMaxT)
-    return kMaxT;
+  if (g.nt > kMaxT && work >= (long long)kBalanceCtas * kMaxT) return kMaxT;
   return kChunk;
 }
 
+// Query-side geometry (forward, dQ).
 __host__ __device__ inline Geom make_geom(const Problem& p) {
   return make_geom(p.L, p.bs, global_chunk_tiles(p));
+}
+
+// Key-side geometry (dK/dV): the same items, except that from the length
+// where the global key blocks run in a launch of their own their chunks are
+// kChunk query tiles (that launch holds only them and needs many items).
+__host__ __device__ inline Geom make_kgeom(const Problem& p) {
+  return make_geom(p.L, p.bs, p.L >= kSplitMinL ? kChunk : global_chunk_tiles(p));
 }
 
 // Block of token row `tok`.

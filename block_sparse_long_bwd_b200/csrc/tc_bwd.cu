@@ -201,7 +201,8 @@ struct DqBars {
   uint64_t s_full, s_free, dp_free, p_full, dq_done, dq_full, dq_empty;
 };
 
-template <bool kDrop>
+// kMask: a key mask is given (else every key is attended).
+template <bool kDrop, bool kMask>
 __global__ void __launch_bounds__(kThreads2, 2)
     tc_dq_kernel(const __grid_constant__ BwdArgs ba,
                  const __grid_constant__ CUtensorMap tmQ,
@@ -498,7 +499,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free);
-        const uint64_t kb = (m2 && p.key_mask) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
+        const uint64_t kb = (kMask && m2) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
         const uint64_t db = (kDrop && m2)
                                 ? (p.keep_bits ? dbs : keep_row64(p, im.b, im.h, tq, L.tile[t]))
                                 : 0ull;
@@ -1206,7 +1207,9 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
 
   const size_t smem_dq = 1024 + (4 + 2 * kKvStages) * kTileBytes;
   const bool drop = p.drop_thr != 0;
-  auto* dq_kernel = drop ? tc_dq_kernel<true> : tc_dq_kernel<false>;
+  const bool masked = p.key_mask != nullptr;
+  auto* dq_kernel = drop ? (masked ? tc_dq_kernel<true, true> : tc_dq_kernel<true, false>)
+                         : (masked ? tc_dq_kernel<false, true> : tc_dq_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(
       dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
   if (e != cudaSuccess) return e;

@@ -70,7 +70,10 @@ __device__ __forceinline__ float max64(const float* z) {
 
 // kDrop: seeded attention dropout on the probabilities that enter P V (the
 // row sums, hence the lse, stay those of the undropped softmax).
-template <bool kDrop>
+// kWhole: global items run whole (one chunk), so every row of every item is
+// final in this kernel; else global items leave chunk partials.
+// kMask: a key mask is given (else every key is attended).
+template <bool kDrop, bool kWhole, bool kMask>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
@@ -393,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
         if (att) {
-          const uint64_t kb = p.key_mask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
+          const uint64_t kb = kMask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
           const uint64_t hb = half_bits(m2);
           float mx;
           if (kb == ~0ull && hb == ~0ull && c > 0.f) {
@@ -498,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const bool write = (im.gvalid >> quarter) & 1;
       // Rows of a middle window or of an unchunked global item are final
       // here; a global chunk leaves an unnormalised partial (m, l, O).
-      const bool whole = !im.global || a.geo.nchunks == 1;
+      const bool whole = kWhole || !im.global;
       float inv = whole ? 1.f / l : 1.f;
       // Query-side mask: the output row of a padding token is 0 (chunked
       // global rows are zeroed when their chunks are combined).
@@ -635,7 +638,17 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
                           cudaStream_t s, EventMarks* marks) {
   const PairArgs a = make_pair_args(p);
   const size_t smem = 1024 + (2 * 2 + 2 * kNST) * kTileBytes;
-  auto* kernel = p.drop_thr ? tc_fwd_kernel<true> : tc_fwd_kernel<false>;
+  const bool whole = a.geo.nchunks == 1;
+  const bool masked = p.key_mask != nullptr;
+  using Kernel = void (*)(const PairArgs, const CUtensorMap, const CUtensorMap,
+                          const CUtensorMap, const CUtensorMap);
+  // [dropout][whole][mask]
+  static const Kernel kernels[2][2][2] = {
+      {{tc_fwd_kernel<false, false, false>, tc_fwd_kernel<false, false, true>},
+       {tc_fwd_kernel<false, true, false>, tc_fwd_kernel<false, true, true>}},
+      {{tc_fwd_kernel<true, false, false>, tc_fwd_kernel<true, false, true>},
+       {tc_fwd_kernel<true, true, false>, tc_fwd_kernel<true, true, true>}}};
+  const Kernel kernel = kernels[p.drop_thr ? 1 : 0][whole ? 1 : 0][masked ? 1 : 0];
   cudaError_t e = cudaFuncSetAttribute(
       kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -202,7 +202,8 @@ struct DqBars {
 };
 
 // kMask: a key mask is given (else every key is attended).
-template <bool kDrop, bool kMask>
+// kWhole: global rows run whole (every item's rows are final here).
+template <bool kDrop, bool kMask, bool kWhole>
 __global__ void __launch_bounds__(kThreads2, 2)
     tc_dq_kernel(const __grid_constant__ BwdArgs ba,
                  const __grid_constant__ CUtensorMap tmQ,
@@ -563,7 +564,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.dq_empty);
       if (rvalid) {
-        if (!im.global || a.geo.nchunks == 1) {  // final rows (no chunk partials)
+        if (kWhole || !im.global) {  // final rows (no chunk partials)
           store_grad_row(p, p.dq, grow, q0, q1, p.scale);
         } else {
           float4* dst = reinterpret_cast<float4*>(
@@ -641,7 +642,8 @@ struct KvBars {
 // lengths' register budget.
 // kDrop: seeded attention dropout (P^T kept times 1 / keep probability for
 // dV; dS^T = P^T (m dP^T - D)).
-template <bool kSplit, bool kDrop>
+// kWhole: the global key blocks run whole (every item's rows are final here).
+template <bool kSplit, bool kDrop, bool kWhole>
 __global__ void __launch_bounds__(kThreads1, 1)
     tc_dkdv_kernel(const __grid_constant__ BwdArgs ba,
                    const __grid_constant__ CUtensorMap tmQ,
@@ -1071,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty);
       if (rvalid) {
-        if (!it.global || ba.kgeo.nchunks == 1) {  // final rows (no chunk partials)
+        if (kWhole || !it.global) {  // final rows (no chunk partials)
           store_grad_half(p, p.dk, krow, hc * 32, kx, p.scale);
           store_grad_half(p, p.dv, krow, hc * 32, vx, 1.0f);
         } else {
@@ -1208,8 +1210,16 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
   const size_t smem_dq = 1024 + (4 + 2 * kKvStages) * kTileBytes;
   const bool drop = p.drop_thr != 0;
   const bool masked = p.key_mask != nullptr;
-  auto* dq_kernel = drop ? (masked ? tc_dq_kernel<true, true> : tc_dq_kernel<true, false>)
-                         : (masked ? tc_dq_kernel<false, true> : tc_dq_kernel<false, false>);
+  using DqKernel = void (*)(const BwdArgs, const CUtensorMap, const CUtensorMap,
+                            const CUtensorMap, const CUtensorMap);
+  // [dropout][mask][whole]
+  static const DqKernel dq_kernels[2][2][2] = {
+      {{tc_dq_kernel<false, false, false>, tc_dq_kernel<false, false, true>},
+       {tc_dq_kernel<false, true, false>, tc_dq_kernel<false, true, true>}},
+      {{tc_dq_kernel<true, false, false>, tc_dq_kernel<true, false, true>},
+       {tc_dq_kernel<true, true, false>, tc_dq_kernel<true, true, true>}}};
+  const DqKernel dq_kernel =
+      dq_kernels[drop ? 1 : 0][masked ? 1 : 0][ba.qa.geo.nchunks == 1 ? 1 : 0];
   cudaError_t e = cudaFuncSetAttribute(
       dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_dq);
   if (e != cudaSuccess) return e;
@@ -1243,10 +1253,15 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     bk.knloc = parts[i].per_bh;
     bk.kitems = p.B * p.H * parts[i].per_bh;
     bk.kctr = p.sched + 1 + i;  // sched[0]: dQ
-    auto* kv_kernel = parts[i].split ? (drop ? tc_dkdv_kernel<true, true>
-                                             : tc_dkdv_kernel<true, false>)
-                                     : (drop ? tc_dkdv_kernel<false, true>
-                                             : tc_dkdv_kernel<false, false>);
+    // The split launch holds only chunked global items.
+    const bool kwhole = g.nchunks == 1;
+    auto* kv_kernel =
+        parts[i].split ? (drop ? tc_dkdv_kernel<true, true, false>
+                               : tc_dkdv_kernel<true, false, false>)
+                       : (drop ? (kwhole ? tc_dkdv_kernel<false, true, true>
+                                         : tc_dkdv_kernel<false, true, false>)
+                               : (kwhole ? tc_dkdv_kernel<false, false, true>
+                                         : tc_dkdv_kernel<false, false, false>));
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);
     if (e != cudaSuccess) return e;

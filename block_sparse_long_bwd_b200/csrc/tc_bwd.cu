@@ -653,6 +653,10 @@ __global__ void __launch_bounds__(kThreads1, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ KvBars bars;
   __shared__ int4 kitem[2];  // (b, h, loc, 1) of the item in pair slot s; w = 0: no more items
+  // Walk of the item in pair slot s, as the loader read it: entries [x, y)
+  // of the head's walk area and the first two entries (so the other warps
+  // start the item without global loads).
+  __shared__ int4 kwalk[2];
   // flat tile g at g % kTinfo: pair slot | kp_full parity << 1 | last tile
   // of its item << 2, or kTinfoEnd
   __shared__ uint8_t tinfo[kTinfo];
@@ -729,6 +733,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.kgeo, it, e0, e1);
+        const uint32_t wfirst = e0 < e1 ? __ldg(walk + e0) : 0u;
+        kwalk[ps] = make_int4(e0, e1, (int)wfirst, e0 + 1 < e1 ? (int)__ldg(walk + e0 + 1) : 0);
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
         uint8_t* kv = KV + ps * 4 * kTileBytes;
@@ -741,7 +747,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
         kp_issued[ps] = 1;
         kp_par[ps] = (k >> 1) & 1;
         if (e1 == e0) mma_commit(&bars.kp_empty[ps]);  // no MMA reads this pair
-        uint32_t nxt = e0 < e1 ? __ldg(walk + e0) : 0u;  // loaded a tile ahead
+        uint32_t nxt = wfirst;  // loaded a tile ahead
         for (int e = e0; e < e1; ++e) {
           const int i = (int)(nxt & 0xFFFFu);  // query tile
           if (e + 1 < e1) nxt = __ldg(walk + e + 1);
@@ -836,11 +842,10 @@ __global__ void __launch_bounds__(kThreads1, 1)
       const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
-      int w0, w1;
-      walk_range(p, ba.kgeo, it, w0, w1);
-      const int nwalk = w1 - w0;
+      const int4 kw = kwalk[ps];
+      const int nwalk = kw.y - kw.x;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
+      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem, kwalk read
       for (int t = 0; t < nwalk; ++t) {
         const uint32_t g = u;
         const int b = g & 1;
@@ -906,11 +911,11 @@ __global__ void __launch_bounds__(kThreads1, 1)
       const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
+      const int4 kw = kwalk[ps];
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem read
+      if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem, kwalk read
       const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-      int e0, e1;
-      walk_range(p, ba.kgeo, it, e0, e1);
+      const int e0 = kw.x, e1 = kw.y;
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;
@@ -927,8 +932,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
         return __ldg(keep_ptr(p, it.bh, it.h, (int)(ent & 0xFFFFu) * kTile + hc * 32 + lane,
                               (int)(ktok & ~(size_t)31)));
       };
-      uint32_t cur = e0 < e1 ? __ldg(walk + e0) : 0u;
-      uint32_t nxt = e0 + 1 < e1 ? __ldg(walk + e0 + 1) : 0u;
+      uint32_t cur = (uint32_t)kw.z, nxt = (uint32_t)kw.w;
       uint32_t kwn = (kDrop && p.keep_bits && e0 < e1) ? keep_word(cur) : 0u;
       for (int e = e0; e < e1; ++e) {
         const uint32_t ent = cur;

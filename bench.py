@@ -98,6 +98,13 @@ def parse():
 def workload(name):
     if name in synth.WORKLOADS:
         return dict(synth.WORKLOADS[name])
+    if name == "base_train_l4096":
+        # The BigBird-base layer's padded batch through a training step,
+        # with the key mask also masking the query side.
+        cfg = dict(synth.WORKLOADS["base_fwd_l4096"])
+        cfg["passes"] = "fwd+bwd"
+        cfg["mask_queries"] = 1
+        return cfg
     if name.startswith("sweep_"):  # sweep_L_bs_r
         _, L, bs, r = name.split("_")
         return synth.sweep_point(int(L), int(bs), int(r))
@@ -319,7 +326,7 @@ def run_ours(args, world, rank, local):
     att = bb.Attention(B, H, L, bs, r, dt, d=cfg["d"], seed=synth.TABLE_SEED,
                        device=dev, dropout=args.dropout,
                        dropout_seed=args.dropout_seed,
-                       mask_queries=int(args.mask_queries),
+                       mask_queries=int(args.mask_queries or cfg.get("mask_queries", 0)),
                        keep_dropout_bits=not args.redraw_dropout)
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     g = inp["dout"].to(dev) if backward else None
@@ -473,7 +480,7 @@ def run_ours(args, world, rank, local):
                                          if att.dropout_bits is not None
                                          else "drawn in every pass")
                    if args.dropout else None,
-                   "mask_queries": bool(args.mask_queries),
+                   "mask_queries": bool(args.mask_queries or cfg.get("mask_queries", 0)),
                    "global_batch": B * world, "seq_len": L,
                    "parallelism": f"replicas x{world} (independent batches)",
                    "l2": "flushed between steps (256 MiB write, untimed)"},
@@ -676,7 +683,7 @@ def run_reference(args, world, rank):
         h = s % H
         drop = (oracle.Dropout(args.dropout, args.dropout_seed, b0=0, h0=h)
                 if args.dropout else None)
-        qm = km if args.mask_queries else None
+        qm = km if (args.mask_queries or cfg.get("mask_queries", 0)) else None
         oracle.forward(f(inp["q"], h), f(inp["k"], h), f(inp["v"], h), km,
                        table[h:h + 1], bs, dropout=drop, query_mask=qm)
         if backward:
@@ -708,7 +715,7 @@ def run_reference(args, world, rank):
         "config": {"workload": args.workload, "B": B, "H": H, "L": L,
                    "block_size": bs, "d": cfg["d"], "r": r,
                    "dropout": args.dropout,
-                   "mask_queries": bool(args.mask_queries),
+                   "mask_queries": bool(args.mask_queries or cfg.get("mask_queries", 0)),
                    "global_batch": B, "seq_len": L},
         "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
                          "cores": cores, "kind": "oracle", "sample": sample},
@@ -814,7 +821,7 @@ def time_workload(name, steps, dev, flush):
     B, H, L, bs, r = cfg["B"], cfg["H"], cfg["L"], cfg["block_size"], cfg["r"]
     inp = synth.make_inputs(cfg, with_grad=backward)
     att = bb.Attention(B, H, L, bs, r, synth.torch_dtype(cfg["dtype"]),
-                       d=cfg["d"], device=dev)
+                       d=cfg["d"], device=dev, mask_queries=cfg.get("mask_queries", 0))
     q, k, v = (inp[n].to(dev) for n in ("q", "k", "v"))
     g = inp["dout"].to(dev) if backward else None
     km = None if inp["key_mask"] is None else inp["key_mask"].to(dev)
@@ -934,12 +941,13 @@ def time_projections(name, B, L, hidden, H, steps, dev, flush, peaks):
 
 def sub_records(dev, peaks, sweep_steps=5):
     """The other workloads and the sweep, timed in the same run after the
-    headline: the BigBird-base forward (its padded batch), the 16K pattern
+    headline: the BigBird-base forward (its padded batch), the same batch
+    through a training step with the query-side mask, the 16K pattern
     (fwd+bwd), the layer's projections at the BigBird-large and -base
     widths, and every sweep point with the linear-in-L verdict."""
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     subs = {n: time_workload(n, 10, dev, flush)
-            for n in ("base_fwd_l4096", "long_l16384")}
+            for n in ("base_fwd_l4096", "base_train_l4096", "long_l16384")}
     subs["projections"] = [
         time_projections("bigbird_large_layer_l4096", 4, 4096, 1024, 16, 10, dev, flush, peaks),
         time_projections("bigbird_base_layer_l4096", 8, 4096, 768, 12, 10, dev, flush, peaks)]

@@ -450,7 +450,7 @@ __device__ void plan_k_item(const Problem& p, const Geom& g, int h, int loc,
   }
 }
 
-// One word of the forward's masked-tile bitmap (see Problem::tdead): warp w
+// One word of the masked-tile bitmap (see Problem::tdead): warp w
 // of batch b writes word w (w = 0: the flag word, from the first 32 keys;
 // w >= 1: tiles 32 (w - 1) .. 32 (w - 1) + 31, lane i testing the 64 keys of
 // one tile).
@@ -479,7 +479,7 @@ __device__ void dead_tile_word(const Problem& p, int nt, int b, int w, int lane)
 
 // Plans, one warp per item: query-side lists (do_q) and key-side walks
 // (do_k, after the CSR exists); with do_dead, then one warp per word of the
-// forward's masked-tile bitmap.
+// masked-tile bitmap.
 __global__ void __launch_bounds__(32 * kPlanWarps) plan_kernel(Problem p, int do_q,
                                                                int do_k, int do_dead) {
   __shared__ int cand[kPlanWarps][128];
@@ -598,11 +598,12 @@ __device__ int* build_head_csr(const Problem& p, int h, int* sm, int*& offs) {
 constexpr int kFusedWarps = 8;
 
 // Backward plans in one launch: the first qctas CTAs plan query-side items
-// (one warp each); the others each build one head's transposed adjacency in
+// (one warp each); the next dctas CTAs write the masked-tile bitmap (one
+// warp per word); the others each build one head's transposed adjacency in
 // shared memory and plan a slice of that head's key-side items from it
 // (kslices CTAs per head, so no CTA waits for another).
 __global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, int qctas,
-                                                                    int kslices) {
+                                                                    int dctas, int kslices) {
   extern __shared__ int csr_sm[];
   __shared__ int cand[kFusedWarps][128];
   __shared__ int merged[kFusedWarps][128];
@@ -616,7 +617,13 @@ __global__ void __launch_bounds__(32 * kFusedWarps) plan_bwd_kernel(Problem p, i
       plan_q_item(p, g, id / g.per_bh, id % g.per_bh, cand[warp], merged[warp], lane);
     return;
   }
-  const int kb = blockIdx.x - qctas;
+  if ((int)blockIdx.x < qctas + dctas) {
+    const int x = ((int)blockIdx.x - qctas) * kFusedWarps + warp;
+    if (x < p.B * p.tdead_words)
+      dead_tile_word(p, g.nt, x / p.tdead_words, x % p.tdead_words, lane);
+    return;
+  }
+  const int kb = blockIdx.x - qctas - dctas;
   const int h = kb / kslices, slice = kb % kslices;
   int* offs;
   const int* list = build_head_csr(p, h, csr_sm, offs);
@@ -639,11 +646,16 @@ cudaError_t launch_plan_bwd(const Problem& p, cudaStream_t s) {
   // One key-side item per warp (each CTA rebuilds its head's small
   // adjacency, so more CTAs per head cost only parallel work).
   const int kslices = max(1, (make_kgeom(p).per_bh + kFusedWarps - 1) / kFusedWarps);
+  // With a key mask, the masked-tile bitmap.
+  const int dctas = (p.key_mask && p.tdead)
+                        ? (p.B * p.tdead_words + kFusedWarps - 1) / kFusedWarps
+                        : 0;
   const size_t smem = fused_plan_smem(p);
   cudaError_t e = cudaFuncSetAttribute(
       plan_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  plan_bwd_kernel<<<qctas + p.H * kslices, 32 * kFusedWarps, smem, s>>>(p, qctas, kslices);
+  plan_bwd_kernel<<<qctas + dctas + p.H * kslices, 32 * kFusedWarps, smem, s>>>(p, qctas, dctas,
+                                                                                kslices);
   return cudaGetLastError();
 }
 
@@ -678,8 +690,8 @@ int tc_tdead_words(const Problem& p) { return 1 + (make_geom(p).nt + 31) / 32; }
 cudaError_t launch_plan(const Problem& p, bool key_side, cudaStream_t s) {
   const int items = p.H * (int)tc_items_per_bh(p);
   const int kitems = key_side ? p.H * (int)tc_key_items_per_bh(p) : 0;
-  // The forward with a key mask also writes its masked-tile bitmap.
-  const int dead = (!key_side && p.key_mask && p.tdead) ? 1 : 0;
+  // With a key mask the plans also write the masked-tile bitmap.
+  const int dead = (p.key_mask && p.tdead) ? 1 : 0;
   const int n = items + kitems + (dead ? p.B * p.tdead_words : 0);
   plan_kernel<<<(n + kPlanWarps - 1) / kPlanWarps, 32 * kPlanWarps, 0, s>>>(
       p, 1, key_side ? 1 : 0, dead);

@@ -44,6 +44,8 @@ WsLayout ws_layout(const Problem& p, int pass) {
       off = align_up(off + ((size_t)p.H * tc_key_items_per_bh(p) * 2 + p.H) * sizeof(int), 256);
       w.kplan_off = off;
       off = align_up(off + (size_t)p.H * tc_kplan_cap(p) * sizeof(uint32_t), 256);
+      w.tdead_off = off;
+      off = align_up(off + (size_t)p.B * tc_tdead_words(p) * sizeof(uint32_t), 256);
       w.total = off;
       return w;
     }

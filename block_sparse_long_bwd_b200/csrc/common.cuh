@@ -58,9 +58,10 @@ struct Problem {
                      // then [H] allocation counters
   uint32_t* kplan;   // [H][kcap] key-side walk entries
   int kcap;
-  // forward, with a key mask: per batch b, word 0 = 1 when key tiles may be
-  // skipped (a key among the first 32 is valid), then one bit per 64-key
-  // tile whose keys are all masked; [B][tdead_words]
+  // with a key mask: per batch b, word 0 = 1 when key tiles may be skipped
+  // (a key among the first 32 is valid), then one bit per 64-token tile
+  // whose keys are all masked; [B][tdead_words] (built by the plan launch of
+  // either pass)
   uint32_t* tdead;
   int tdead_words;
   // dropout keep decisions carried from the forward to the backward

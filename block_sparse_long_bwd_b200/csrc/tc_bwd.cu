@@ -195,7 +195,9 @@ __device__ __forceinline__ void dq_ds_half_drop(const uint32_t (&pv)[32],
 }
 
 struct DqBars {
-  uint64_t list_full[2], list_empty[2];
+  // list_full: the slot's tile list landed (the producer's bulk copy);
+  // list_ready: the list, compacted, and the item are published.
+  uint64_t list_full[2], list_ready[2], list_empty[2];
   uint64_t q_full, q_empty;
   uint64_t kv_full[kKvStages], kv_empty[kKvStages];
   uint64_t s_full, s_free, dp_free, p_full, dq_done, dq_full, dq_empty;
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
     abort_flag = 0;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars.list_full[s], 1);
+      mbar_init(&bars.list_ready[s], 1);
       mbar_init(&bars.list_empty[s], 5);
     }
     mbar_init(&bars.q_full, 1);
@@ -276,12 +279,12 @@ __global__ void __launch_bounds__(kThreads2, 2)
                        p.status))
           break;
         // Planned key-tile list: one bulk copy into the slot.
-        // Items are taken from the launch's counter (middle windows first);
-        // the slot's (b, h, loc) is published by the list_full arrive.
+        // Items are taken from the launch's counter (longest first); the
+        // slot's (b, h, loc) is published by the list_ready arrive.
         int ib, ih, iloc;
         if (!next_work(a.geo, p.B, p.H, 0, a.geo.per_bh, p.sched, ib, ih, iloc)) {
           item_sh[slot] = make_int4(0, 0, 0, 0);
-          mbar_arrive_release(&bars.list_full[slot]);
+          mbar_arrive_release(&bars.list_ready[slot]);
           break;
         }
         item_sh[slot] = make_int4(ib, ih, iloc, 1);
@@ -291,9 +294,32 @@ __global__ void __launch_bounds__(kThreads2, 2)
         bulk_load(&lists[slot],
                   static_cast<const TileList*>(p.qplan) + (size_t)m.h * a.geo.per_bh + m.loc,
                   sizeof(TileList), &bars.list_full[slot]);
-        if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status) ||
-            !mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status))
-          break;
+        if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status)) break;
+        if (p.key_mask && p.tdead) {
+          const uint32_t* dw = p.tdead + (size_t)m.b * p.tdead_words;
+          auto dead = [&](int j) { return (__ldg(dw + 1 + (j >> 5)) >> (j & 31)) & 1u; };
+          TileList& Lw = lists[slot];
+          if (p.mask_q && dead(m.t[0]) && (m.t[1] < 0 || dead(m.t[1]))) {
+            // Every row is a padding token (query-side mask): P is 0 on
+            // them, so their dq is 0 and no key tile is needed.
+            Lw.n = 0;
+          } else if (__ldg(dw) & 1u) {
+            // Drop key tiles whose 64 keys are all masked: exact when every
+            // row has a valid attended key (the flag word), as in the
+            // forward.
+            int n2 = 0;
+            for (int t = 0; t < Lw.n; ++t) {
+              if (dead(Lw.tile[t])) continue;
+              Lw.tile[n2] = Lw.tile[t];
+              Lw.mask[n2] = Lw.mask[t];
+              ++n2;
+            }
+            Lw.n = n2;
+          }
+          fence_proxy_async_smem();  // before the slot's next bulk copy
+        }
+        mbar_arrive_release(&bars.list_ready[slot]);
+        if (!mbar_wait(&bars.q_empty, (k & 1) ^ 1, &abort_flag, p.status)) break;
         const int row0 = m.bh * p.L;
         const int nh = m.t[1] >= 0 ? 2 : 1;
         mbar_expect_tx(&bars.q_full, 2u * nh * kTileBytes);
@@ -346,7 +372,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       const int slot = k & 1;
-      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
+      if (!mbar_wait(&bars.list_ready[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
       if (!item_sh[slot].w) break;
       const int n = lists[slot].n;
@@ -439,7 +465,7 @@ __global__ void __launch_bounds__(kThreads2, 2)
     uint32_t u = 0;
     for (int k = 0;; ++k) {
       const int slot = k & 1;
-      if (!mbar_wait(&bars.list_full[slot], (k >> 1) & 1, &abort_flag, p.status))
+      if (!mbar_wait(&bars.list_ready[slot], (k >> 1) & 1, &abort_flag, p.status))
         break;
       const int4 wi = item_sh[slot];
       if (!wi.w) break;
@@ -560,6 +586,10 @@ __global__ void __launch_bounds__(kThreads2, 2)
       tmem_ld32(tDQ + lane_off, q0);
       tmem_ld32(tDQ + 32 + lane_off, q1);
       tmem_ld_wait();
+      if (n == 0) {  // no tile accumulated: the rows' dq is 0
+#pragma unroll
+        for (int e = 0; e < 32; ++e) q0[e] = q1[e] = 0u;
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.dq_empty);
@@ -636,10 +666,12 @@ struct KvBars {
   uint64_t acc_full, acc_empty;
 };
 
-// kSplit: bf16 hi/lo split of the global key blocks' P^T and dS^T, for
-// lengths where they sum over enough query rows (>= 16K) for bf16 products
-// to cost accuracy.  A template flag keeps the low parts out of the shorter
-// lengths' register budget.
+// kSplit: bf16 hi/lo split of the global key blocks' P^T and dS^T, where
+// their gradients can grow large enough for bf16 products to cost accuracy:
+// lengths >= 16K (they sum over every query row), and calls with a key mask
+// (masked keys can concentrate many rows' probability on them).  A
+// template flag keeps the low parts out of the other calls' register
+// budget.
 // kDrop: seeded attention dropout (P^T kept times 1 / keep probability for
 // dV; dS^T = P^T (m dP^T - D)).
 // kWhole: the global key blocks run whole (every item's rows are final here).
@@ -733,6 +765,14 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.kgeo, it, e0, e1);
+        if (p.key_mask && p.tdead) {
+          // Key rows whose keys are all masked get probability 0 from every
+          // row when every row has a valid attended key (the flag word):
+          // their dK and dV are 0, so the item visits no query tile.
+          const uint32_t* dw = p.tdead + (size_t)it.b * p.tdead_words;
+          auto dead = [&](int j) { return (__ldg(dw + 1 + (j >> 5)) >> (j & 31)) & 1u; };
+          if ((__ldg(dw) & 1u) && dead(it.t[0]) && (it.t[1] < 0 || dead(it.t[1]))) e1 = e0;
+        }
         const uint32_t wfirst = e0 < e1 ? __ldg(walk + e0) : 0u;
         kwalk[ps] = make_int4(e0, e1, (int)wfirst, e0 + 1 < e1 ? (int)__ldg(walk + e0 + 1) : 0);
         const int row0 = it.bh * p.L;
@@ -1065,17 +1105,23 @@ __global__ void __launch_bounds__(kThreads1, 1)
         ++u;
       }
       if (!ok) break;
-      if (e1 == e0) continue;  // nothing accumulated (not planned)
-      if (!mbar_wait(&bars.acc_full, ai & 1, &abort_flag, p.status)) break;
-      ++ai;
-      tc_fence_after();
       uint32_t kx[32], vx[32];
-      tmem_ld32(tmem + kKvDK + hc * 32 + lane_off, kx);
-      tmem_ld32(tmem + kKvDV + hc * 32 + lane_off, vx);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.acc_empty);
+      if (e1 == e0) {
+        // No query tile visits these keys (none attends them, or all their
+        // keys are masked): their dK and dV are 0.
+#pragma unroll
+        for (int e = 0; e < 32; ++e) kx[e] = vx[e] = 0u;
+      } else {
+        if (!mbar_wait(&bars.acc_full, ai & 1, &abort_flag, p.status)) break;
+        ++ai;
+        tc_fence_after();
+        tmem_ld32(tmem + kKvDK + hc * 32 + lane_off, kx);
+        tmem_ld32(tmem + kKvDV + hc * 32 + lane_off, vx);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.acc_empty);
+      }
       if (rvalid) {
         if (kWhole || !it.global) {  // final rows (no chunk partials)
           store_grad_half(p, p.dk, krow, hc * 32, kx, p.scale);
@@ -1249,7 +1295,16 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     parts[nparts++] = {true, nglob, 0};
     if (g.n_mid > 0) parts[nparts++] = {false, g.n_mid, nglob};
   } else {
-    parts[nparts++] = {false, g.per_bh, 0};
+    // One launch.  Masked keys can concentrate the probability of many rows
+    // on the global blocks and raise their gradients as a long sequence
+    // does: the largest grows like sqrt(L) / block size (7.4 at L = 4096,
+    // block 32, with three quarters of the keys masked), and bf16 products
+    // cost ~1.7e-3 of it.  So with a key mask, from L = 2048 (block / 32)^2
+    // on, the launch is the split variant (the global key blocks' P^T and
+    // dS^T carry the bf16 low part).
+    const bool masked_split =
+        p.key_mask != nullptr && (long long)p.L * 1024 >= 2048LL * p.bs * p.bs;
+    parts[nparts++] = {masked_split, g.per_bh, 0};
   }
   for (int i = 0; i < nparts; ++i) {
     BwdArgs bk = ba;
@@ -1257,15 +1312,17 @@ cudaError_t launch_tc_bwd(const Problem& p, const TensorMaps& tm,
     bk.knloc = parts[i].per_bh;
     bk.kitems = p.B * p.H * parts[i].per_bh;
     bk.kctr = p.sched + 1 + i;  // sched[0]: dQ
-    // The split launch holds only chunked global items.
     const bool kwhole = g.nchunks == 1;
-    auto* kv_kernel =
-        parts[i].split ? (drop ? tc_dkdv_kernel<true, true, false>
-                               : tc_dkdv_kernel<true, false, false>)
-                       : (drop ? (kwhole ? tc_dkdv_kernel<false, true, true>
-                                         : tc_dkdv_kernel<false, true, false>)
-                               : (kwhole ? tc_dkdv_kernel<false, false, true>
-                                         : tc_dkdv_kernel<false, false, false>));
+    using KvKernel = void (*)(const BwdArgs, const CUtensorMap, const CUtensorMap,
+                              const CUtensorMap, const CUtensorMap);
+    // [split][dropout][whole]
+    static const KvKernel kv_kernels[2][2][2] = {
+        {{tc_dkdv_kernel<false, false, false>, tc_dkdv_kernel<false, false, true>},
+         {tc_dkdv_kernel<false, true, false>, tc_dkdv_kernel<false, true, true>}},
+        {{tc_dkdv_kernel<true, false, false>, tc_dkdv_kernel<true, false, true>},
+         {tc_dkdv_kernel<true, true, false>, tc_dkdv_kernel<true, true, true>}}};
+    const KvKernel kv_kernel =
+        kv_kernels[parts[i].split ? 1 : 0][drop ? 1 : 0][kwhole ? 1 : 0];
     e = cudaFuncSetAttribute(kv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_kv);
     if (e != cudaSuccess) return e;

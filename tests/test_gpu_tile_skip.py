@@ -15,7 +15,8 @@ import pytest
 import torch
 
 from block_sparse_long_bwd_b200 import synth
-from gpu_util import ATOL, assert_close, oracle_slice, run_gpu
+from gpu_util import (ATOL, assert_bf16_is_rounded_fp32, assert_close, oracle_slice,
+                      run_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,3 +62,79 @@ def test_skip_rule_per_batch(bs):
     res = run_gpu(cfg, inp, backward=False)
     assert res["status_fwd"] == 0
     _compare(cfg, inp, res)
+
+
+# ---- the backward: the same bitmap, in dQ's tile lists and dK/dV's items --
+
+
+def _compare_backward(cfg, inp, mask_queries):
+    """Forward outputs at the bf16 tolerance; gradients through their fp32
+    form (with few valid keys the global key blocks' exact gradients exceed
+    4, where bf16's own spacing is above 1e-2), the bf16 gradients of the
+    same kernels being those values rounded to nearest even."""
+    res = run_gpu(cfg, inp, mask_queries=mask_queries)
+    r32 = run_gpu(cfg, inp, mask_queries=mask_queries, grad_fp32=1)
+    for r in (res, r32):
+        assert r["status_fwd"] == 0 and r["status_bwd"] == 0
+    assert_bf16_is_rounded_fp32(res, r32)
+    tol = ATOL[cfg["dtype"]]
+    for b in range(cfg["B"]):
+        for h in range(cfg["H"]):
+            ora = oracle_slice(cfg, inp, res["table"], b, h,
+                               mask_queries=mask_queries)
+            assert_close(res, ora, b, h, tol, FWD)
+            assert_close(r32, ora, b, h, tol, ("dq", "dk", "dv"))
+    return res
+
+
+@pytest.mark.parametrize("bs", [32, 64, 128])
+@pytest.mark.parametrize("mq", [0, 1])
+def test_backward_skip_rule_per_batch(bs, mq):
+    """dQ drops key tiles whose keys are all masked (and, with the
+    query-side mask, whole items of padding rows); dK/dV writes zeros for
+    key items whose keys are all masked.  Same batches as the forward case:
+    batch 0 keeps every tile (keys 0..31 masked), batch 1 has 1024 valid
+    keys of 4096 (most items and whole global chunks empty), batch 2 a
+    masked run in the middle."""
+    L = 4096
+    cfg = dict(B=3, H=2, L=L, block_size=bs, d=64, r=3, dtype="bf16",
+               seed=72, mask=None, passes="fwd+bwd")
+    inp = synth.make_inputs(cfg)
+    km = np.ones((3, L), np.uint8)
+    km[0, :32] = 0
+    km[0, 1024:2048] = 0
+    km[1, 1024:] = 0
+    km[2, 1280:2560] = 0
+    inp["key_mask"] = torch.from_numpy(km)
+    res = _compare_backward(cfg, inp, mq)
+    # fully masked keys get exactly zero dK and dV (batch 1's tail)
+    assert bool((res["dk"][1, :, 1024:] == 0).all())
+    assert bool((res["dv"][1, :, 1024:] == 0).all())
+    if mq:  # and padding rows exactly zero dQ
+        assert bool((res["dq"][1, :, 1024:] == 0).all())
+
+
+def test_backward_skip_base_layer_shape():
+    """The BigBird-base shape (B 8, H 12, its tail mask) through fwd + bwd
+    with the query-side mask: whole global rows, skipped tiles on both
+    sides; every (b, h) slice against the oracle."""
+    cfg = dict(synth.WORKLOADS["base_fwd_l4096"])
+    cfg["passes"] = "fwd+bwd"
+    inp = synth.make_inputs(cfg)
+    _compare_backward(cfg, inp, 1)
+
+
+@pytest.mark.parametrize("L,bs", [(8192, 64), (1024, 32)])
+def test_backward_heavy_padding_without_query_mask(L, bs):
+    """Three quarters of the keys masked and the padding rows computed (no
+    query-side mask): their probability concentrates on the global blocks'
+    valid keys, whose gradients then grow like a long sequence's.  Block 64
+    at 8192 tokens takes the split dK/dV variant (the bf16 low part), block
+    32 at 1024 does not need it; both within the tolerance."""
+    cfg = dict(B=1, H=2, L=L, block_size=bs, d=64, r=3, dtype="bf16",
+               seed=73, mask=None, passes="fwd+bwd")
+    inp = synth.make_inputs(cfg)
+    km = np.zeros((1, L), np.uint8)
+    km[0, :L // 4] = 1
+    inp["key_mask"] = torch.from_numpy(km)
+    _compare_backward(cfg, inp, 0)

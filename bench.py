@@ -52,11 +52,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 NCU_TRAFFIC = {
     # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, one
     # launch each, captured on the sources these hashes describe)
-    "tc_fwd": (120679424 + 19203584, "b61b794bceb29db9", "tc_fwd.cu",
+    "tc_fwd": (120624128 + 17051904, "2ed3afd7e8d4b020", "tc_fwd.cu",
                "large_train_l4096"),
-    "tc_dq": (200576000 + 23244032, "42a1b4fe7e95eb80", "tc_bwd.cu",
+    "tc_dq": (200682496 + 24587008, "cd42c42c999abe14", "tc_bwd.cu",
               "large_train_l4096"),
-    "tc_dkdv": (178062080 + 42365952, "42a1b4fe7e95eb80", "tc_bwd.cu",
+    "tc_dkdv": (177972736 + 40992000, "cd42c42c999abe14", "tc_bwd.cu",
                 "large_train_l4096"),
 }
 

@@ -401,6 +401,19 @@ __global__ void __launch_bounds__(kThreads, 2)
           float mx;
           if (kb == ~0ull && hb == ~0ull && c > 0.f) {
             mx = max64(z) * c;
+          } else if (kMask && hb == ~0ull) {
+            // Every column attended, some keys masked (the finite offset):
+            // paired, each element rounded once as below.
+            const float2 c2 = make_float2(c, c);
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const float2 o = make_float2(((kb >> e) & 1ull) ? 0.f : mvl,
+                                           ((kb >> (e + 1)) & 1ull) ? 0.f : mvl);
+              const float2 r = fma2(make_float2(z[e], z[e + 1]), c2, o);
+              z[e] = r.x;
+              z[e + 1] = r.y;
+            }
+            mx = max64(z);
           } else {
             // Columns outside the attended blocks are absent (-inf, p = 0);
             // masked keys inside them get the finite offset.

@@ -158,10 +158,18 @@ __device__ __forceinline__ void dq_p_half(uint32_t (&s)[32], uint64_t kb, int co
     }
     return;
   }
+  // Some keys masked: their offset added, paired (each element rounded as
+  // in the form fmaf(s, c, nl2 + offset)).
+  const float2 c2 = make_float2(c, c);
+  const float nlm = nl2 + mvl;
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    const float off = ((kb >> (col0 + e)) & 1ull) ? 0.f : mvl;
-    s[e] = __float_as_uint(ex2(fmaf(__uint_as_float(s[e]), c, nl2 + off)));
+  for (int e = 0; e < 32; e += 2) {
+    const float2 b2 = make_float2(((kb >> (col0 + e)) & 1ull) ? nl2 : nlm,
+                                  ((kb >> (col0 + e + 1)) & 1ull) ? nl2 : nlm);
+    const float2 a =
+        fma2(make_float2(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), c2, b2);
+    s[e] = __float_as_uint(ex2(a.x));
+    s[e + 1] = __float_as_uint(ex2(a.y));
   }
 }
 

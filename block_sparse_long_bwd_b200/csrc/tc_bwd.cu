@@ -22,8 +22,11 @@
 //   dV += P^T dO and dK += dS^T Q (issued by the MMA warp) accumulate in
 //   TMEM.  One CTA per SM holds all 512 TMEM columns.  From kSplitMinL
 //   the global key blocks run in a launch of their own with a bf16 low part
-//   of P^T and dS^T.  Each key row is owned by exactly one item (or one
-//   chunk partial), so there are no atomics on data.
+//   of P^T and dS^T.  The loader hands each visited query tile's walk entry
+//   to the other warps through shared memory with the tile's stage, so it
+//   can leave tiles out per (b, h): with the query-side mask, query tiles
+//   whose tokens are all padding (P = 0).  Each key row is owned by exactly
+//   one item (or one chunk partial), so there are no atomics on data.
 // bwd_finish_kernel: sums the chunk partials of the global query rows (dQ)
 //   and of the global key blocks (dK, dV) in a fixed order.
 #include "dropout.cuh"
@@ -693,13 +696,14 @@ __global__ void __launch_bounds__(kThreads1, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ KvBars bars;
   __shared__ int4 kitem[2];  // (b, h, loc, 1) of the item in pair slot s; w = 0: no more items
-  // Walk of the item in pair slot s, as the loader read it: entries [x, y)
-  // of the head's walk area and the first two entries (so the other warps
-  // start the item without global loads).
-  __shared__ int4 kwalk[2];
+  // Item in pair slot s visits at least one query tile (published with it).
+  __shared__ int kwalk[2];
   // flat tile g at g % kTinfo: pair slot | kp_full parity << 1 | last tile
-  // of its item << 2, or kTinfoEnd
+  // of its item << 2, or kTinfoEnd; its walk entry (query tile | group
+  // mask << 16) and the entry of the item's next visited tile.  Written by
+  // the loader before the tile's qt_full arrive.
   __shared__ uint8_t tinfo[kTinfo];
+  __shared__ uint32_t went[kTinfo], wnext[kTinfo];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -773,16 +777,31 @@ __global__ void __launch_bounds__(kThreads1, 1)
         const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
         int e0, e1;
         walk_range(p, ba.kgeo, it, e0, e1);
-        if (p.key_mask && p.tdead) {
-          // Key rows whose keys are all masked get probability 0 from every
-          // row when every row has a valid attended key (the flag word):
-          // their dK and dV are 0, so the item visits no query tile.
-          const uint32_t* dw = p.tdead + (size_t)it.b * p.tdead_words;
-          auto dead = [&](int j) { return (__ldg(dw + 1 + (j >> 5)) >> (j & 31)) & 1u; };
-          if ((__ldg(dw) & 1u) && dead(it.t[0]) && (it.t[1] < 0 || dead(it.t[1]))) e1 = e0;
-        }
-        const uint32_t wfirst = e0 < e1 ? __ldg(walk + e0) : 0u;
-        kwalk[ps] = make_int4(e0, e1, (int)wfirst, e0 + 1 < e1 ? (int)__ldg(walk + e0 + 1) : 0);
+        const bool tdead = p.key_mask && p.tdead;
+        const uint32_t* dw = tdead ? p.tdead + (size_t)it.b * p.tdead_words : nullptr;
+        auto dead = [&](int j) { return (__ldg(dw + 1 + (j >> 5)) >> (j & 31)) & 1u; };
+        // Key rows whose keys are all masked get probability 0 from every
+        // row when every row has a valid attended key (the flag word): their
+        // dK and dV are 0, so the item visits no query tile.
+        if (tdead && (__ldg(dw) & 1u) && dead(it.t[0]) && (it.t[1] < 0 || dead(it.t[1])))
+          e1 = e0;
+        // With the query-side mask, padding rows pass no gradient (P = 0):
+        // query tiles whose tokens are all padding are left out of the walk.
+        const bool qskip = tdead && p.mask_q;
+        int e = e0;  // next walk entry to read
+        auto next_live = [&](uint32_t& ent) -> bool {
+          for (; e < e1; ++e) {
+            ent = __ldg(walk + e);
+            if (!qskip || !dead((int)(ent & 0xFFFFu))) {
+              ++e;
+              return true;
+            }
+          }
+          return false;
+        };
+        uint32_t ent = 0u;
+        bool have = next_live(ent);
+        kwalk[ps] = have ? 1 : 0;
         const int row0 = it.bh * p.L;
         const int nh = it.t[1] >= 0 ? 2 : 1;
         uint8_t* kv = KV + ps * 4 * kTileBytes;
@@ -794,11 +813,13 @@ __global__ void __launch_bounds__(kThreads1, 1)
         }
         kp_issued[ps] = 1;
         kp_par[ps] = (k >> 1) & 1;
-        if (e1 == e0) mma_commit(&bars.kp_empty[ps]);  // no MMA reads this pair
-        uint32_t nxt = wfirst;  // loaded a tile ahead
-        for (int e = e0; e < e1; ++e) {
-          const int i = (int)(nxt & 0xFFFFu);  // query tile
-          if (e + 1 < e1) nxt = __ldg(walk + e + 1);
+        if (!have) mma_commit(&bars.kp_empty[ps]);  // no MMA reads this pair
+        while (have) {
+          const int i = (int)(ent & 0xFFFFu);  // query tile
+          // The next visited entry (read while the stage is awaited): this
+          // tile is the item's last when there is none.
+          uint32_t nent = 0u;
+          const bool nhave = next_live(nent);
           const uint32_t g = gq;
           const uint32_t st = g % kKvQStages;
           if (!mbar_wait(&bars.qt_empty[st], ((g / kKvQStages) & 1) ^ 1, &abort_flag,
@@ -806,7 +827,9 @@ __global__ void __launch_bounds__(kThreads1, 1)
             ok = false;
             break;
           }
-          tinfo[g % kTinfo] = (uint8_t)(ps | (((k >> 1) & 1) << 1) | (e == e1 - 1 ? 4 : 0));
+          tinfo[g % kTinfo] = (uint8_t)(ps | (((k >> 1) & 1) << 1) | (nhave ? 0 : 4));
+          went[g % kTinfo] = ent;
+          wnext[g % kTinfo] = nent;
           uint8_t* q = QT + st * kQStageBytes;
           mbar_expect_tx(&bars.qt_full[st], 2 * kTileBytes + 512);
           const int y = row0 + i * kTile;
@@ -815,6 +838,8 @@ __global__ void __launch_bounds__(kThreads1, 1)
           bulk_load(q + 2 * kTileBytes, ba.NL + y, 256, &bars.qt_full[st]);
           bulk_load(q + 2 * kTileBytes + 256, ba.D + y, 256, &bars.qt_full[st]);
           ++gq;
+          ent = nent;
+          have = nhave;
         }
         if (!ok) break;
       }
@@ -890,11 +915,12 @@ __global__ void __launch_bounds__(kThreads1, 1)
       const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
-      const int4 kw = kwalk[ps];
-      const int nwalk = kw.y - kw.x;
+      const bool has = kwalk[ps] != 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem, kwalk read
-      for (int t = 0; t < nwalk; ++t) {
+      // The item's tiles, up to the one marked last (its P^T / dS^T arrive
+      // after the softmax observed the loader's tile information).
+      for (int t = 0; has; ++t) {
         const uint32_t g = u;
         const int b = g & 1;
         const uint32_t st = g % kKvQStages;
@@ -904,6 +930,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
           break;
         }
         tc_fence_after();
+        const bool last = (tinfo[g % kTinfo] & 4) != 0;
         if (lane == 0) {
           const uint32_t qaddr = smem_u32(QT + st * kQStageBytes);
           const uint32_t gaddr = qaddr + kTileBytes;
@@ -932,12 +959,13 @@ __global__ void __launch_bounds__(kThreads1, 1)
           }
           mma_commit(&bars.g_done[b]);
           mma_commit(&bars.qt_empty[st]);
-          if (t == nwalk - 1) mma_commit(&bars.acc_full);
+          if (last) mma_commit(&bars.acc_full);
         }
         __syncwarp();
         ++u;
+        if (last) break;
       }
-      if (nwalk > 0) ++ai;
+      if (has) ++ai;
     }
   } else {
     // Softmax warps 3-10: two per TMEM lane quarter (one per SM sub-
@@ -959,11 +987,9 @@ __global__ void __launch_bounds__(kThreads1, 1)
       const int4 wi = kitem[ps];
       if (!wi.w) break;
       const ItemMeta it = item_meta_at(ba.kgeo, wi.x, wi.y, p.H, wi.z);
-      const int4 kw = kwalk[ps];
+      const bool has = kwalk[ps] != 0;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.kp_empty[ps]);  // kitem, kwalk read
-      const uint32_t* walk = p.kplan + (size_t)it.h * p.kcap;
-      const int e0 = kw.x, e1 = kw.y;
       const bool rvalid = (it.gvalid >> quarter) & 1;
       const size_t ktok = (size_t)(rvalid ? it.t[half] : 0) * kTile + r64;
       const size_t krow = (size_t)it.bh * p.L + ktok;
@@ -972,28 +998,42 @@ __global__ void __launch_bounds__(kThreads1, 1)
         off = p.key_mask[(size_t)it.b * p.L + ktok] ? 0.f : mvl;
       const bool split = kSplit && it.global;  // bf16 low parts too
       bool ok = true;
-      // Walk entries are loaded two tiles ahead; with stored dropout
-      // decisions, lane l loads the word of query token t0 + l against the
-      // warp's 32 keys one tile ahead (transposed below).
+      // With stored dropout decisions, lane l loads the word of query token
+      // t0 + l against the warp's 32 keys (transposed below).
       auto keep_word = [&](uint32_t ent) -> uint32_t {
         if (!(((int)(ent >> 16) >> (gshift + hc)) & 1)) return 0u;
         return __ldg(keep_ptr(p, it.bh, it.h, (int)(ent & 0xFFFFu) * kTile + hc * 32 + lane,
                               (int)(ktok & ~(size_t)31)));
       };
-      uint32_t cur = (uint32_t)kw.z, nxt = (uint32_t)kw.w;
-      uint32_t kwn = (kDrop && p.keep_bits && e0 < e1) ? keep_word(cur) : 0u;
-      for (int e = e0; e < e1; ++e) {
-        const uint32_t ent = cur;
-        cur = nxt;
-        if (e + 2 < e1) nxt = __ldg(walk + e + 2);
-        const int mask = (int)(ent >> 16);
-        const int qtile = (int)(ent & 0xFFFFu);
-        const uint32_t kw = kwn;
-        if (kDrop && p.keep_bits && e + 1 < e1) kwn = keep_word(cur);
+      // The item's tiles as the loader published them, up to the one
+      // marked last.  With stored dropout decisions, each tile's keep word
+      // is loaded one tile ahead (from the next entry published with the
+      // tile).
+      const bool keep_ahead = kDrop && p.keep_bits;
+      uint32_t kwn = 0u;
+      if (keep_ahead && has) {
+        if (!mbar_wait(&bars.qt_full[u % kKvQStages], (u / kKvQStages) & 1, &abort_flag,
+                       p.status))
+          break;
+        kwn = keep_word(went[u % kTinfo]);
+      }
+      for (bool more = has; more;) {
         const uint32_t g = u;
         const int b = g & 1;
         const int sb = kSplit ? 0 : b;  // S^T / dP^T buffer (as the score warp)
         const uint32_t st = g % kKvQStages;
+        // The tile's walk entry and last mark were written before its
+        // stage's qt_full arrive (its NL / D arrive by bulk copy there too).
+        if (!mbar_wait(&bars.qt_full[st], (g / kKvQStages) & 1, &abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint32_t ent = went[g % kTinfo];
+        more = (tinfo[g % kTinfo] & 4) == 0;
+        const int mask = (int)(ent >> 16);
+        const int qtile = (int)(ent & 0xFFFFu);
+        const uint32_t kw = kwn;
+        if (keep_ahead && more) kwn = keep_word(wnext[g % kTinfo]);
         // Do query rows of this warp's column half attend this key group?
         const bool att = (mask >> (gshift + hc)) & 1;
         if (!mbar_wait(&bars.s_full[sb], kSplit ? (g & 1) : ((g >> 1) & 1), &abort_flag,
@@ -1002,12 +1042,6 @@ __global__ void __launch_bounds__(kThreads1, 1)
           break;
         }
         tc_fence_after();
-        // The stage's NL / D arrived by bulk copy: observe its barrier too.
-        if (att && !mbar_wait(&bars.qt_full[st], (g / kKvQStages) & 1, &abort_flag,
-                              p.status)) {
-          ok = false;
-          break;
-        }
         const float* NLs =
             reinterpret_cast<const float*>(QT + st * kQStageBytes + 2 * kTileBytes);
         const float* Ds = NLs + 64;
@@ -1114,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
       }
       if (!ok) break;
       uint32_t kx[32], vx[32];
-      if (e1 == e0) {
+      if (!has) {
         // No query tile visits these keys (none attends them, or all their
         // keys are masked): their dK and dV are 0.
 #pragma unroll

@@ -8,7 +8,10 @@ result is the oracle's.  Global chunks can lose all their tiles (empty
 partials).  Cases: the BigBird-base workload with the query-side mask on
 every (b, h) slice; a batch whose first 32 keys are masked (skipping must
 stay off there) beside one that skips; short valid lengths that empty
-whole chunks; block sizes 32 and 128."""
+whole chunks; block sizes 32 and 128.  The backward uses the same bitmap:
+dQ drops the key tiles, dK/dV writes zeros for key items whose keys are all
+masked, and with the query-side mask dQ skips items of padding rows and
+dK/dV's walks leave out query tiles of padding rows (their P is 0)."""
 
 import numpy as np
 import pytest
@@ -138,3 +141,50 @@ def test_backward_heavy_padding_without_query_mask(L, bs):
     km[0, :L // 4] = 1
     inp["key_mask"] = torch.from_numpy(km)
     _compare_backward(cfg, inp, 0)
+
+
+def test_backward_query_skip_long_chunked():
+    """16384 tokens with the query-side mask and a tail of padding: the
+    global key blocks run in their own split launch on 8-tile chunks of
+    query tiles, and the chunks that lie wholly in the padding lose every
+    query tile (zero partials merged by the finish launch); the middle key
+    items drop their padded query tiles.  Every slice against the oracle."""
+    L = 16384
+    cfg = dict(B=2, H=1, L=L, block_size=64, d=64, r=3, dtype="bf16",
+               seed=74, mask=None, passes="fwd+bwd")
+    inp = synth.make_inputs(cfg)
+    km = np.ones((2, L), np.uint8)
+    km[0, 5000:] = 0          # 11384 padding tokens (tiles 79..255 dead)
+    km[1, 9000:12288] = 0     # a padded run inside the sequence
+    inp["key_mask"] = torch.from_numpy(km)
+    res = _compare_backward(cfg, inp, 1)
+    assert bool((res["dq"][0, :, 5000:] == 0).all())
+
+
+def test_backward_query_skip_with_stored_dropout():
+    """Dropout with the forward's decisions stored, together with the
+    query-side mask: the dK/dV softmax warps load each visited tile's keep
+    words (one tile ahead when its entry is already published), over walks
+    with padded query tiles left out."""
+    L = 4096
+    cfg = dict(B=2, H=2, L=L, block_size=64, d=64, r=3, dtype="bf16",
+               seed=75, mask=None, passes="fwd+bwd")
+    inp = synth.make_inputs(cfg)
+    km = np.ones((2, L), np.uint8)
+    km[0, 2600:] = 0
+    km[1, 700:1900] = 0
+    inp["key_mask"] = torch.from_numpy(km)
+    seed = 0x1234ABCD5678EF01
+    res = run_gpu(cfg, inp, mask_queries=1, dropout=0.1, dropout_seed=seed)
+    redrawn = run_gpu(cfg, inp, mask_queries=1, dropout=0.1,
+                      dropout_seed=seed, keep_dropout_bits=False)
+    for r in (res, redrawn):
+        assert r["status_fwd"] == 0 and r["status_bwd"] == 0
+    for n in ("out", "lse", "dq", "dk", "dv"):
+        assert torch.equal(res[n], redrawn[n]), n
+    tol = ATOL[cfg["dtype"]]
+    for b in range(cfg["B"]):
+        for h in range(cfg["H"]):
+            ora = oracle_slice(cfg, inp, res["table"], b, h, dropout=0.1,
+                               dropout_seed=seed, mask_queries=1)
+            assert_close(res, ora, b, h, tol, ("out", "lse", "dq", "dk", "dv"))

@@ -521,6 +521,8 @@ __global__ void __launch_bounds__(kThreads2, 2)
         const int m2 = (L.mask[t] >> gshift) & 3;  // attended column halves
         const uint64_t dbs = dbn;
         if (kDrop && p.keep_bits && t + 1 < n) dbn = keep_words(t + 1);
+        // Valid keys of the tile (loaded while the scores are computed).
+        const uint64_t kb = (kMask && m2) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
         if (!mbar_wait(&bars.s_full, u & 1, &abort_flag, p.status)) {
           ok = false;
           break;
@@ -537,7 +539,6 @@ __global__ void __launch_bounds__(kThreads2, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_free);
-        const uint64_t kb = (kMask && m2) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
         const uint64_t db = (kDrop && m2)
                                 ? (p.keep_bits ? dbs : keep_row64(p, im.b, im.h, tq, L.tile[t]))
                                 : 0ull;

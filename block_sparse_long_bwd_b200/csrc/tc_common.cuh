@@ -443,22 +443,15 @@ struct KeyWalk {
   }
 };
 
-// Validity bitmap of the 64 keys of key tile j (bit k set = attend).
+// Validity bitmap of the 64 keys of key tile j (bit k set = attend): one
+// mask byte per lane and half, gathered by two ballots.  All 32 lanes of the
+// warp must call it.
 __device__ __forceinline__ uint64_t key_bits(const Problem& p, int b, int j) {
-  const uint4* m4 = reinterpret_cast<const uint4*>(
-      p.key_mask + (size_t)b * p.L + (size_t)j * kTile);
-  uint64_t bits = 0;
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint4 w = __ldg(m4 + c);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-#pragma unroll
-      for (int by = 0; by < 4; ++by)
-        if ((ws[e] >> (8 * by)) & 0xFFu) bits |= 1ull << (16 * c + 4 * e + by);
-  }
-  return bits;
+  const uint8_t* m = p.key_mask + (size_t)b * p.L + (size_t)j * kTile;
+  const int lane = threadIdx.x & 31;
+  const uint32_t lo = __ballot_sync(0xffffffffu, __ldg(m + lane) != 0);
+  const uint32_t hi = __ballot_sync(0xffffffffu, __ldg(m + 32 + lane) != 0);
+  return ((uint64_t)hi << 32) | lo;
 }
 
 // Column-validity bitmap of a tile from its two mask bits for one group

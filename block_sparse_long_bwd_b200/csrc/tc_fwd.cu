@@ -367,6 +367,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         // (worked out while the scores are still being computed).
         int ks0 = -1, ks1 = -1;
         if (keep_out && att) keep_slots64(p, im.h, kr, L.tile[t], m2, ks0, ks1);
+        // Valid keys of the tile (loaded while the scores are computed).
+        const uint64_t kb = (kMask && att) ? key_bits(p, im.b, L.tile[t]) : ~0ull;
         if (!mbar_wait(&bars.s_full[b2], par, &abort_flag, p.status)) {
           ok = false;
           break;
@@ -396,7 +398,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
         if (att) {
-          const uint64_t kb = kMask ? key_bits(p, im.b, L.tile[t]) : ~0ull;
           const uint64_t hb = half_bits(m2);
           float mx;
           if (kb == ~0ull && hb == ~0ull && c > 0.f) {

@@ -68,12 +68,26 @@ __device__ __forceinline__ float max64(const float* z) {
   return fmax3(a, b, fmaxf(n[6], n[7]));
 }
 
+// Maximum of 32 values with three-input max: 16 instructions, depth 4.
+__device__ __forceinline__ float max32(const float* z) {
+  float m[11];
+#pragma unroll
+  for (int i = 0; i < 10; ++i) m[i] = fmax3(z[3 * i], z[3 * i + 1], z[3 * i + 2]);
+  m[10] = fmaxf(z[30], z[31]);
+  const float a = fmax3(m[0], m[1], m[2]), b = fmax3(m[3], m[4], m[5]),
+              d = fmax3(m[6], m[7], m[8]);
+  return fmax3(fmax3(a, b, d), m[9], m[10]);
+}
+
 // kDrop: seeded attention dropout on the probabilities that enter P V (the
 // row sums, hence the lse, stay those of the undropped softmax).
 // kWhole: global items run whole (one chunk), so every row of every item is
 // final in this kernel; else global items leave chunk partials.
 // kMask: a key mask is given (else every key is attended).
-template <bool kDrop, bool kWhole, bool kMask>
+// kHalf: block size 32, where a row group often attends only one 32-column
+// half of a key tile: then only that half's scores are loaded and
+// exponentiated (the other half's P is 0).
+template <bool kDrop, bool kWhole, bool kMask, bool kHalf>
 __global__ void __launch_bounds__(kThreads, 2)
     tc_fwd_kernel(const __grid_constant__ PairArgs a,
                   const __grid_constant__ CUtensorMap tmQ,
@@ -374,8 +388,18 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         tc_fence_after();
+        // One attended half (block 32): its scores in z[0, 32), written to
+        // P half h0.
+        const bool one = kHalf && m2 != 3;
+        const int h0 = one ? (m2 >> 1) : 0;
         float z[64];
-        if (att) {
+        if (att && one) {
+          uint32_t s0[32];
+          tmem_ld32(tmem + kColS + b2 * 64 + h0 * 32 + lane_off, s0);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) z[e] = __uint_as_float(s0[e]);
+        } else if (att) {
           uint32_t s0[32], s1[32];
           tmem_ld32(tmem + kColS + b2 * 64 + lane_off, s0);
           tmem_ld32(tmem + kColS + b2 * 64 + 32 + lane_off, s1);
@@ -398,34 +422,55 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_fence_after();
         const uint32_t tP = tmem + kColP + b2 * 32 + lane_off;
         if (att) {
-          const uint64_t hb = half_bits(m2);
           float mx;
-          if (kb == ~0ull && hb == ~0ull && c > 0.f) {
-            mx = max64(z) * c;
-          } else if (kMask && hb == ~0ull) {
-            // Every column attended, some keys masked (the finite offset):
-            // paired, each element rounded once as below.
-            const float2 c2 = make_float2(c, c);
+          bool scaled;
+          if (one) {
+            // One attended half: its keys' offsets (if any masked), paired.
+            const uint32_t kbh = (uint32_t)(kb >> (32 * h0));
+            scaled = !(kbh == ~0u && c > 0.f);
+            if (!scaled) {
+              mx = max32(z) * c;
+            } else {
+              const float2 c2 = make_float2(c, c);
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-              const float2 o = make_float2(((kb >> e) & 1ull) ? 0.f : mvl,
-                                           ((kb >> (e + 1)) & 1ull) ? 0.f : mvl);
-              const float2 r = fma2(make_float2(z[e], z[e + 1]), c2, o);
-              z[e] = r.x;
-              z[e + 1] = r.y;
+              for (int e = 0; e < 32; e += 2) {
+                const float2 o = make_float2(((kbh >> e) & 1u) ? 0.f : mvl,
+                                             ((kbh >> (e + 1)) & 1u) ? 0.f : mvl);
+                const float2 r = fma2(make_float2(z[e], z[e + 1]), c2, o);
+                z[e] = r.x;
+                z[e + 1] = r.y;
+              }
+              mx = max32(z);
             }
-            mx = max64(z);
           } else {
-            // Columns outside the attended blocks are absent (-inf, p = 0);
-            // masked keys inside them get the finite offset.
+            const uint64_t hb = half_bits(m2);
+            if (kb == ~0ull && hb == ~0ull && c > 0.f) {
+              mx = max64(z) * c;
+            } else if (kMask && hb == ~0ull) {
+              // Every column attended, some keys masked (the finite offset):
+              // paired, each element rounded once as below.
+              const float2 c2 = make_float2(c, c);
 #pragma unroll
-            for (int e = 0; e < 64; ++e)
-              z[e] = ((hb >> e) & 1ull)
-                         ? fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl)
-                         : -INFINITY;
-            mx = max64(z);
+              for (int e = 0; e < 64; e += 2) {
+                const float2 o = make_float2(((kb >> e) & 1ull) ? 0.f : mvl,
+                                             ((kb >> (e + 1)) & 1ull) ? 0.f : mvl);
+                const float2 r = fma2(make_float2(z[e], z[e + 1]), c2, o);
+                z[e] = r.x;
+                z[e + 1] = r.y;
+              }
+              mx = max64(z);
+            } else {
+              // Columns outside the attended blocks are absent (-inf, p = 0);
+              // masked keys inside them get the finite offset.
+#pragma unroll
+              for (int e = 0; e < 64; ++e)
+                z[e] = ((hb >> e) & 1ull)
+                           ? fmaf(z[e], c, ((kb >> e) & 1ull) ? 0.f : mvl)
+                           : -INFINITY;
+              mx = max64(z);
+            }
+            scaled = !(kb == ~0ull && hb == ~0ull && c > 0.f);
           }
-          const bool scaled = !(kb == ~0ull && hb == ~0ull && c > 0.f);
           // Lazy running max: move it only when the row max exceeds it by
           // more than the threshold (or on the row's first attended tile).
           const bool first = (m == -INFINITY);
@@ -469,6 +514,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             keep_store64(p, im.bh, tq, L.tile[t], ks0, ks1, db);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
+            // z half hh goes to P half h0 + hh (one attended half: hh = 0
+            // only).
+            if (one && hh == 1) break;
             uint32_t Ph[16];
 #pragma unroll
             for (int e = 0; e < 32; e += 2) {
@@ -477,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               sum2[(e >> 1) & 3] = add2(sum2[(e >> 1) & 3], pp);
               if (kDrop) {
                 // Kept probabilities times 1 / keep probability, dropped 0.
-                const uint32_t dw = (uint32_t)(db >> (32 * hh));
+                const uint32_t dw = (uint32_t)(db >> (32 * (h0 + hh)));
                 const float2 mk = make_float2(keep_factor(dw, e, p.drop_scale),
                                               keep_factor(dw, e + 1, p.drop_scale));
                 const float2 pk = mul2(pp, mk);
@@ -486,7 +534,13 @@ __global__ void __launch_bounds__(kThreads, 2)
                 Ph[e >> 1] = pack_bf16(pp.x, pp.y);
               }
             }
-            tmem_st16(tP + 16 * hh, Ph);
+            tmem_st16(tP + 16 * (h0 + hh), Ph);
+          }
+          if (one) {
+            uint32_t Z[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) Z[e] = 0u;
+            tmem_st16(tP + 16 * (1 - h0), Z);
           }
           const float2 s01 = add2(sum2[0], sum2[1]), s23 = add2(sum2[2], sum2[3]);
           const float2 s4 = add2(s01, s23);
@@ -656,13 +710,18 @@ cudaError_t launch_tc_fwd(const Problem& p, const TensorMaps& tm,
   const bool masked = p.key_mask != nullptr;
   using Kernel = void (*)(const PairArgs, const CUtensorMap, const CUtensorMap,
                           const CUtensorMap, const CUtensorMap);
-  // [dropout][whole][mask]
-  static const Kernel kernels[2][2][2] = {
-      {{tc_fwd_kernel<false, false, false>, tc_fwd_kernel<false, false, true>},
-       {tc_fwd_kernel<false, true, false>, tc_fwd_kernel<false, true, true>}},
-      {{tc_fwd_kernel<true, false, false>, tc_fwd_kernel<true, false, true>},
-       {tc_fwd_kernel<true, true, false>, tc_fwd_kernel<true, true, true>}}};
-  const Kernel kernel = kernels[p.drop_thr ? 1 : 0][whole ? 1 : 0][masked ? 1 : 0];
+  // [dropout][whole][mask][block 32]
+  static const Kernel kernels[2][2][2][2] = {
+      {{{tc_fwd_kernel<false, false, false, false>, tc_fwd_kernel<false, false, false, true>},
+        {tc_fwd_kernel<false, false, true, false>, tc_fwd_kernel<false, false, true, true>}},
+       {{tc_fwd_kernel<false, true, false, false>, tc_fwd_kernel<false, true, false, true>},
+        {tc_fwd_kernel<false, true, true, false>, tc_fwd_kernel<false, true, true, true>}}},
+      {{{tc_fwd_kernel<true, false, false, false>, tc_fwd_kernel<true, false, false, true>},
+        {tc_fwd_kernel<true, false, true, false>, tc_fwd_kernel<true, false, true, true>}},
+       {{tc_fwd_kernel<true, true, false, false>, tc_fwd_kernel<true, true, false, true>},
+        {tc_fwd_kernel<true, true, true, false>, tc_fwd_kernel<true, true, true, true>}}}};
+  const Kernel kernel = kernels[p.drop_thr ? 1 : 0][whole ? 1 : 0][masked ? 1 : 0]
+                               [p.bs == 32 ? 1 : 0];
   cudaError_t e = cudaFuncSetAttribute(
       kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

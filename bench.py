@@ -52,11 +52,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 NCU_TRAFFIC = {
     # profiles/tc_kernels_large_train_l4096.md (BigBird-large step, one
     # launch each, captured on the sources these hashes describe)
-    "tc_fwd": (119720704 + 17426944, "becc424fb000fcd8", "tc_fwd.cu",
+    "tc_fwd": (120852736 + 16990208, "e1206fd0b08f0603", "tc_fwd.cu",
                "large_train_l4096"),
-    "tc_dq": (200686336 + 24174336, "03a3188d085a68e2", "tc_bwd.cu",
+    "tc_dq": (200619264 + 23349248, "03a3188d085a68e2", "tc_bwd.cu",
               "large_train_l4096"),
-    "tc_dkdv": (177508608 + 43217408, "03a3188d085a68e2", "tc_bwd.cu",
+    "tc_dkdv": (178125568 + 40513792, "03a3188d085a68e2", "tc_bwd.cu",
                 "large_train_l4096"),
 }
 

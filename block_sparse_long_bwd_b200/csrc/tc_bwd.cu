@@ -983,7 +983,7 @@ __global__ void __launch_bounds__(kThreads1, 1)
     uint32_t u = 0, ai = 0;
     for (int k = 0;; ++k) {
       const int ps = k & 1;
-      // The item of this round: published with its K / V pair (kp_full).
+      // This iteration's item: published with its K / V pair (kp_full).
       if (!mbar_wait(&bars.kp_full[ps], (k >> 1) & 1, &abort_flag, p.status)) break;
       const int4 wi = kitem[ps];
       if (!wi.w) break;

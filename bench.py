@@ -54,9 +54,9 @@ NCU_TRAFFIC = {
     # launch each, captured on the sources these hashes describe)
     "tc_fwd": (120852736 + 16990208, "e1206fd0b08f0603", "tc_fwd.cu",
                "large_train_l4096"),
-    "tc_dq": (200619264 + 23349248, "0803a3f6ef836ebe", "tc_bwd.cu",
+    "tc_dq": (200619264 + 23349248, "9cad32704d22b2fb", "tc_bwd.cu",
               "large_train_l4096"),
-    "tc_dkdv": (178125568 + 40513792, "0803a3f6ef836ebe", "tc_bwd.cu",
+    "tc_dkdv": (178125568 + 40513792, "9cad32704d22b2fb", "tc_bwd.cu",
                 "large_train_l4096"),
 }
 

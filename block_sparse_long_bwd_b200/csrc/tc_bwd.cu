@@ -669,7 +669,7 @@ constexpr uint32_t kKvPL = kKvS + 64, kKvDSL = kKvDP + 64;
 struct KvBars {
   // K / V pair of item k in slot k & 1: kp_full = landed (and kitem[] of the
   // slot published); kp_empty = its last S^T / dP^T MMAs completed and the
-  // MMA warp and the four softmax warps have read kitem[].
+  // MMA warp and the eight softmax warps have read kitem[].
   uint64_t kp_full[2], kp_empty[2];
   uint64_t qt_full[kKvQStages], qt_empty[kKvQStages];
   // per tile buffer b: S^T / dP^T computed; read by the softmax; P^T / dS^T
